@@ -1,0 +1,58 @@
+/* Declarations of the CPU oracle (test infrastructure only; see dq_oracle.cpp).
+ * This header belongs to the oracle alone: the CUDA library neither includes
+ * it nor shares any of its constants. */
+#ifndef DQ_ORACLE_H
+#define DQ_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element storage types of floating-point inputs */
+enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
+/* output code containers */
+enum { ORACLE_Y_INT8 = 0, ORACLE_Y_INT4X2 = 1, ORACLE_Y_INT32 = 2 };
+/* quantization mode */
+enum { ORACLE_SYMMETRIC = 0, ORACLE_ASYMMETRIC = 1 };
+/* status */
+enum {
+  ORACLE_OK = 0,
+  ORACLE_ERR_SHAPE = -1,
+  ORACLE_ERR_DTYPE = -2,
+  ORACLE_ERR_ARGUMENT = -3,
+  ORACLE_ERR_GROUP_INDEX = -4
+};
+
+/* Per-token dynamic quantization (aclnnDynamicQuantV2, Formula).
+ * x: [rows, cols] row-major; smooth: NULL, [cols] or [num_groups, cols];
+ * group_index: NULL or [num_groups] cumulative end rows; y: int8 [rows, cols],
+ * packed uint8 [rows, cols/2] or uint32 [rows, cols/8]; scale: [rows];
+ * offset: [rows] (asymmetric only, else may be NULL). */
+int oracle_dynamic_quant(const void* x, int x_dtype, int64_t rows, int64_t cols,
+                         const void* smooth, int smooth_dtype,
+                         const int32_t* group_index, int32_t num_groups,
+                         int mode, int y_dtype,
+                         void* y, float* scale, float* offset);
+
+/* AdaLayerNorm prologue (aclnnAdaLayerNormQuant, Formula steps 1-3): writes the
+ * fp32 value that is quantized, plus per-row mean and sqrt(var+eps). */
+int oracle_ada_layernorm_pre(const void* x, int x_dtype, int64_t batch, int64_t seq, int64_t hidden,
+                             const void* ada_scale, const void* ada_shift,
+                             const void* weight, const void* bias, const void* smooth,
+                             int param_dtype, float epsilon,
+                             float* y, float* mean_out, float* std_out);
+
+/* Fused AdaLayerNormQuant (aclnnAdaLayerNormQuant, Formula steps 1-5). */
+int oracle_ada_layernorm_quant(const void* x, int x_dtype, int64_t batch, int64_t seq, int64_t hidden,
+                               const void* ada_scale, const void* ada_shift,
+                               const void* weight, const void* bias, const void* smooth,
+                               int param_dtype, float epsilon,
+                               int8_t* out, float* quant_scale);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_ORACLE_H */
