@@ -1,0 +1,573 @@
+#!/usr/bin/env python3
+"""Throughput benchmark of the B200 per-token dynamic quantization path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--graph]
+
+One step = one call of the hot path over one batch of the workload (default:
+symmetric INT8 with fp32 smooth scales, bf16 x [8192, 4096], the size the
+headline metric is quoted on). The metric is GB/s of algorithmic HBM traffic
+(x read + codes and scales written + side tables read), with rows/s and the
+fraction of the measured HBM copy bandwidth alongside.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+device synchronize on both sides, timed with CUDA events on the launching
+stream; the max over ranks is reported. Consecutive steps rotate over several
+input/output buffer sets whose total exceeds the 126 MB L2, so no step reads
+data the previous one left in L2. SM clocks and throttle reasons are sampled
+through NVML during the timed region.
+
+Multi-GPU (torchrun, one process per GPU): rows are independent, so each rank
+quantizes its own full batch with no collective on the data path (weak
+scaling); only the timing uses a MAX all-reduce.
+
+--impl reference times the CPU oracle (the plain sequential implementation of
+the same formulas) on the same metric, on the host cores of rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "sym_int8_smooth_bf16_8192x4096"
+METRIC = "DynamicQuant GB/s and % of B200 HBM roofline (rows/s at 8192x4096 bf16)"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- helpers
+
+def algorithmic_bytes(wl) -> int:
+    """HBM bytes one call must move: x read, codes + per-row floats written, side tables read."""
+    t = wl.tensors
+    x = t["x"]
+    rows, cols = wl.rows, wl.cols
+    total = x.numel() * x.element_size()
+    if wl.kind == "dynamic_quant":
+        code_bytes = rows * cols if wl.y_dtype == "int8" else rows * cols // 2
+        per_row = 4 * (2 if wl.mode == "asymmetric" else 1)
+        total += code_bytes + rows * per_row
+        for k in ("smooth", "group_index"):
+            if t.get(k) is not None:
+                total += t[k].numel() * t[k].element_size()
+    else:
+        total += rows * cols + rows * 4
+        for k in ("ada_scale", "ada_shift", "weight", "bias", "smooth"):
+            if t.get(k) is not None:
+                total += t[k].numel() * t[k].element_size()
+    return int(total)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "token_dynamic_quantization_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"ncu_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+class ClockSampler:
+    """NVML sampling of SM clock, power and throttle reasons in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.samples = []  # (t, sm_mhz, max_mhz, reasons_mask)
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                try:
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                self.samples.append((time.perf_counter(), sm, mask))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread.start()
+
+    def stop(self):
+        self._stop.set()
+        if self.ok:
+            self._thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "NVML unavailable"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if len(inside) < 3:
+            inside = [s for s in self.samples if s[0] <= t1]
+            inside = inside[-max(3, len(inside) // 4):] if inside else []
+            window = "timed+warmup (timed region shorter than the sampling period)"
+        reasons = set()
+        for _, _, mask in inside:
+            for bit, name in self.REASONS.items():
+                if mask & bit and name != "gpu_idle":
+                    reasons.add(name)
+        sm = [s[1] for s in inside]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- the CUDA arm
+
+class Launcher:
+    """Pointer-level calls of the C ABI over a ring of buffer sets on one stream."""
+
+    def __init__(self, dq, wl, device, sets: int):
+        import torch
+
+        self.dq, self.wl = dq, wl
+        t = wl.tensors
+        self.stream = torch.cuda.Stream(device)
+        self.sptr = self.stream.cuda_stream
+        self.sets = []
+        xs = t["x"].to(device)
+        for i in range(sets):
+            x = xs if i == 0 else xs.clone()
+            if wl.kind == "dynamic_quant":
+                cols = wl.cols
+                ycols = cols if wl.y_dtype == "int8" else (cols // 2 if wl.y_dtype == "int4" else cols // 8)
+                ydt = {"int8": torch.int8, "int4": torch.uint8, "int32": torch.int32}[wl.y_dtype]
+                y = torch.empty((wl.rows, ycols), dtype=ydt, device=device)
+                scale = torch.empty(wl.rows, dtype=torch.float32, device=device)
+                offset = torch.empty(wl.rows, dtype=torch.float32, device=device) if wl.mode == "asymmetric" else None
+                self.sets.append(dict(x=x, y=y, scale=scale, offset=offset))
+            else:
+                out = torch.empty(tuple(t["x"].shape), dtype=torch.int8, device=device)
+                qs = torch.empty(tuple(t["x"].shape[:2]), dtype=torch.float32, device=device)
+                self.sets.append(dict(x=x, out=out, qs=qs))
+        self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k != "x"}
+        if wl.kind == "dynamic_quant":
+            gi = self.side.get("group_index")
+            self.ngroups = int(gi.numel()) if gi is not None else 0
+            x_dt = dq.DQ_BF16 if t["x"].dtype == torch.bfloat16 else dq.DQ_F16
+            self.ws_bytes = dq.dq_get_workspace_size(wl.rows, wl.cols, x_dt,
+                                                     dq.DQ_ASYMMETRIC if wl.mode == "asymmetric" else dq.DQ_SYMMETRIC,
+                                                     {"int8": dq.DQ_INT8, "int4": dq.DQ_INT4X2,
+                                                      "int32": dq.DQ_INT32}[wl.y_dtype], self.ngroups)
+            self.ws = torch.zeros(max(1, self.ws_bytes // 4), dtype=torch.int32, device=device)
+        self._prepare_args()
+
+    def _prepare_args(self):
+        import torch
+
+        dq, wl = self.dq, self.wl
+        p = lambda t: None if t is None else t.data_ptr()
+        code = {torch.float32: dq.DQ_F32, torch.float16: dq.DQ_F16, torch.bfloat16: dq.DQ_BF16}
+        self.calls = []
+        for s in self.sets:
+            if wl.kind == "dynamic_quant":
+                sm = self.side.get("smooth")
+                gi = self.side.get("group_index")
+                args = (p(s["x"]), code[s["x"].dtype], wl.rows, wl.cols, p(sm), code[sm.dtype] if sm is not None
+                        else dq.DQ_F32, p(gi), self.ngroups,
+                        dq.DQ_ASYMMETRIC if wl.mode == "asymmetric" else dq.DQ_SYMMETRIC,
+                        {"int8": dq.DQ_INT8, "int4": dq.DQ_INT4X2, "int32": dq.DQ_INT32}[wl.y_dtype],
+                        p(s["y"]), p(s["scale"]), p(s["offset"]), p(self.ws) if self.ws_bytes else None,
+                        self.ws_bytes, self.sptr)
+                self.calls.append((dq.dq_dynamic_quant, args))
+            else:
+                d = self.side
+                b, sq, h = (int(v) for v in s["x"].shape)
+                args = (p(s["x"]), code[s["x"].dtype], b, sq, h, p(d["ada_scale"]), p(d["ada_shift"]),
+                        p(d.get("weight")), p(d.get("bias")), p(d.get("smooth")), code[d["ada_scale"].dtype],
+                        float(wl.epsilon), p(s["out"]), p(s["qs"]), None, 0, self.sptr)
+                self.calls.append((dq.dq_ada_layernorm_quant, args))
+
+    def step(self, i: int):
+        fn, args = self.calls[i % len(self.calls)]
+        st = fn(*args)
+        if st != 0:
+            raise RuntimeError(f"launch failed: {self.dq.dq_status_string(st)}")
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from token_dynamic_quantization_b200 import dq
+    from token_dynamic_quantization_b200 import workloads
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = workloads.make(args.workload)
+    nbytes = algorithmic_bytes(wl)
+    per_set = wl.tensors["x"].numel() * wl.tensors["x"].element_size() + nbytes
+    sets = max(2, math.ceil(3 * L2_BYTES / per_set))
+    L = Launcher(dq, wl, device, sets)
+    torch.cuda.synchronize(device)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    graph = None
+    with torch.cuda.stream(L.stream):
+        for i in range(args.warmup):
+            L.step(i)
+        if args.graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=L.stream):
+                for i in range(args.steps):
+                    L.step(i)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    torch.cuda.synchronize(device)
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    start.record(L.stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            L.step(i)
+    end.record(L.stream)
+    torch.cuda.synchronize(device)
+    t1 = time.perf_counter()
+    barrier(world)
+    sampler.stop()
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, world, device)
+    clocks = sampler.summary(t0, t1)
+    if graph is not None:
+        del graph
+
+    ms_per_step = ms / args.steps
+    gbs_per_gpu = nbytes / (ms_per_step * 1e-3) / 1e9
+    value = gbs_per_gpu * world  # every rank moved nbytes per step in ms_per_step (max over ranks)
+    rows_per_s = wl.rows * world / (ms_per_step * 1e-3)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs, the call, D2H of its outputs, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(dq, wl, device, nbytes, world, min(args.steps, 20))
+
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (ms_local / args.steps * 1e-3) / 1e9
+    result = None
+    if rank == 0:
+        traffic = profiled_traffic(args.workload)
+        result = {
+            "metric": METRIC,
+            "value": round(value, 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if "bf16" in args.workload else "f16",
+            "data": "synthetic",
+            "config": {
+                "workload": args.workload,
+                "rows": wl.rows,
+                "cols": wl.cols,
+                "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric",
+                "y_dtype": wl.y_dtype,
+                "algorithmic_bytes_per_step": nbytes,
+                "rows_per_s": round(rows_per_s, 1),
+                "parallelism": f"dp{world} (independent row batches, no collective)",
+                "l2": f"inputs larger than L2: {sets} rotating buffer sets, {sets * per_set / 1e6:.0f} MB > 126 MB",
+                "launch": "cuda graph of K launches" if args.graph else "eager C-ABI launches",
+            },
+            "roofline": {
+                "bound": "hbm",
+                "achieved": round(achieved, 2),
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy kernel)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s",
+                "traffic": traffic,
+                "kernel": "dynamic_quant_vec_kernel" if wl.kind == "dynamic_quant" else
+                "ada_layernorm_quant_vec_kernel",
+            },
+            "clocks": clocks,
+            "gpu_launches": args.steps * world,
+        }
+        if e2e is not None:
+            result["e2e"] = e2e
+        if not args.no_cpu_baseline and world == 1:
+            result["cpu_baseline"] = cpu_baseline(wl, nbytes, target_s=args.cpu_seconds)
+    return result
+
+
+def run_e2e(dq, wl, device, nbytes, world, steps):
+    import torch
+
+    t = wl.tensors
+    host = {k: (v.pin_memory() if v is not None else None) for k, v in t.items()}
+    stream = torch.cuda.Stream(device)
+    dev = {k: (torch.empty_like(v, device=device) if v is not None else None) for k, v in host.items()}
+
+    def one():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        if wl.kind == "dynamic_quant":
+            y, s, o, _ = dq.dynamic_quant(dev["x"], dev.get("smooth"), dev.get("group_index"), mode=wl.mode,
+                                          y_dtype=wl.y_dtype, stream=stream.cuda_stream)
+            outs = [y, s] + ([o] if o is not None else [])
+        else:
+            y, s = dq.ada_layernorm_quant(dev["x"], dev["ada_scale"], dev["ada_shift"], dev.get("weight"),
+                                          dev.get("bias"), dev.get("smooth"), epsilon=wl.epsilon,
+                                          stream=stream.cuda_stream)
+            outs = [y, s]
+        hs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        for h, o in zip(hs, outs):
+            h.copy_(o, non_blocking=True)
+        return outs
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            outs = one()
+        torch.cuda.synchronize(device)
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for _ in range(steps):
+            outs = one()
+        end.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(start.elapsed_time(end), world, device) / steps
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    return {"value": round(nbytes * world / (ms * 1e-3) / 1e9, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": steps,
+            "note": "pinned host buffers -> device, C-ABI call, device -> pinned host, per step"}
+
+
+# ---------------------------------------------------------------- the oracle (CPU) arm
+
+def _oracle_rows(wl, r0, r1):
+    import oracle
+
+    t = wl.tensors
+    if wl.kind == "dynamic_quant":
+        gi = t.get("group_index")
+        smooth = t.get("smooth")
+        if gi is not None:
+            # rows [r0, r1) with their experts: rebase the cumulative end rows
+            g = gi.numpy().astype("int64") - r0
+            g = g.clip(0, r1 - r0).astype("int32")
+            return oracle.dynamic_quant(t["x"][r0:r1], smooth=smooth, group_index=g, mode=wl.mode,
+                                        y_dtype=wl.y_dtype)
+        return oracle.dynamic_quant(t["x"][r0:r1], smooth=smooth, mode=wl.mode, y_dtype=wl.y_dtype)
+    b, s, h = t["x"].shape
+    x = t["x"].reshape(b * s, h)
+    # rows of one batch entry at a time (the adaptive parameters are per batch)
+    bi = r0 // s
+    r1 = min(r1, (bi + 1) * s)
+    xs = x[r0:r1].reshape(1, r1 - r0, h)
+    return oracle.ada_layernorm_quant(xs, t["ada_scale"][bi:bi + 1], t["ada_shift"][bi:bi + 1], t.get("weight"),
+                                      t.get("bias"), t.get("smooth"), epsilon=wl.epsilon)
+
+
+def cpu_baseline(wl, nbytes, target_s: float = 10.0):
+    """The oracle as it stands, single-threaded, on a bounded sample of rows."""
+    rows = wl.rows
+    bytes_per_row = nbytes / rows
+    # calibrate on a small slice, then size the sample to ~target_s of CPU work
+    n0 = min(rows, 64)
+    t0 = time.perf_counter()
+    _oracle_rows(wl, 0, n0)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    per_row = dt / n0
+    n = int(min(rows, max(n0, target_s / per_row)))
+    passes, elapsed, done = 0, 0.0, 0
+    while elapsed < target_s and passes < 1000:
+        t0 = time.perf_counter()
+        _oracle_rows(wl, 0, n)
+        elapsed += time.perf_counter() - t0
+        done += n
+        passes += 1
+    gbs = done * bytes_per_row / elapsed / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of {rows} rows x {passes} pass(es) ({elapsed:.1f} s), "
+                      "single-threaded C++ oracle, GB/s of the same algorithmic bytes",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args, world, rank):
+    from token_dynamic_quantization_b200 import workloads
+
+    if rank != 0:
+        return None
+    wl = workloads.make(args.workload)
+    nbytes = algorithmic_bytes(wl)
+    rows = wl.rows
+    bytes_per_row = nbytes / rows
+    # size each step so that warmup + steps take about args.cpu_seconds in total
+    n0 = min(rows, 64)
+    t0 = time.perf_counter()
+    _oracle_rows(wl, 0, n0)
+    per_row = max(time.perf_counter() - t0, 1e-6) / n0
+    budget = args.cpu_seconds * 3
+    n = int(max(1, min(rows, budget / (per_row * max(1, args.steps + args.warmup)))))
+    for _ in range(args.warmup):
+        _oracle_rows(wl, 0, n)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_rows(wl, 0, n)
+    elapsed = time.perf_counter() - t0
+    ms_per_step = elapsed / args.steps * 1e3
+    gbs = n * bytes_per_row * args.steps / elapsed / 1e9
+    sample = f"first {n} of {rows} rows per step, single-threaded C++ oracle"
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(gbs, 4),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if "bf16" in args.workload else "f16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "rows": rows, "cols": wl.cols,
+                   "rows_per_step": n, "rows_per_s": round(n * args.steps / elapsed, 1)},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "reference arm = the CPU oracle (the pages ship no runnable implementation)",
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--graph", action="store_true", help="replay the K timed launches as one CUDA graph")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_ours(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

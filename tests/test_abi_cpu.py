@@ -1,0 +1,162 @@
+"""C-ABI checks that need no GPU: exports and host-side validation.
+
+Every call here is rejected by the host validation before anything is
+launched, so the fake pointers below are never dereferenced (on any machine).
+"""
+
+import os
+import re
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+FAKE = 0x10000  # 64 KiB-aligned fake device address (never dereferenced)
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w]*\s*\*?\s*(dq_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant", "dq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(dq_lib):
+    import ctypes
+
+    lib = ctypes.CDLL(dq_lib.LIBRARY_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"libdq.so does not export {n}"
+
+
+def test_status_strings(dq_lib):
+    for s in range(0, 9):
+        text = dq_lib.dq_status_string(s)
+        assert text.startswith("DQ_")
+    assert "unknown" in dq_lib.dq_status_string(99)
+
+
+def test_workspace_size(dq_lib):
+    d = dq_lib
+    assert d.dq_get_workspace_size(8192, 4096, d.DQ_BF16, d.DQ_SYMMETRIC, d.DQ_INT8, 0) == 0
+    assert d.dq_get_workspace_size(32768, 7168, d.DQ_BF16, d.DQ_SYMMETRIC, d.DQ_INT8, 64) == 4
+    assert d.dq_get_workspace_size(0, 2, d.DQ_F16, d.DQ_ASYMMETRIC, d.DQ_INT4X2, 0) == 0
+    bad = [
+        ((-1, 8, d.DQ_F16, 0, d.DQ_INT8, 0), d.DQ_ERR_BAD_SHAPE),
+        ((4, 0, d.DQ_F16, 0, d.DQ_INT8, 0), d.DQ_ERR_BAD_SHAPE),
+        ((4, 7, d.DQ_F16, 0, d.DQ_INT4X2, 0), d.DQ_ERR_BAD_SHAPE),
+        ((4, 12, d.DQ_F16, 0, d.DQ_INT32, 0), d.DQ_ERR_BAD_SHAPE),
+        ((4, 8, d.DQ_F32, 0, d.DQ_INT8, 0), d.DQ_ERR_BAD_DTYPE),
+        ((4, 8, d.DQ_F16, 0, d.DQ_F16, 0), d.DQ_ERR_BAD_DTYPE),
+        ((4, 8, d.DQ_F16, 2, d.DQ_INT8, 0), d.DQ_ERR_BAD_ARGUMENT),
+        ((4, 8, d.DQ_F16, 0, d.DQ_INT8, -1), d.DQ_ERR_BAD_ARGUMENT),
+        ((4, 8, d.DQ_F16, 0, d.DQ_INT8, d.DQ_MAX_GROUPS + 1), d.DQ_ERR_UNSUPPORTED),
+    ]
+    for args, want in bad:
+        with pytest.raises(d.DQError) as ei:
+            d.dq_get_workspace_size(*args)
+        assert ei.value.status == want, args
+
+
+def _dq(d, **kw):
+    a = dict(x=FAKE, x_dtype=d.DQ_BF16, rows=4, cols=64, smooth=None, smooth_dtype=d.DQ_F32, group_index=None,
+             num_groups=0, mode=d.DQ_SYMMETRIC, y_dtype=d.DQ_INT8, y=FAKE, scale=FAKE, offset=None,
+             workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return d.dq_dynamic_quant(**a)
+
+
+def test_dynamic_quant_validation(dq_lib):
+    d = dq_lib
+    assert _dq(d, rows=0, x=None, y=None, scale=None) == d.DQ_OK  # empty input: no-op, no launch
+    cases = [
+        (dict(x=None), d.DQ_ERR_NULL_POINTER),
+        (dict(y=None), d.DQ_ERR_NULL_POINTER),
+        (dict(scale=None), d.DQ_ERR_NULL_POINTER),
+        (dict(mode=d.DQ_ASYMMETRIC), d.DQ_ERR_NULL_POINTER),           # offset missing
+        (dict(rows=-3), d.DQ_ERR_BAD_SHAPE),
+        (dict(cols=0), d.DQ_ERR_BAD_SHAPE),
+        (dict(cols=63, y_dtype=d.DQ_INT4X2), d.DQ_ERR_BAD_SHAPE),
+        (dict(cols=60, y_dtype=d.DQ_INT32), d.DQ_ERR_BAD_SHAPE),
+        (dict(x_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
+        (dict(y_dtype=d.DQ_BF16), d.DQ_ERR_BAD_DTYPE),
+        (dict(smooth=FAKE, smooth_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
+        (dict(mode=7), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(group_index=FAKE, num_groups=0, smooth=FAKE), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(group_index=None, num_groups=3, smooth=FAKE), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(group_index=FAKE, num_groups=3), d.DQ_ERR_BAD_ARGUMENT),  # MoE needs smooth scales
+        (dict(group_index=FAKE, num_groups=3, smooth=FAKE), d.DQ_ERR_WORKSPACE_TOO_SMALL),
+        (dict(group_index=FAKE, num_groups=3, smooth=FAKE, workspace=FAKE, workspace_bytes=2),
+         d.DQ_ERR_WORKSPACE_TOO_SMALL),
+        (dict(group_index=FAKE, num_groups=d.DQ_MAX_GROUPS + 1, smooth=FAKE, workspace=FAKE, workspace_bytes=4),
+         d.DQ_ERR_UNSUPPORTED),
+        (dict(x=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(mode=d.DQ_ASYMMETRIC, offset=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(smooth=FAKE + 2, smooth_dtype=d.DQ_F32), d.DQ_ERR_MISALIGNED),
+        (dict(y=FAKE + 2, y_dtype=d.DQ_INT32), d.DQ_ERR_MISALIGNED),
+        (dict(group_index=FAKE + 2, num_groups=3, smooth=FAKE, workspace=FAKE, workspace_bytes=4),
+         d.DQ_ERR_MISALIGNED),
+        (dict(group_index=FAKE, num_groups=3, smooth=FAKE, workspace=FAKE + 2, workspace_bytes=4),
+         d.DQ_ERR_MISALIGNED),
+    ]
+    for kw, want in cases:
+        assert _dq(d, **kw) == want, kw
+
+
+def _ada(d, **kw):
+    a = dict(x=FAKE, x_dtype=d.DQ_BF16, batch=2, seq=3, hidden=64, ada_scale=FAKE, ada_shift=FAKE, weight=None,
+             bias=None, smooth=None, param_dtype=d.DQ_BF16, epsilon=1e-6, out=FAKE, quant_scale=FAKE,
+             workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return d.dq_ada_layernorm_quant(**a)
+
+
+def test_ada_layernorm_quant_validation(dq_lib):
+    d = dq_lib
+    assert _ada(d, batch=0, x=None, out=None) == d.DQ_OK
+    assert _ada(d, seq=0, x=None, out=None) == d.DQ_OK
+    cases = [
+        (dict(x=None), d.DQ_ERR_NULL_POINTER),
+        (dict(ada_scale=None), d.DQ_ERR_NULL_POINTER),
+        (dict(ada_shift=None), d.DQ_ERR_NULL_POINTER),
+        (dict(out=None), d.DQ_ERR_NULL_POINTER),
+        (dict(quant_scale=None), d.DQ_ERR_NULL_POINTER),
+        (dict(batch=-1), d.DQ_ERR_BAD_SHAPE),
+        (dict(hidden=0), d.DQ_ERR_BAD_SHAPE),
+        (dict(x_dtype=d.DQ_F32), d.DQ_ERR_BAD_DTYPE),
+        (dict(param_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
+        (dict(epsilon=float("nan")), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(epsilon=-1.0), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(epsilon=float("inf")), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(x=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(quant_scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(param_dtype=d.DQ_F32, ada_scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(weight=FAKE + 1), d.DQ_ERR_MISALIGNED),
+    ]
+    for kw, want in cases:
+        assert _ada(d, **kw) == want, kw
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    """The product path has no fallback: without libdq.so the import raises."""
+    pkg = os.path.join(ROOT, "token_dynamic_quantization_b200")
+    dst = tmp_path / "token_dynamic_quantization_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    code = "import token_dynamic_quantization_b200.dq"
+    res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
+    assert res.returncode != 0
+    assert "ImportError" in res.stderr and "no CPU fallback" in res.stderr
