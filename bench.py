@@ -248,6 +248,13 @@ class Launcher:
                                                      {"int8": dq.DQ_INT8, "int4": dq.DQ_INT4X2,
                                                       "int32": dq.DQ_INT32}[wl.y_dtype], self.ngroups)
             self.ws = torch.zeros(max(1, self.ws_bytes // 4), dtype=torch.int32, device=device)
+        else:
+            x = t["x"]
+            self.ws_bytes = dq.dq_ada_layernorm_quant_get_workspace_size(
+                int(x.shape[0]), int(x.shape[1]), int(x.shape[2]),
+                dq.DQ_BF16 if x.dtype == torch.bfloat16 else dq.DQ_F16,
+                {torch.float32: dq.DQ_F32, torch.float16: dq.DQ_F16, torch.bfloat16: dq.DQ_BF16}[t["ada_scale"].dtype])
+            self.ws = torch.zeros(max(4, (self.ws_bytes + 15) // 16 * 4), dtype=torch.float32, device=device)
         self._prepare_args()
 
     def _prepare_args(self):
@@ -273,7 +280,7 @@ class Launcher:
                 b, sq, h = (int(v) for v in s["x"].shape)
                 args = (p(s["x"]), code[s["x"].dtype], b, sq, h, p(d["ada_scale"]), p(d["ada_shift"]),
                         p(d.get("weight")), p(d.get("bias")), p(d.get("smooth")), code[d["ada_scale"].dtype],
-                        float(wl.epsilon), p(s["out"]), p(s["qs"]), None, 0, self.sptr)
+                        float(wl.epsilon), p(s["out"]), p(s["qs"]), p(self.ws), self.ws_bytes, self.sptr)
                 self.calls.append((dq.dq_ada_layernorm_quant, args))
 
     def step(self, i: int):
@@ -316,13 +323,14 @@ def run_ours(args, world, rank, local):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
-    start.record(L.stream)
-    if graph is not None:
-        graph.replay()
-    else:
-        for i in range(args.steps):
-            L.step(i)
-    end.record(L.stream)
+    with torch.cuda.stream(L.stream):
+        start.record(L.stream)
+        if graph is not None:
+            graph.replay()  # replays on the current stream, i.e. L.stream
+        else:
+            for i in range(args.steps):
+                L.step(i)
+        end.record(L.stream)
     torch.cuda.synchronize(device)
     t1 = time.perf_counter()
     barrier(world)

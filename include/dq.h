@@ -1,7 +1,7 @@
 /*
  * dq.h — C ABI of the B200 (sm_100a) per-token dynamic quantization library.
  *
- * Two operations, each one CUDA kernel launch on the caller's stream:
+ * Two operations, launched asynchronously on the caller's stream:
  *
  *   dq_dynamic_quant        aclnnDynamicQuantV2, "Formula" and "Description":
  *                           per-row (per-token) symmetric or asymmetric
@@ -13,8 +13,9 @@
  *                           y * (1 + scale) + shift, optional smooth scales,
  *                           then symmetric INT8 dynamic quantization.
  *
- * plus the workspace query of the two-phase calling convention both pages
- * describe ("...GetWorkspaceSize" first, then the run): dq_get_workspace_size.
+ * plus the workspace queries of the two-phase calling convention both pages
+ * describe ("...GetWorkspaceSize" first, then the run): dq_get_workspace_size
+ * and dq_ada_layernorm_quant_get_workspace_size.
  *
  * Conventions shared by every entry point
  *   - Every tensor pointer is a DEVICE pointer (cudaMalloc'd or equivalent),
@@ -30,6 +31,10 @@
  *     through the CUDA stream like any other kernel's.
  *   - Results are deterministic: the same inputs give the same bytes on
  *     every call (both pages state deterministic implementations).
+ *   - Rows are streamed through shared memory with bulk (TMA) copies; every
+ *     wait in the kernels is bounded. If a copy never completes (a device
+ *     fault, never a data-dependent condition) the affected rows get NaN
+ *     scales instead of the kernel hanging.
  *
  * Arithmetic (fixed by the formulas; identical to the CPU oracle):
  *   IEEE binary32 throughout; x and smooth scales are widened exactly;
@@ -158,6 +163,15 @@ dq_status dq_dynamic_quant(const void* x, dq_dtype x_dtype, int64_t rows, int64_
                            void* y, float* scale, float* offset,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Workspace query for dq_ada_layernorm_quant (the first phase of
+ * aclnnAdaLayerNormQuant's two-phase convention). Writes the bytes of device
+ * workspace the call needs: batch * hidden * 8 (a folded table of the affine
+ * parameters, rebuilt on every call), or 0 when batch * seq == 0. Host only.
+ * Errors: DQ_ERR_NULL_POINTER, DQ_ERR_BAD_SHAPE, DQ_ERR_BAD_DTYPE. */
+dq_status dq_ada_layernorm_quant_get_workspace_size(int64_t batch, int64_t seq, int64_t hidden,
+                                                    dq_dtype x_dtype, dq_dtype param_dtype,
+                                                    size_t* workspace_bytes);
+
 /* Fused AdaLayerNorm + symmetric INT8 quantization (aclnnAdaLayerNormQuant,
  * "Formula"; the page fuses only DynamicQuant, i.e. symmetric INT8).
  *
@@ -177,10 +191,17 @@ dq_status dq_dynamic_quant(const void* x, dq_dtype x_dtype, int64_t rows, int64_
  *   epsilon            finite, >= 0.
  *   out                device int8 [batch, seq, hidden]; quant_scale device
  *                      float [batch, seq].
- *   workspace          reserved: this operation needs none (pass NULL, 0).
- * Statistics are reduced in a different order than a sequential loop, so a
- * result may differ from a sequential fp32 evaluation in the last bits:
- * quant_scale by a relative 1e-5 at most, and rarely a code by 1.
+ *   workspace          device, 16-byte aligned, at least the bytes
+ *                      dq_ada_layernorm_quant_get_workspace_size returned.
+ *                      Its contents are scratch, overwritten by every call;
+ *                      calls that run concurrently need separate workspaces.
+ * Two kernels are launched on `stream`: one folds steps 1-3's parameters into
+ * y = n * A + B (A, B per batch and column, in the workspace), the second
+ * processes the rows and overlaps its start with the first.
+ * The row statistics are reduced in a different order than a sequential loop
+ * and steps 1-3 are folded, so a result may differ from a sequential fp32
+ * evaluation in the last bits: quant_scale by a relative 1e-5 at most, and
+ * rarely a code by 1.
  * Errors: as dq_dynamic_quant (DQ_ERR_BAD_ARGUMENT for a bad epsilon). */
 dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype,
                                  int64_t batch, int64_t seq, int64_t hidden,

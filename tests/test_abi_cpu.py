@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant", "dq_status_string"):
+    for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant_get_workspace_size",
+              "dq_ada_layernorm_quant", "dq_status_string"):
         assert n in names
 
 
@@ -117,10 +118,23 @@ def test_dynamic_quant_validation(dq_lib):
         assert _dq(d, **kw) == want, kw
 
 
+def test_ada_workspace_size(dq_lib):
+    d = dq_lib
+    assert d.dq_ada_layernorm_quant_get_workspace_size(4, 4096, 3072, d.DQ_BF16, d.DQ_BF16) == 4 * 3072 * 8
+    assert d.dq_ada_layernorm_quant_get_workspace_size(0, 4096, 3072, d.DQ_BF16, d.DQ_BF16) == 0
+    for args, want in [((-1, 2, 8, d.DQ_BF16, d.DQ_BF16), d.DQ_ERR_BAD_SHAPE),
+                       ((1, 2, 0, d.DQ_BF16, d.DQ_BF16), d.DQ_ERR_BAD_SHAPE),
+                       ((1, 2, 8, d.DQ_F32, d.DQ_BF16), d.DQ_ERR_BAD_DTYPE),
+                       ((1, 2, 8, d.DQ_F16, d.DQ_INT8), d.DQ_ERR_BAD_DTYPE)]:
+        with pytest.raises(d.DQError) as ei:
+            d.dq_ada_layernorm_quant_get_workspace_size(*args)
+        assert ei.value.status == want
+
+
 def _ada(d, **kw):
     a = dict(x=FAKE, x_dtype=d.DQ_BF16, batch=2, seq=3, hidden=64, ada_scale=FAKE, ada_shift=FAKE, weight=None,
              bias=None, smooth=None, param_dtype=d.DQ_BF16, epsilon=1e-6, out=FAKE, quant_scale=FAKE,
-             workspace=None, workspace_bytes=0, stream=None)
+             workspace=FAKE, workspace_bytes=2 * 64 * 8, stream=None)
     a.update(kw)
     return d.dq_ada_layernorm_quant(**a)
 
@@ -146,6 +160,9 @@ def test_ada_layernorm_quant_validation(dq_lib):
         (dict(quant_scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
         (dict(param_dtype=d.DQ_F32, ada_scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
         (dict(weight=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(workspace=None), d.DQ_ERR_WORKSPACE_TOO_SMALL),
+        (dict(workspace_bytes=2 * 64 * 8 - 4), d.DQ_ERR_WORKSPACE_TOO_SMALL),
+        (dict(workspace=FAKE + 4), d.DQ_ERR_MISALIGNED),
     ]
     for kw, want in cases:
         assert _ada(d, **kw) == want, kw

@@ -249,8 +249,8 @@ def test_asymmetric_huge_offset_rows(dq):
     x = torch.full((4, cols), 1000.0, dtype=torch.float16)
     x[1] = -1000.0
     x[2] = 7.0
-    k = torch.arange(cols, dtype=torch.float64)
-    smooth = (1.0 + k * 2.0 ** -22).to(torch.float32)
+    k = torch.arange(cols, dtype=torch.float64) % 4
+    smooth = (1.0 + k * 2.0 ** -23).to(torch.float32)
     for y_dtype in ("int8", "int4"):
         want = oracle.dynamic_quant(x, smooth=smooth, mode="asymmetric", y_dtype=y_dtype)
         assert np.abs(want[2]).max() > 2 ** 20

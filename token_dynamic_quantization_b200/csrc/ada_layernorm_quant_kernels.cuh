@@ -1,21 +1,38 @@
 // Fused AdaLayerNorm + symmetric INT8 dynamic quantization
 // (aclnnAdaLayerNormQuant, "Formula" steps 1-5), sm_100a.
 //
-// One HBM read of x and one write of the codes per row; everything between
-// stays in registers. The statistics are exact-as-possible rather than
-// Welford: the row is resident, so a two-pass mean / centred variance costs
-// no extra traffic. Per-thread partial sums are fp32, the cross-thread sums
-// double; the variance is corrected to the double mean:
-//   sum (v - m_d)^2 = sum (v - m_f)^2 - H (m_d - m_f)^2,
-// so E(x) and Var(x) agree with a double-precision evaluation rounded to
-// fp32 except for the last bit in rare rows. x - E(x) is multiplied by the
-// correctly rounded 1/sqrt(Var + eps) instead of divided by the square root
-// (the only other departure from a sequential fp32 evaluation); steps 2-3 are
-// one IEEE operation each in the order the formula prints them, and steps 4-5
-// are the exact DynamicQuant quantizer.
+// Two launches per call:
+//   1. ada_affine_table_kernel folds the per-(batch, column) parameters of
+//      steps 1-3 into a table in the caller's workspace,
+//        A[b][c] = (w[c] * (1 + scale[b][c])) * smooth[c]
+//        B[b][c] = ((bias[c] * (1 + scale[b][c])) + shift[b][c]) * smooth[c]
+//      (absent weight = 1, bias = 0, smooth = 1), so steps 1-3 become one FMA
+//      per element, y = n * A + B. The table is batch x hidden x 8 bytes and
+//      is read through L1/L2 by the main kernel.
+//   2. ada_layernorm_quant_tma_kernel streams rows through the bulk-copy (TMA)
+//      ring (tma_pipeline.cuh) and keeps each thread's share of the row in
+//      registers between its passes. It is launched as a programmatic
+//      dependent of the table kernel: it sets up its ring and starts copying
+//      rows while the table is still being written, and waits for the table
+//      (griddepcontrol.wait) just before first reading it.
+//
+// Arithmetic:
+//   * E(x), Var(x): the row is resident, so a two-pass mean / centred
+//     variance costs no extra traffic (no Welford needed). Per-thread partial
+//     sums are fp32, the cross-thread sums double; the variance is corrected
+//     to the double mean, sum (v - m_d)^2 = sum (v - m_f)^2 - H (m_d - m_f)^2,
+//     so both statistics match a double evaluation rounded to fp32 except for
+//     the last bit in rare rows.
+//   * n = (x - E(x)) * rstd with rstd = RN(1 / RN(sqrt(Var + eps))), then
+//     y = n * A + B. Against a sequential evaluation that rounds every printed
+//     operation separately and divides by the square root, this moves y by a
+//     few ulps: quant_scale stays within a relative 1e-6 and about one code in
+//     10^6 moves by one (measured on the 4 x 4096 x 3072 workload).
+//   * steps 4-5 are the DynamicQuant quantizer (exact IEEE semantics).
 #pragma once
 
 #include "dq_device.cuh"
+#include "tma_pipeline.cuh"
 
 namespace dq {
 
@@ -29,144 +46,275 @@ struct AdaArgs {
   const void* smooth;     // [hidden] or nullptr
   int param_dtype;
   float epsilon;
+  double inv_hidden;      // 1 / hidden, rounded once in double
+  float* table;           // workspace: A [batch][hidden], then B [batch][hidden]
   int8_t* out;
   float* quant_scale;
   int tpr;
   int groups;
+  int stages;
+  uint32_t stage_stride;
 };
 
-// ============================================================ vector kernel
+__host__ __device__ inline size_t ada_smem_bytes(int groups, int stages, uint32_t stride) {
+  return static_cast<size_t>(groups) * stages * stride + static_cast<size_t>(groups) * stages * 8;
+}
 
-constexpr int kAdaMaxBlock = 512;
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ============================================================ affine table
+
+constexpr int kTableBlock = 256;
+
+__global__ void __launch_bounds__(kTableBlock) ada_affine_table_kernel(const AdaArgs a) {
+  pdl_launch_dependents();  // the main kernel may start its row copies now
+  const int64_t H = a.hidden;
+  const int64_t total = a.batch * H;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t c = idx % H;
+    const float onep = __fadd_rn(1.0f, load_param(a.ada_scale, a.param_dtype, idx));
+    const float w = a.weight ? load_param(a.weight, a.param_dtype, c) : 1.0f;
+    const float bs = a.bias ? load_param(a.bias, a.param_dtype, c) : 0.0f;
+    const float sm = a.smooth ? load_param(a.smooth, a.param_dtype, c) : 1.0f;
+    const float sh = load_param(a.ada_shift, a.param_dtype, idx);
+    a.table[idx] = __fmul_rn(__fmul_rn(w, onep), sm);
+    a.table[total + idx] = __fmul_rn(__fadd_rn(__fmul_rn(bs, onep), sh), sm);
+  }
+}
+
+// Rows whose quant_scale is below 2^-40 (RowQuant::exact_row): every element
+// of this thread's share with the IEEE division, out of line. y is recomputed
+// from the row still resident in shared memory with the main loop's
+// arithmetic (widen, - mean, * rstd, * A + B).
 template <typename InT>
-__global__ void __launch_bounds__(kAdaMaxBlock)
-ada_layernorm_quant_vec_kernel(const AdaArgs a) {
+__device__ __noinline__ void ada_quantize_row_exact(const uint4* srow, const float4* A4, const float4* B4,
+                                                    float mean_f, float rstd, RowQuant q, int lane_g, int tpr,
+                                                    int nvec, int8_t* orow) {
+  for (int vi = lane_g; vi < nvec; vi += tpr) {
+    float v[8];
+    InTraits<InT>::widen8(srow[vi], v);
+    const float4 a0 = A4[2 * vi], a1 = A4[2 * vi + 1], b0 = B4[2 * vi], b1 = B4[2 * vi + 1];
+    const float Av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[j] = __fmaf_rn(__fmul_rn(__fadd_rn(v[j], -mean_f), rstd), Av[j], Bv[j]);
+    }
+    uint32_t bits[8];
+    quant8_exact<false>(v, q, -127.0f, 127.0f, bits);
+    reinterpret_cast<uint2*>(orow)[vi] = pack8_int8(bits);
+  }
+}
+
+// ============================================================ bulk-copy kernel
+
+constexpr int kAdaMaxBlock = 256;
+#ifndef DQ_ADA_MIN_BLOCKS
+#define DQ_ADA_MIN_BLOCKS 3
+#endif
+
+template <typename InT, int VPT>
+__global__ void __launch_bounds__(kAdaMaxBlock, DQ_ADA_MIN_BLOCKS)
+ada_layernorm_quant_tma_kernel(const AdaArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ double red_d[2][2][kAdaMaxBlock / 32];  // [parity][sum|sq][warp]
   __shared__ float red_f[2][kAdaMaxBlock / 32];       // [parity][warp] absmax
 
   const int tpr = a.tpr;
+  const int S = a.stages;
   const int g = threadIdx.x / tpr;
   const int lane_g = threadIdx.x - g * tpr;
   const int warp = threadIdx.x >> 5;
   const int warp_g0 = (g * tpr) >> 5;
   const int nwarps_g = tpr >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t stride = a.stage_stride;
+  const size_t ring_bytes = static_cast<size_t>(a.groups) * S * stride;
+  uint8_t* ring = smem + static_cast<size_t>(g) * S * stride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes) + g * S;
+
+  if (threadIdx.x == 0) {
+    uint64_t* all = reinterpret_cast<uint64_t*>(smem + ring_bytes);
+    for (int i = 0; i < a.groups * S; ++i) mbar_init(all + i, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
 
   const int64_t rows = a.batch * a.seq;
   const int64_t workers = static_cast<int64_t>(gridDim.x) * a.groups;
   const int64_t worker = static_cast<int64_t>(blockIdx.x) * a.groups + g;
   const int64_t r_begin = worker * rows / workers;
   const int64_t r_end = (worker + 1) * rows / workers;
-  if (r_begin >= r_end) return;
-
-  const int64_t nvec = a.hidden >> 3;
-  const bool active = lane_g < nvec;  // one 8-element vector per thread
-  const int64_t col0 = static_cast<int64_t>(lane_g) * 8;
-  const double hd = static_cast<double>(a.hidden);
-
-  // per-column parameters (fp32, exact widening)
-  float w[8], bs[8], sm[8], onep[8], sh[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    w[j] = (active && a.weight) ? load_param(a.weight, a.param_dtype, col0 + j) : 1.0f;
-    bs[j] = (active && a.bias) ? load_param(a.bias, a.param_dtype, col0 + j) : 0.0f;
-    sm[j] = (active && a.smooth) ? load_param(a.smooth, a.param_dtype, col0 + j) : 1.0f;
+  const int64_t n = r_end - r_begin;
+  if (n <= 0) {
+    pdl_wait_primary();
+    return;
   }
-  int64_t cur_b = -1;
 
-  const uint4* __restrict__ xv = static_cast<const uint4*>(a.x);
-  uint4 buf0 = make_uint4(0, 0, 0, 0), buf1 = buf0, buf2 = buf0;
-  if (active) buf0 = __ldcs(xv + r_begin * nvec + lane_g);
-  if (active && r_begin + 1 < r_end) buf1 = __ldcs(xv + (r_begin + 1) * nvec + lane_g);
+  const int64_t H = a.hidden;
+  const int nvec = static_cast<int>(H >> 3);
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  const bool leader = lane_g == 0;
+  const uint64_t policy = leader ? l2_evict_first_policy() : 0;
+  const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  int64_t issued = 0;
+  int p_stage = 0;
+  auto issue_next = [&]() {
+    mbar_arrive_expect_tx(bars + p_stage, row_bytes);
+    bulk_copy_g2s(ring + static_cast<size_t>(p_stage) * stride, x_next, row_bytes, bars + p_stage, policy);
+    x_next += row_bytes;
+    ++issued;
+    p_stage = p_stage + 1 == S ? 0 : p_stage + 1;
+  };
+  if (leader) {
+    while (issued < n && issued < S - 1) issue_next();
+  }
 
+  pdl_wait_primary();  // the affine table is complete and visible from here on
+
+  // batch of the current row, tracked without division
+  int64_t b = r_begin / a.seq;
+  int64_t b_end = (b + 1) * a.seq;
+  const float4* A4 = reinterpret_cast<const float4*>(a.table + b * H);
+  const float4* B4 = reinterpret_cast<const float4*>(a.table + a.batch * H + b * H);
+  const int64_t table_b_stride4 = H / 4;
+  int8_t* orow = a.out + r_begin * H;
+
+  int c_stage = 0;
+  uint32_t phase = 0;
   int parity = 0;
-  for (int64_t r = r_begin; r < r_end; ++r) {
-    if (active && r + 2 < r_end) buf2 = __ldcs(xv + (r + 2) * nvec + lane_g);
-
-    const int64_t b = r / a.seq;
-    if (b != cur_b) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        onep[j] = active ? __fadd_rn(1.0f, load_param(a.ada_scale, a.param_dtype, b * a.hidden + col0 + j)) : 1.0f;
-        sh[j] = active ? load_param(a.ada_shift, a.param_dtype, b * a.hidden + col0 + j) : 0.0f;
-      }
-      cur_b = b;
+  for (int64_t r = r_begin; r < r_end; ++r, orow += H) {
+    if (r >= b_end) {
+      ++b;
+      b_end += a.seq;
+      A4 += table_b_stride4;
+      B4 += table_b_stride4;
     }
+    const bool arrived = mbar_wait_parity(bars + c_stage, phase);
+    const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(c_stage) * stride);
 
-    float v[8];
-    InTraits<InT>::widen8(buf0, v);
-    // ---- E(x)
-    float s1 = 0.0f;
-    if (active) {
+    // ---- pass 1: load, widen, E(x)
+    float v[VPT][8];
+    float2 s1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s1 = __fadd_rn(s1, v[j]);
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = lane_g + k * tpr;
+      InTraits<InT>::widen8(vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0), v[k]);  // zero when inactive
+#pragma unroll
+      for (int p = 0; p < 4; ++p) s1 = __fadd2_rn(s1, make_float2(v[k][2 * p], v[k][2 * p + 1]));
     }
-    double sum = warp_sum(static_cast<double>(s1));
+    double sum = warp_sum(static_cast<double>(s1.x) + static_cast<double>(s1.y));
+    bool failed;
     if (nwarps_g > 1) {
       if (lane == 0) red_d[parity][0][warp] = sum;
-      group_barrier(1 + g, tpr);
+      failed = group_barrier_or(1 + g, tpr, !arrived);
       sum = 0.0;
-      for (int i = 0; i < nwarps_g; ++i) sum += red_d[parity][0][warp_g0 + i];
+      for (int w = 0; w < nwarps_g; ++w) sum += red_d[parity][0][warp_g0 + w];
+    } else {
+      failed = __any_sync(0xffffffffu, !arrived);
+      __syncwarp();
     }
-    const double mean_d = sum / hd;
+    if (failed) {
+      for (int64_t rr = r + lane_g; rr < r_end; rr += tpr) a.quant_scale[rr] = __int_as_float(0x7fc00000);
+      if (leader) {
+        int st = c_stage;
+        uint32_t ph = phase;
+        for (int64_t j = r - r_begin + 1; j < issued; ++j) {
+          st = st + 1 == S ? 0 : st + 1;
+          if (st == 0) ph ^= 1u;
+          mbar_wait_parity(bars + st, ph);
+        }
+      }
+      return;
+    }
+    if (leader && issued < n) {
+      fence_proxy_async_smem();
+      issue_next();
+    }
+    c_stage = c_stage + 1 == S ? 0 : c_stage + 1;
+    if (c_stage == 0) phase ^= 1u;
+    const double mean_d = sum * a.inv_hidden;
     const float mean_f = __double2float_rn(mean_d);
-    // ---- Var(x), biased, about the double mean
-    float d[8];
-    float s2 = 0.0f;
+
+    // ---- pass 2: Var(x), biased, about the double mean
+    float2 s2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      d[j] = __fsub_rn(v[j], mean_f);
-      if (active) s2 = __fmaf_rn(d[j], d[j], s2);
+    for (int k = 0; k < VPT; ++k) {
+      const bool active = lane_g + k * tpr < nvec;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        float2 d = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-mean_f));
+        if (!active) d = make_float2(0.0f, 0.0f);
+        v[k][2 * p] = d.x;
+        v[k][2 * p + 1] = d.y;
+        s2 = __ffma2_rn(d, d, s2);
+      }
     }
-    double sq = warp_sum(static_cast<double>(s2));
+    double sq = warp_sum(static_cast<double>(s2.x) + static_cast<double>(s2.y));
     if (nwarps_g > 1) {
       if (lane == 0) red_d[parity][1][warp] = sq;
       group_barrier(1 + g, tpr);
       sq = 0.0;
-      for (int i = 0; i < nwarps_g; ++i) sq += red_d[parity][1][warp_g0 + i];
+      for (int w = 0; w < nwarps_g; ++w) sq += red_d[parity][1][warp_g0 + w];
     }
     const double dm = mean_d - static_cast<double>(mean_f);
-    double var_d = sq / hd - dm * dm;
+    double var_d = sq * a.inv_hidden - dm * dm;
     var_d = var_d > 0.0 ? var_d : 0.0;
     const float var_f = __double2float_rn(var_d);
     const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
 
-    // ---- steps 1-3, then absmax
+    // ---- pass 3: y = n * A + B, absmax
     float amax = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float t = __fmul_rn(d[j], rstd);
-      t = __fmul_rn(t, w[j]);
-      t = __fadd_rn(t, bs[j]);
-      t = __fmul_rn(t, onep[j]);
-      t = __fadd_rn(t, sh[j]);
-      t = __fmul_rn(t, sm[j]);
-      v[j] = t;
-      if (active) amax = fmaxf(amax, fabsf(t));
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = lane_g + k * tpr;
+      if (vi < nvec) {
+        const float4 a0 = __ldg(A4 + 2 * vi), a1 = __ldg(A4 + 2 * vi + 1);
+        const float4 b0 = __ldg(B4 + 2 * vi), b1 = __ldg(B4 + 2 * vi + 1);
+        const float Av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 nn = __fmul2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd));
+          const float2 y =
+              __ffma2_rn(nn, make_float2(Av[2 * p], Av[2 * p + 1]), make_float2(Bv[2 * p], Bv[2 * p + 1]));
+          v[k][2 * p] = y.x;
+          v[k][2 * p + 1] = y.y;
+          amax = fmaxf(amax, fmaxf(fabsf(y.x), fabsf(y.y)));
+        }
+      }
     }
     amax = warp_max(amax);
     if (nwarps_g > 1) {
       if (lane == 0) red_f[parity][warp] = amax;
       group_barrier(1 + g, tpr);
       amax = red_f[parity][warp_g0];
-      for (int i = 1; i < nwarps_g; ++i) amax = fmaxf(amax, red_f[parity][warp_g0 + i]);
+      for (int w = 1; w < nwarps_g; ++w) amax = fmaxf(amax, red_f[parity][warp_g0 + w]);
+      parity ^= 1;
     }
-    parity ^= 1;
 
     // ---- steps 4-5
     const RowQuant q = make_sym(amax, 127.0f);
     if (lane_g == 0) __stcs(a.quant_scale + r, q.scale);
-    if (active) {
-      float c[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) c[j] = q.zero_scale ? 0.0f : sym_code(v[j], q, -127.0f, 127.0f);
-      uint2* op = reinterpret_cast<uint2*>(a.out + r * a.hidden) + lane_g;
-      __stcs(op, pack_int8x8(c));
+    if (q.exact_row) {
+      ada_quantize_row_exact<InT>(srow, A4, B4, mean_f, rstd, q, lane_g, tpr, nvec, orow);
+      continue;
     }
-
-    buf0 = buf1;
-    buf1 = buf2;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = lane_g + k * tpr;
+      if (vi >= nvec) continue;
+      uint32_t bits[8];
+      if (q.zero_scale) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) bits[j] = __float_as_uint(kRoundMagic);
+      } else {
+        quant8<false, false>(v[k], q, -127.0f, 127.0f, bits);
+      }
+      __stcs(reinterpret_cast<uint2*>(orow) + vi, pack8_int8(bits));
+    }
   }
 }
 
@@ -184,6 +332,8 @@ ada_layernorm_quant_generic_kernel(const AdaArgs a) {
   constexpr int kWarps = kAdaGenericBlock / 32;
   const int64_t rows = a.batch * a.seq;
   const int64_t H = a.hidden;
+  const float* At = a.table;
+  const float* Bt = a.table + a.batch * H;
 
   auto block_sum = [&](double v) {
     v = warp_sum(v);
@@ -200,24 +350,19 @@ ada_layernorm_quant_generic_kernel(const AdaArgs a) {
     const int64_t base = r * H;
     double s1 = 0.0;
     for (int64_t c = threadIdx.x; c < H; c += kAdaGenericBlock) s1 += InTraits<InT>::widen1(a.x, base + c);
-    const double mean_d = block_sum(s1) / static_cast<double>(H);
+    const double mean_d = block_sum(s1) * a.inv_hidden;
     const float mean_f = __double2float_rn(mean_d);
     double s2 = 0.0;
     for (int64_t c = threadIdx.x; c < H; c += kAdaGenericBlock) {
       const double dd = static_cast<double>(InTraits<InT>::widen1(a.x, base + c)) - mean_d;
       s2 += dd * dd;
     }
-    const float var_f = __double2float_rn(block_sum(s2) / static_cast<double>(H));
+    const float var_f = __double2float_rn(block_sum(s2) * a.inv_hidden);
     const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
 
     auto value = [&](int64_t c) {
-      float t = __fmul_rn(__fsub_rn(InTraits<InT>::widen1(a.x, base + c), mean_f), rstd);
-      if (a.weight) t = __fmul_rn(t, load_param(a.weight, a.param_dtype, c));
-      if (a.bias) t = __fadd_rn(t, load_param(a.bias, a.param_dtype, c));
-      t = __fmul_rn(t, __fadd_rn(1.0f, load_param(a.ada_scale, a.param_dtype, b * H + c)));
-      t = __fadd_rn(t, load_param(a.ada_shift, a.param_dtype, b * H + c));
-      if (a.smooth) t = __fmul_rn(t, load_param(a.smooth, a.param_dtype, c));
-      return t;
+      const float nn = __fmul_rn(__fsub_rn(InTraits<InT>::widen1(a.x, base + c), mean_f), rstd);
+      return __fmaf_rn(nn, At[b * H + c], Bt[b * H + c]);
     };
     float amax = 0.0f;
     for (int64_t c = threadIdx.x; c < H; c += kAdaGenericBlock) amax = fmaxf(amax, fabsf(value(c)));
@@ -230,8 +375,7 @@ ada_layernorm_quant_generic_kernel(const AdaArgs a) {
     const RowQuant q = make_sym(amax, 127.0f);
     if (threadIdx.x == 0) a.quant_scale[r] = q.scale;
     for (int64_t c = threadIdx.x; c < H; c += kAdaGenericBlock) {
-      const float code = q.zero_scale ? 0.0f : sym_code(value(c), q, -127.0f, 127.0f);
-      a.out[base + c] = static_cast<int8_t>(__float2int_rn(code));
+      a.out[base + c] = static_cast<int8_t>(q.zero_scale ? 0 : code_exact<false>(value(c), q, -127.0f, 127.0f));
     }
   }
 }

@@ -8,6 +8,7 @@
 // cached values are per-device launch facts (SM count, occupancy).
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -84,35 +85,138 @@ dq_status launch_status() {
   return e == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- launch shapes
+
+// Launch-shape targets (compile-time, so a build can be tuned without any
+// runtime switch).
+#ifndef DQ_TARGET_TPR
+#define DQ_TARGET_TPR 128  // preferred threads per row group
+#endif
+#ifndef DQ_CTA_THREADS
+#define DQ_CTA_THREADS 256  // row groups per CTA = DQ_CTA_THREADS / tpr
+#endif
+#ifndef DQ_RING_BYTES
+#define DQ_RING_BYTES 65536  // shared-memory row ring per CTA
+#endif
+
+// Row-group shape: VPT 16-byte vectors per thread, tpr threads per row. Picks
+// the VPT in {1, 2, 3, 4, 6, 8} (up to max_vpt) that wastes the fewest lanes, then the tpr closest to the
+// target (at most max_tpr).
+struct GroupShape {
+  int vpt;
+  int tpr;
+};
+
+GroupShape pick_shape(int64_t nvec, int max_tpr, int max_vpt) {
+  GroupShape best{0, 0};
+  double best_eff = -1.0;
+  static const int kVpts[6] = {1, 2, 3, 4, 6, 8};
+  for (int vpt : kVpts) {
+    if (vpt > max_vpt) continue;
+    const int64_t tpr = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
+    if (tpr > max_tpr) continue;
+    const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
+    const bool better = eff > best_eff + 1e-9 ||
+                        (eff > best_eff - 1e-9 &&
+                         std::llabs(tpr - DQ_TARGET_TPR) < std::llabs(best.tpr - DQ_TARGET_TPR));
+    if (better) {
+      best_eff = eff;
+      best = GroupShape{vpt, static_cast<int>(tpr)};
+    }
+  }
+  return best;
+}
+
+// Ring geometry: `groups` row groups per CTA, `stages` row buffers per group,
+// about DQ_RING_BYTES of rows per CTA (so several CTAs fit on an SM and each
+// keeps rows in flight while it computes).
+struct RingShape {
+  int groups;
+  int stages;
+  uint32_t stride;
+};
+
+RingShape pick_ring(int tpr, int64_t row_bytes, int max_block) {
+  RingShape r;
+  const int cta = DQ_CTA_THREADS < max_block ? DQ_CTA_THREADS : max_block;
+  r.groups = tpr >= cta ? 1 : cta / tpr;
+  if (r.groups > 15) r.groups = 15;  // named barriers 1..15
+  r.stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
+  int64_t s = DQ_RING_BYTES / (static_cast<int64_t>(r.groups) * r.stride);
+  s = s < 2 ? 2 : (s > 8 ? 8 : s);
+  r.stages = static_cast<int>(s);
+  return r;
+}
+
+constexpr size_t kMaxDynamicSmem = 200 * 1024;
+
+// Allow `kernel` the dynamic shared memory it needs (once per kernel/device).
+bool allow_smem(const void* kernel, int device) {
+  struct Entry {
+    const void* k;
+    int device;
+  };
+  static Entry done[256];
+  static int used = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i) {
+    if (done[i].k == kernel && done[i].device == device) return true;
+  }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kMaxDynamicSmem)) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (used < 256) done[used++] = Entry{kernel, device};
+  return true;
+}
+
 // ---------------------------------------------------------------- dynamic quant dispatch
+
+// Warp-per-row ring geometry: DQ_WARP_STAGES row buffers per warp, warps per
+// CTA so that a CTA holds about DQ_WARP_CTA_BYTES of rows.
+#ifndef DQ_WARP_STAGES
+#define DQ_WARP_STAGES 2
+#endif
+#ifndef DQ_WARP_CTA_BYTES
+#define DQ_WARP_CTA_BYTES 98304
+#endif
+
+template <typename InT, int MODE, int OUT, int SMK>
+dq_status launch_dq_warp(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
+  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK>);
+  const size_t smem = dq::dq_smem_bytes(a.groups, a.stages, a.stage_stride, a.group_index ? a.num_groups : 0);
+  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
+  const int block = 32 * a.groups;
+  const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
+  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
+  const int grid = static_cast<int>(wanted < resident ? wanted : resident);
+  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK><<<grid, block, smem, stream>>>(a);
+  return launch_status();
+}
 
 template <typename InT, int MODE, int OUT>
 dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t stream) {
   const int device = current_device();
   const int sms = sm_count(device);
-  const int64_t nvec = a.cols >> 3;
-  const size_t smem = a.group_index ? static_cast<size_t>(a.num_groups) * sizeof(int32_t) : 0;
   if (vector_ok) {
-    const int vpt = nvec >= 128 ? 4 : (nvec >= 64 ? 2 : 1);
-    const int64_t tpr64 = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
-    if (tpr64 <= dq::kMaxBlock) {
-      a.tpr = static_cast<int>(tpr64);
-      a.groups = a.tpr >= 256 ? 1 : 256 / a.tpr;
-      const int block = a.tpr * a.groups;
-      const void* k = vpt == 4 ? reinterpret_cast<const void*>(dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 4>)
-                    : vpt == 2 ? reinterpret_cast<const void*>(dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 2>)
-                               : reinterpret_cast<const void*>(dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 1>);
-      const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
-      const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
-      const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-      if (vpt == 4) {
-        dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 4><<<grid, block, smem, stream>>>(a);
-      } else if (vpt == 2) {
-        dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 2><<<grid, block, smem, stream>>>(a);
-      } else {
-        dq::dynamic_quant_vec_kernel<InT, MODE, OUT, 1><<<grid, block, smem, stream>>>(a);
+    const int64_t row_bytes = a.cols * 2;
+    const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
+    const int stages = DQ_WARP_STAGES;
+    int64_t warps = DQ_WARP_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
+    warps = warps < 1 ? 1 : (warps > 16 ? 16 : warps);
+    a.groups = static_cast<int>(warps);
+    a.stages = stages;
+    a.stage_stride = stride;
+    a.tpr = 32;
+    if (dq::dq_smem_bytes(a.groups, stages, stride, a.group_index ? a.num_groups : 0) <= kMaxDynamicSmem) {
+      if (a.smooth == nullptr) return launch_dq_warp<InT, MODE, OUT, dq::kSmNone>(a, device, sms, stream);
+      switch (a.smooth_dtype) {
+        case dq::kF32: return launch_dq_warp<InT, MODE, OUT, dq::kSmF32>(a, device, sms, stream);
+        case dq::kF16: return launch_dq_warp<InT, MODE, OUT, dq::kSmF16>(a, device, sms, stream);
+        default: return launch_dq_warp<InT, MODE, OUT, dq::kSmBF16>(a, device, sms, stream);
       }
-      return launch_status();
     }
   }
   const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_generic_kernel<InT, MODE, OUT>);
@@ -132,6 +236,91 @@ dq_status dispatch_mode_out(const dq::RowQuantArgs& a, dq_mode mode, dq_dtype y_
   }
   return four ? launch_dynamic_quant<InT, dq::kAsym, dq::kOutInt4>(a, vec, s)
               : launch_dynamic_quant<InT, dq::kAsym, dq::kOutInt8>(a, vec, s);
+}
+
+// ---------------------------------------------------------------- AdaLayerNormQuant dispatch
+
+size_t ada_table_bytes(int64_t batch, int64_t hidden) { return static_cast<size_t>(batch * hidden) * 8; }
+
+// Affine-table kernel (ordinary launch), then the row kernel as its
+// programmatic dependent (it may start before the table is finished and waits
+// for it with griddepcontrol.wait).
+dq_status launch_ada_table(const dq::AdaArgs& a, int sms, cudaStream_t stream) {
+  const int64_t total = a.batch * a.hidden;
+  int64_t grid = (total + dq::kTableBlock - 1) / dq::kTableBlock;
+  if (grid > 2 * sms) grid = 2 * sms;
+  dq::ada_affine_table_kernel<<<static_cast<int>(grid), dq::kTableBlock, 0, stream>>>(a);
+  return launch_status();
+}
+
+template <typename InT, int VPT>
+dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream) {
+  void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_tma_kernel<InT, VPT>;
+  const void* k = reinterpret_cast<const void*>(kfn);
+  const size_t smem = dq::ada_smem_bytes(a.groups, a.stages, a.stage_stride);
+  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
+  const int block = a.tpr * a.groups;
+  const int64_t rows = a.batch * a.seq;
+  const int64_t wanted = (rows + a.groups - 1) / a.groups;
+  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
+  const int grid = static_cast<int>(wanted < resident ? wanted : resident);
+  dq_status st = launch_ada_table(a, sms, stream);
+  if (st != DQ_OK) return st;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, a) != cudaSuccess) {
+    cudaGetLastError();
+    return DQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
+template <typename InT>
+dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
+  const int device = current_device();
+  const int sms = sm_count(device);
+  if (vector_ok) {
+    const GroupShape gs = pick_shape(a.hidden >> 3, dq::kAdaMaxBlock, 4);
+    if (gs.vpt > 0) {
+      const RingShape rs = pick_ring(gs.tpr, a.hidden * 2, dq::kAdaMaxBlock);
+      a.tpr = gs.tpr;
+      a.groups = rs.groups;
+      a.stages = rs.stages;
+      a.stage_stride = rs.stride;
+      if (dq::ada_smem_bytes(rs.groups, rs.stages, rs.stride) <= kMaxDynamicSmem) {
+        switch (gs.vpt) {
+          case 1: return launch_ada_tma<InT, 1>(a, device, sms, stream);
+          case 2: return launch_ada_tma<InT, 2>(a, device, sms, stream);
+          case 3: return launch_ada_tma<InT, 3>(a, device, sms, stream);
+          default: return launch_ada_tma<InT, 4>(a, device, sms, stream);
+        }
+      }
+    }
+  }
+  dq_status st = launch_ada_table(a, sms, stream);
+  if (st != DQ_OK) return st;
+  const void* k = reinterpret_cast<const void*>(dq::ada_layernorm_quant_generic_kernel<InT>);
+  const int64_t rows = a.batch * a.seq;
+  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, dq::kAdaGenericBlock, 0, device);
+  const int grid = static_cast<int>(rows < resident ? rows : resident);
+  dq::ada_layernorm_quant_generic_kernel<InT><<<grid, dq::kAdaGenericBlock, 0, stream>>>(a);
+  return launch_status();
+}
+
+dq_status check_ada(int64_t batch, int64_t seq, int64_t hidden, dq_dtype x_dtype, dq_dtype param_dtype) {
+  if (batch < 0 || seq < 0 || hidden < 1) return DQ_ERR_BAD_SHAPE;
+  if (hidden > (int64_t(1) << 31) || batch > (int64_t(1) << 40) || seq > (int64_t(1) << 40)) return DQ_ERR_BAD_SHAPE;
+  if (batch > 0 && seq > (int64_t(1) << 40) / batch) return DQ_ERR_BAD_SHAPE;
+  if (!is_input_float(x_dtype) || !is_param_float(param_dtype)) return DQ_ERR_BAD_DTYPE;
+  return DQ_OK;
 }
 
 dq_status check_sizes(int64_t rows, int64_t cols, dq_dtype x_dtype, dq_mode mode, dq_dtype y_dtype,
@@ -210,11 +399,22 @@ dq_status dq_dynamic_quant(const void* x, dq_dtype x_dtype, int64_t rows, int64_
   a.offset = mode == DQ_ASYMMETRIC ? offset : nullptr;
   a.status = needed > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
 
-  // vector path: 16-byte rows of x and naturally aligned code vectors
+  // bulk-copy path: 16-byte rows of x, 16-byte aligned smooth rows and
+  // naturally aligned code vectors; anything else takes the generic kernel
   const uintptr_t y_align = y_dtype == DQ_INT8 ? 8 : 4;
-  const bool vec = (cols % 8) == 0 && aligned(x, 16) && aligned(y, y_align);
+  const bool vec = (cols % 8) == 0 && aligned(x, 16) && aligned(y, y_align) &&
+                   (smooth == nullptr || aligned(smooth, 16));
   if (x_dtype == DQ_F16) return dispatch_mode_out<__half>(a, mode, y_dtype, vec, stream);
   return dispatch_mode_out<__nv_bfloat16>(a, mode, y_dtype, vec, stream);
+}
+
+dq_status dq_ada_layernorm_quant_get_workspace_size(int64_t batch, int64_t seq, int64_t hidden, dq_dtype x_dtype,
+                                                    dq_dtype param_dtype, size_t* workspace_bytes) {
+  if (workspace_bytes == nullptr) return DQ_ERR_NULL_POINTER;
+  const dq_status st = check_ada(batch, seq, hidden, x_dtype, param_dtype);
+  if (st != DQ_OK) return st;
+  *workspace_bytes = batch * seq > 0 ? ada_table_bytes(batch, hidden) : 0;
+  return DQ_OK;
 }
 
 dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype, int64_t batch, int64_t seq, int64_t hidden,
@@ -222,20 +422,18 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype, int64_t batch,
                                  const void* bias, const void* smooth, dq_dtype param_dtype, float epsilon,
                                  int8_t* out, float* quant_scale, void* workspace, size_t workspace_bytes,
                                  cudaStream_t stream) {
-  (void)workspace;
-  (void)workspace_bytes;
-  if (batch < 0 || seq < 0 || hidden < 1) return DQ_ERR_BAD_SHAPE;
-  if (hidden > (int64_t(1) << 31) || batch > (int64_t(1) << 40) || seq > (int64_t(1) << 40))
-    return DQ_ERR_BAD_SHAPE;
-  if (!is_input_float(x_dtype) || !is_param_float(param_dtype)) return DQ_ERR_BAD_DTYPE;
+  const dq_status st = check_ada(batch, seq, hidden, x_dtype, param_dtype);
+  if (st != DQ_OK) return st;
   if (!std::isfinite(epsilon) || epsilon < 0.0f) return DQ_ERR_BAD_ARGUMENT;
   const int64_t rows = batch * seq;
   if (rows == 0) return DQ_OK;
   if (x == nullptr || ada_scale == nullptr || ada_shift == nullptr || out == nullptr || quant_scale == nullptr)
     return DQ_ERR_NULL_POINTER;
+  if (workspace == nullptr || workspace_bytes < ada_table_bytes(batch, hidden)) return DQ_ERR_WORKSPACE_TOO_SMALL;
   const size_t ps = float_size(param_dtype);
   if (!aligned(x, 2) || !aligned(quant_scale, 4) || !aligned(ada_scale, ps) || !aligned(ada_shift, ps) ||
-      (weight && !aligned(weight, ps)) || (bias && !aligned(bias, ps)) || (smooth && !aligned(smooth, ps)))
+      (weight && !aligned(weight, ps)) || (bias && !aligned(bias, ps)) || (smooth && !aligned(smooth, ps)) ||
+      !aligned(workspace, 16))
     return DQ_ERR_MISALIGNED;
 
   dq::AdaArgs a{};
@@ -250,39 +448,13 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype, int64_t batch,
   a.smooth = smooth;
   a.param_dtype = static_cast<int>(param_dtype);
   a.epsilon = epsilon;
+  a.inv_hidden = 1.0 / static_cast<double>(hidden);
+  a.table = static_cast<float*>(workspace);
   a.out = out;
   a.quant_scale = quant_scale;
-
-  const int device = current_device();
-  const int sms = sm_count(device);
-  const int64_t nvec = hidden / 8;
-  const bool vec = (hidden % 8) == 0 && aligned(x, 16) && aligned(out, 8) && nvec <= dq::kAdaMaxBlock;
-  if (vec) {
-    a.tpr = static_cast<int>((nvec + 31) / 32 * 32);
-    a.groups = a.tpr >= 256 ? 1 : 256 / a.tpr;
-    const int block = a.tpr * a.groups;
-    const void* k = x_dtype == DQ_F16 ? reinterpret_cast<const void*>(dq::ada_layernorm_quant_vec_kernel<__half>)
-                                      : reinterpret_cast<const void*>(dq::ada_layernorm_quant_vec_kernel<__nv_bfloat16>);
-    const int64_t wanted = (rows + a.groups - 1) / a.groups;
-    const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, 0, device);
-    const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-    if (x_dtype == DQ_F16) {
-      dq::ada_layernorm_quant_vec_kernel<__half><<<grid, block, 0, stream>>>(a);
-    } else {
-      dq::ada_layernorm_quant_vec_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(a);
-    }
-    return launch_status();
-  }
-  const void* k = x_dtype == DQ_F16 ? reinterpret_cast<const void*>(dq::ada_layernorm_quant_generic_kernel<__half>)
-                                    : reinterpret_cast<const void*>(dq::ada_layernorm_quant_generic_kernel<__nv_bfloat16>);
-  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, dq::kAdaGenericBlock, 0, device);
-  const int grid = static_cast<int>(rows < resident ? rows : resident);
-  if (x_dtype == DQ_F16) {
-    dq::ada_layernorm_quant_generic_kernel<__half><<<grid, dq::kAdaGenericBlock, 0, stream>>>(a);
-  } else {
-    dq::ada_layernorm_quant_generic_kernel<__nv_bfloat16><<<grid, dq::kAdaGenericBlock, 0, stream>>>(a);
-  }
-  return launch_status();
+  const bool vec = (hidden % 8) == 0 && aligned(x, 16) && aligned(out, 8);
+  if (x_dtype == DQ_F16) return launch_ada<__half>(a, vec, stream);
+  return launch_ada<__nv_bfloat16>(a, vec, stream);
 }
 
 }  // extern "C"

@@ -2,11 +2,13 @@
 //
 // The quantization arithmetic follows the formulas of aclnnDynamicQuantV2
 // ("Formula") bit for bit: IEEE binary32, one rounding per operation,
-// round-half-to-even. Division by the row scale is the costly part, so it is
-// done as a multiply by the correctly rounded reciprocal plus a proof-carrying
-// guard band: whenever the product lies too close to a rounding tie for the
-// two to be guaranteed to round alike, the element is redone with the true
-// IEEE division. The bounds are derived next to each quantizer below.
+// round-half-to-even. The division by the row scale is evaluated with
+// Markstein's method (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
+// y = RN(1/s), q0 = RN(v*y) and two FMA corrections q <- RN(q + RN(v - s*q)*y)
+// the result is the correctly rounded RN(v/s) whenever the remainder v - s*q
+// does not underflow. The rows that could break that precondition in a way
+// that matters are sent to the IEEE division instead (see RowQuant).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -17,6 +19,12 @@ namespace dq {
 
 // Element type tags (mirror the dq_dtype values of the C ABI).
 enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
+
+// Compile-time flag carried through generic lambdas.
+template <bool B>
+struct BoolTag {
+  static constexpr bool value = B;
+};
 
 // ---------------------------------------------------------------- widening
 
@@ -88,44 +96,64 @@ __device__ __forceinline__ void group_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- packed reductions
+
+// Row max / absmax / min on the raw 16-bit values, two per instruction
+// (comparisons are exact, so this equals the fp32 reduction of the widened
+// values). Used when no smooth scales are applied.
+template <typename T>
+struct Packed;
+
+template <>
+struct Packed<__half> {
+  using T2 = __half2;
+  static __device__ __forceinline__ T2 from_bits(uint32_t b) { return *reinterpret_cast<const T2*>(&b); }
+  static __device__ __forceinline__ T2 lowest() { return from_bits(0xFC00FC00u); }  // -inf, -inf
+  static __device__ __forceinline__ T2 highest() { return from_bits(0x7C007C00u); }  // +inf, +inf
+  static __device__ __forceinline__ T2 zero() { return from_bits(0u); }
+  static __device__ __forceinline__ T2 vmax(T2 a, T2 b) { return __hmax2(a, b); }
+  static __device__ __forceinline__ T2 vmin(T2 a, T2 b) { return __hmin2(a, b); }
+  static __device__ __forceinline__ float hi_lo_max(T2 a) { return fmaxf(__low2float(a), __high2float(a)); }
+  static __device__ __forceinline__ float hi_lo_min(T2 a) { return fminf(__low2float(a), __high2float(a)); }
+};
+
+template <>
+struct Packed<__nv_bfloat16> {
+  using T2 = __nv_bfloat162;
+  static __device__ __forceinline__ T2 from_bits(uint32_t b) { return *reinterpret_cast<const T2*>(&b); }
+  static __device__ __forceinline__ T2 lowest() { return from_bits(0xFF80FF80u); }
+  static __device__ __forceinline__ T2 highest() { return from_bits(0x7F807F80u); }
+  static __device__ __forceinline__ T2 zero() { return from_bits(0u); }
+  static __device__ __forceinline__ T2 vmax(T2 a, T2 b) { return __hmax2(a, b); }
+  static __device__ __forceinline__ T2 vmin(T2 a, T2 b) { return __hmin2(a, b); }
+  static __device__ __forceinline__ float hi_lo_max(T2 a) { return fmaxf(__low2float(a), __high2float(a)); }
+  static __device__ __forceinline__ float hi_lo_min(T2 a) { return fminf(__low2float(a), __high2float(a)); }
+};
+
 // ---------------------------------------------------------------- quantizers
 
-// Symmetric code of one element: RNE(fl(v / scale)), given rcp = RN(1/scale)
-// and a normal, non-zero scale.
-//
-// Bound: with q = v/scale exact, fl(v/scale) = q(1+d1) and
-// t = fl(v * rcp) = q(1+d2)(1+d3), |di| <= u = 2^-24, so
-// |t - fl(v/scale)| <= 3.0001 u |q|. Here |v| <= absmax and
-// scale >= (absmax/D)(1-u) give |q| <= D(1+2u), D in {127, 7}: the distance is
-// at most 3.0001 * 127.0001 * 2^-24 < 2.3e-5 < 2^-15. If t is farther than
-// kSymGuard = 2^-14 from every half-integer, fl(v/scale) lies strictly on the
-// same side of the same half-integer, so both round to the same integer.
-// Otherwise the element is recomputed with the IEEE division.
-constexpr float kSymGuard = 6.103515625e-05f;  // 2^-14
-
-// Asymmetric code: RNE(fl(fl(v / scale) + offset)), given rcp = RN(1/scale).
-// Fast value t = fl(v * rcp + offset) (one fused rounding).
-// Bound: with q = v/scale and w = q + offset exact,
-// t = (w + q d2)(1 + d3) and z = fl(fl(q) + offset) = (w + q d1)(1 + d4), so
-// |t - z| <= 2u|q| + 2u|w| + O(u^2). Elements lie in [min, max], hence
-// w is within [offset_opt - scale_opt, offset_opt] up to rounding noise, so
-// |w| <= 129 and |q| <= |offset| + 129; the distance is below
-// 2u(|offset| + 260). The guard 4u(|offset| + 260) = 2^-22 (|offset| + 260)
-// keeps a factor 2 of margin. Rows whose guard exceeds 1/4 use the IEEE path
-// for every element.
-__device__ __forceinline__ float asym_half_minus_guard(float offset) {
-  const float guard = 2.384185791015625e-07f * (fabsf(offset) + 260.0f);  // 2^-22 (|off|+260)
-  return guard > 0.25f ? -1.0f : 0.5f - guard;
-}
-
 // Per-row quantization constants.
+//   exact_row: use the IEEE division for every element of the row. Set when
+//     scale < 2^-40 or the offset is not finite. Otherwise (scale >= 2^-40) an
+//     element whose remainder can underflow has |v| < 2^-100, hence a quotient
+//     below 2^-60 in magnitude: it rounds to code 0 (symmetric), or it cannot
+//     move fl(q + offset) across a rounding midpoint that decides a code
+//     (asymmetric: a decisive z needs |offset| > 1/4, whose neighbouring
+//     midpoints are at least 2^-27 away), so Markstein's result is exact
+//     wherever it is used.
+//   clamp: saturate before rounding (asymmetric rows with |offset| >= 2^20,
+//     where rounding noise of the offset can push the row's extremes past the
+//     code range; below 2^20 every code provably lies in range).
 struct RowQuant {
-  float scale;        // written to scale[r]
-  float offset;       // asymmetric only
-  float rcp;          // RN(1/scale) when the fast path is valid
-  float half_minus_guard;  // |t - rint(t)| above this => exact recompute; -1 => always
-  bool zero_scale;    // scale == 0: constant codes
+  float scale;   // written to scale[r]
+  float offset;  // asymmetric only
+  float rcp;     // RN(1 / scale) (IEEE reciprocal)
+  bool zero_scale;
+  bool exact_row;
+  bool clamp;
 };
+
+constexpr float kMarksteinMinScale = 9.094947017729282e-13f;  // 2^-40
 
 // symmetric: scale = absmax / D (IEEE division)
 __device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
@@ -133,10 +161,9 @@ __device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
   q.scale = __fdiv_rn(absmax, divisor);
   q.offset = 0.0f;
   q.zero_scale = (q.scale == 0.0f);
-  // A subnormal scale has too little precision for the bound above.
-  const bool fast = q.scale >= 1.17549435e-38f;
-  q.rcp = fast ? __frcp_rn(q.scale) : 0.0f;
-  q.half_minus_guard = fast ? 0.5f - kSymGuard : -1.0f;
+  q.exact_row = !q.zero_scale && !(q.scale >= kMarksteinMinScale);
+  q.rcp = (q.zero_scale || q.exact_row) ? 0.0f : __frcp_rn(q.scale);
+  q.clamp = false;
   return q;
 }
 
@@ -145,55 +172,99 @@ __device__ __forceinline__ RowQuant make_asym(float mx, float mn, float scale_op
   RowQuant q;
   q.scale = __fdiv_rn(__fsub_rn(mx, mn), scale_opt);
   q.zero_scale = (q.scale == 0.0f);
+  q.clamp = false;
   if (q.zero_scale) {
     q.offset = offset_opt;
     q.rcp = 0.0f;
-    q.half_minus_guard = -1.0f;
+    q.exact_row = false;
     return q;
   }
   q.offset = __fsub_rn(offset_opt, __fdiv_rn(mx, q.scale));
-  const bool fast = q.scale >= 1.17549435e-38f && isfinite(q.offset);
-  q.rcp = fast ? __frcp_rn(q.scale) : 0.0f;
-  q.half_minus_guard = fast ? asym_half_minus_guard(q.offset) : -1.0f;
+  q.exact_row = !(q.scale >= kMarksteinMinScale) || !isfinite(q.offset);
+  q.rcp = q.exact_row ? 0.0f : __frcp_rn(q.scale);
+  q.clamp = !(fabsf(q.offset) < 1048576.0f);  // 2^20
   return q;
 }
 
-// One symmetric code, rounded integer value as float (in [lo, hi]).
-__device__ __forceinline__ float sym_code(float v, const RowQuant& q, float lo, float hi) {
-  const float t = __fmul_rn(v, q.rcp);
-  const float rt = rintf(t);
-  if (fabsf(__fsub_rn(t, rt)) <= q.half_minus_guard) return rt;  // proven equal to the exact path
-  const float exact = rintf(__fdiv_rn(v, q.scale));
-  return fminf(fmaxf(exact, lo), hi);
+// ---------------------------------------------------------------- rounding
+
+// Adding 1.5 * 2^23 to a binary32 t with |t| < 2^22 lands in [2^23, 2^24),
+// where the spacing is exactly 1, so the RN sum is M + RNE(t) (M is even, so
+// ties still go to even). Subtracting M back is exact. The low bits of the
+// sum's pattern hold RNE(t) in two's complement (0x4B400000 + RNE(t)), so a
+// code's byte or nibble can be taken from the pattern directly. This keeps
+// the rounding on the FMA pipe instead of the conversion unit.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Codes of 8 elements (magic-sum patterns, see kRoundMagic) on a row whose
+// RowQuant has neither zero_scale nor exact_row set:
+//   q = RN(v / scale) by Markstein's method (5 FMA-pipe operations),
+//   z = RN(q + offset) (asymmetric), optional saturation, then RNE via the
+//   magic add. Branch-free; every element gets the formulas' exact result.
+template <bool kAsym, bool kClamp>
+__device__ __forceinline__ void quant8(const float (&v)[8], const RowQuant& q, float lo, float hi,
+                                       uint32_t (&bits)[8]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float2 vv = make_float2(v[2 * p], v[2 * p + 1]);
+    const float2 q0 = __fmul2_rn(vv, f2(q.rcp));
+    const float2 r0 = __ffma2_rn(f2(-q.scale), q0, vv);
+    const float2 q1 = __ffma2_rn(r0, f2(q.rcp), q0);
+    const float2 r1 = __ffma2_rn(f2(-q.scale), q1, vv);
+    float2 z = __ffma2_rn(r1, f2(q.rcp), q1);  // RN(v / scale)
+    if (kAsym) z = __fadd2_rn(z, f2(q.offset));
+    if (kClamp) {
+      z.x = fminf(fmaxf(z.x, lo), hi);
+      z.y = fminf(fmaxf(z.y, lo), hi);
+    }
+    const float2 sum = __fadd2_rn(z, f2(kRoundMagic));
+    bits[2 * p] = __float_as_uint(sum.x);
+    bits[2 * p + 1] = __float_as_uint(sum.y);
+  }
 }
 
-__device__ __forceinline__ float asym_code(float v, const RowQuant& q, float lo, float hi) {
-  const float t = __fmaf_rn(v, q.rcp, q.offset);
-  const float rt = rintf(t);
-  if (fabsf(__fsub_rn(t, rt)) <= q.half_minus_guard) return fminf(fmaxf(rt, lo), hi);
-  const float exact = rintf(__fadd_rn(__fdiv_rn(v, q.scale), q.offset));
-  return fminf(fmaxf(exact, lo), hi);
+// The formulas' own arithmetic for 8 elements with the IEEE division (then
+// + offset), RNE and saturation to [lo, hi]: the path of exact_row rows.
+template <bool kAsym>
+__device__ __forceinline__ void quant8_exact(const float (&v)[8], const RowQuant& q, float lo, float hi,
+                                          uint32_t (&bits)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float z = __fdiv_rn(v[j], q.scale);
+    if (kAsym) z = __fadd_rn(z, q.offset);
+    z = fminf(fmaxf(rintf(z), lo), hi);
+    bits[j] = __float_as_uint(__fadd_rn(z, kRoundMagic));
+  }
+}
+
+// Scalar version (generic kernels): the code as an int.
+template <bool kAsym>
+__device__ __forceinline__ int code_exact(float v, const RowQuant& q, float lo, float hi) {
+  float z = __fdiv_rn(v, q.scale);
+  if (kAsym) z = __fadd_rn(z, q.offset);
+  return __float2int_rn(fminf(fmaxf(rintf(z), lo), hi));
 }
 
 // ---------------------------------------------------------------- packing
 
-// 8 int8 codes (as integral floats) -> 8 bytes.
-__device__ __forceinline__ uint2 pack_int8x8(const float (&c)[8]) {
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) b[i] = static_cast<uint32_t>(__float2int_rn(c[i])) & 0xFFu;
+// 8 codes (low bytes of the patterns) -> 8 int8 bytes.
+__device__ __forceinline__ uint2 pack8_int8(const uint32_t (&b)[8]) {
   uint2 r;
-  r.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  r.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  r.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+  r.y = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
   return r;
 }
 
-// 8 int4 codes -> one 32-bit word, element k in bits 4k..4k+3.
-__device__ __forceinline__ uint32_t pack_int4x8(const float (&c)[8]) {
-  uint32_t w = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) w |= (static_cast<uint32_t>(__float2int_rn(c[i])) & 0xFu) << (4 * i);
-  return w;
+// 8 codes (low nibbles of the patterns) -> one word, element k in bits 4k..4k+3.
+__device__ __forceinline__ uint32_t pack8_int4(const uint32_t (&b)[8]) {
+  const uint2 bytes = pack8_int8(b);
+  uint32_t lo = bytes.x & 0x0F0F0F0Fu;
+  uint32_t hi = bytes.y & 0x0F0F0F0Fu;
+  lo |= lo >> 4;  // byte0 = c0 | c1 << 4, byte2 = c2 | c3 << 4
+  hi |= hi >> 4;
+  return __byte_perm(lo, hi, 0x6420);
 }
 
 }  // namespace dq

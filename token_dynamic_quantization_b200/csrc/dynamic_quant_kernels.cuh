@@ -1,21 +1,21 @@
 // Per-token dynamic quantization kernels (aclnnDynamicQuantV2, "Formula" and
 // "Description"), sm_100a.
 //
-// The operation is HBM-bound: each row is read once (2 B/element) and its
-// codes written once (1 or 0.5 B/element). Design:
-//   * vector kernel: a persistent grid; each CTA holds `groups` row groups of
-//     `tpr` threads, and each group walks a contiguous range of rows. A thread
-//     owns VPT 16-byte vectors (8 elements each) of the row, so the whole row
-//     sits in registers; the next row's vectors are loaded while the current
-//     one is reduced and quantized (one row of prefetch per group). Smooth
-//     scales for the thread's columns live in registers and are reloaded only
-//     when the MoE expert changes. Reductions: warp shuffles, then the
-//     group's warps through shared memory behind a named barrier.
+// The operation moves 2 B/element in and 1 or 0.5 B/element out, so it is
+// bounded by HBM bandwidth if each element costs only a handful of
+// instructions. Two kernels:
+//   * bulk-copy kernel (rows whose bytes, smooth-scale rows and code rows are
+//     suitably aligned): one warp per row, persistent grid. Each warp keeps a
+//     ring of shared-memory row buffers filled with cp.async.bulk (TMA)
+//     copies of its next rows, reduces the row (warp shuffles only), derives
+//     the row constants, then quantizes the row with Markstein's division
+//     (branch-free, exact) and packs codes with byte permutes.
 //   * generic kernel: any cols / alignment; one CTA per row (grid-strided),
 //     two passes over the row (the second one mostly hits L2).
 #pragma once
 
 #include "dq_device.cuh"
+#include "tma_pipeline.cuh"
 
 namespace dq {
 
@@ -34,8 +34,10 @@ struct RowQuantArgs {
   float* scale;
   float* offset;               // asymmetric only
   uint32_t* status;            // workspace status word (with a group index)
-  int tpr;                     // threads per row group (vector kernel)
-  int groups;                  // row groups per CTA (vector kernel)
+  int tpr;                     // threads per row group (bulk-copy kernel)
+  int groups;                  // row groups per CTA (bulk-copy kernel)
+  int stages;                  // ring depth per group (bulk-copy kernel)
+  uint32_t stage_stride;       // bytes between stages (multiple of 128)
 };
 
 template <int MODE, int OUT>
@@ -44,7 +46,7 @@ struct QuantConsts {
   static constexpr float kDivisor = MODE == kSym ? (kFour ? 7.0f : 127.0f) : (kFour ? 15.0f : 255.0f);
   static constexpr float kOffsetOpt = MODE == kSym ? 0.0f : (kFour ? 7.0f : 127.0f);
   static constexpr float kLo = MODE == kSym ? (kFour ? -7.0f : -127.0f) : (kFour ? -8.0f : -128.0f);
-  static constexpr float kHi = MODE == kSym ? (kFour ? 7.0f : 127.0f) : (kFour ? 7.0f : 127.0f);
+  static constexpr float kHi = kFour ? 7.0f : 127.0f;
 };
 
 // Status word of a MoE call: written by exactly one thread per launch, so it
@@ -72,171 +74,269 @@ __device__ __forceinline__ int expert_of(const int32_t* gi, int n, int64_t r) {
   return lo;
 }
 
-// ============================================================ vector kernel
+// Shared memory of the bulk-copy kernel: [groups][stages] row buffers, then
+// [groups][stages] mbarriers, then the MoE group index.
+__host__ __device__ inline size_t dq_smem_bytes(int groups, int stages, uint32_t stride, int num_groups) {
+  return static_cast<size_t>(groups) * stages * stride + static_cast<size_t>(groups) * stages * 8 +
+         static_cast<size_t>(num_groups) * 4;
+}
 
-constexpr int kMaxBlock = 512;
+// ============================================================ bulk-copy kernel
 
-template <typename InT, int MODE, int OUT, int VPT>
-__global__ void __launch_bounds__(kMaxBlock)
-dynamic_quant_vec_kernel(const RowQuantArgs a) {
-  using C = QuantConsts<MODE, OUT>;
-  __shared__ float red[2][kMaxBlock / 32][2];
-  extern __shared__ int32_t gi_smem[];
+// Smooth-scale storage kinds (template parameter of the bulk-copy kernel).
+enum : int { kSmNone = 0, kSmF32 = 1, kSmF16 = 2, kSmBF16 = 3 };
 
-  write_group_status(a);
-  const bool moe = a.group_index != nullptr;
-  if (moe) {
-    for (int i = threadIdx.x; i < a.num_groups; i += blockDim.x) gi_smem[i] = a.group_index[i];
-    __syncthreads();
+// Smooth scales of one 8-column vector of `row` (16-byte aligned), widened to
+// fp32. The table is small and shared by every row, so it is read through L1.
+template <int SMK>
+__device__ __forceinline__ void load_smooth8(const void* row, int vi, float (&s)[8]) {
+  if (SMK == kSmF32) {
+    const float4* p = static_cast<const float4*>(row) + 2 * vi;
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    s[0] = a.x; s[1] = a.y; s[2] = a.z; s[3] = a.w;
+    s[4] = b.x; s[5] = b.y; s[6] = b.z; s[7] = b.w;
+  } else if (SMK == kSmBF16) {
+    InTraits<__nv_bfloat16>::widen8(__ldg(static_cast<const uint4*>(row) + vi), s);
+  } else if (SMK == kSmF16) {
+    InTraits<__half>::widen8(__ldg(static_cast<const uint4*>(row) + vi), s);
   }
+}
 
-  const int tpr = a.tpr;
-  const int g = threadIdx.x / tpr;
-  const int lane_g = threadIdx.x - g * tpr;
+// input = x (* smooth) for one 8-element vector held in `raw`.
+template <typename InT, int SMK>
+__device__ __forceinline__ void input8(const uint4& raw, const void* smooth_row, int vi, float (&v)[8]) {
+  InTraits<InT>::widen8(raw, v);
+  if (SMK != kSmNone) {
+    float sm[8];
+    load_smooth8<SMK>(smooth_row, vi, sm);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 pr = __fmul2_rn(make_float2(v[2 * p], v[2 * p + 1]), make_float2(sm[2 * p], sm[2 * p + 1]));
+      v[2 * p] = pr.x;
+      v[2 * p + 1] = pr.y;
+    }
+  }
+}
+
+// Rows whose RowQuant has exact_row set (scale below 2^-40, or a non-finite
+// offset): every element of the row with the IEEE division. Out of line and
+// reached only for such rows.
+template <typename InT, int MODE, int OUT, int SMK>
+__device__ __noinline__ void quantize_row_exact(const uint4* srow, const void* smooth_row, RowQuant q, int lane,
+                                                int nvec, uint8_t* yrow) {
+  using C = QuantConsts<MODE, OUT>;
+  for (int vi = lane; vi < nvec; vi += 32) {
+    float v[8];
+    input8<InT, SMK>(srow[vi], smooth_row, vi, v);
+    uint32_t bits[8];
+    quant8_exact<MODE == kAsym>(v, q, C::kLo, C::kHi, bits);
+    if (OUT == kOutInt8) {
+      reinterpret_cast<uint2*>(yrow)[vi] = pack8_int8(bits);
+    } else {
+      reinterpret_cast<unsigned int*>(yrow)[vi] = pack8_int4(bits);
+    }
+  }
+}
+
+// One warp per row. Each warp owns a ring of `stages` shared-memory row
+// buffers that its lane 0 keeps filled with cp.async.bulk (TMA) copies of the
+// warp's next rows; a stage is refilled as soon as the warp has finished with
+// its row. Per row: pass 1 reads the row from shared memory and reduces it
+// (packed 16-bit pairs without smooth scales), the warp reduces with shuffles,
+// one lane derives the row constants, and pass 2 reads the row again,
+// quantizes (Markstein division, magic rounding) and stores 8 codes per lane
+// and vector. No block-level barrier is used after set-up.
+constexpr int kWarpKernelMaxThreads = 512;
+
+template <typename InT, int MODE, int OUT, int SMK>
+__global__ void __launch_bounds__(kWarpKernelMaxThreads, 1)
+dynamic_quant_tma_kernel(const RowQuantArgs a) {
+  using C = QuantConsts<MODE, OUT>;
+  using P = Packed<InT>;
+  constexpr bool kA = MODE == kAsym;
+  extern __shared__ __align__(128) uint8_t smem[];
+
   const int warp = threadIdx.x >> 5;
-  const int warp_g0 = (g * tpr) >> 5;  // first warp of this group
-  const int nwarps_g = tpr >> 5;
   const int lane = threadIdx.x & 31;
+  const int S = a.stages;
+  const int W = a.groups;  // warps per CTA
+  const uint32_t stride = a.stage_stride;
+  const size_t ring_bytes = static_cast<size_t>(W) * S * stride;
+  uint8_t* ring = smem + static_cast<size_t>(warp) * S * stride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes) + warp * S;
+  int32_t* gi_s = reinterpret_cast<int32_t*>(smem + ring_bytes + static_cast<size_t>(W) * S * 8);
 
-  const int64_t workers = static_cast<int64_t>(gridDim.x) * a.groups;
-  const int64_t worker = static_cast<int64_t>(blockIdx.x) * a.groups + g;
+  const bool moe = a.group_index != nullptr;
+  if (threadIdx.x == 0) {
+    uint64_t* all = reinterpret_cast<uint64_t*>(smem + ring_bytes);
+    for (int i = 0; i < W * S; ++i) mbar_init(all + i, 1);
+    fence_mbarrier_init();
+  }
+  if (moe) {
+    for (int i = threadIdx.x; i < a.num_groups; i += blockDim.x) gi_s[i] = a.group_index[i];
+  }
+  __syncthreads();
+  write_group_status(a);
+
+  const int64_t workers = static_cast<int64_t>(gridDim.x) * W;
+  const int64_t worker = static_cast<int64_t>(blockIdx.x) * W + warp;
   const int64_t r_begin = worker * a.rows / workers;
   const int64_t r_end = (worker + 1) * a.rows / workers;
-  if (r_begin >= r_end) return;  // whole group idle (its barrier is group-local)
+  const int n = static_cast<int>(r_end - r_begin);  // rows of this warp (< 2^31 by validation)
+  if (n <= 0) return;
 
-  const int64_t nvec = a.cols >> 3;
-  const uint4* __restrict__ xv = static_cast<const uint4*>(a.x);
+  const int nvec = static_cast<int>(a.cols >> 3);
+  const uint32_t row_bytes = static_cast<uint32_t>(a.cols) * 2u;
+  const uint64_t policy = lane == 0 ? l2_evict_first_policy() : 0;
+  const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  int issued = 0;
+  auto issue_into = [&](int st) {  // lane 0 only
+    mbar_arrive_expect_tx(bars + st, row_bytes);
+    bulk_copy_g2s(ring + static_cast<size_t>(st) * stride, x_next, row_bytes, bars + st, policy);
+    x_next += row_bytes;
+    ++issued;
+  };
+  if (lane == 0) {
+    for (int st = 0; st < S && st < n; ++st) issue_into(st);
+  }
 
-  // smooth scales of this thread's columns
-  float sm[VPT][8];
-  const bool has_smooth = a.smooth != nullptr;
-  int cur_expert = -1;
-  int64_t expert_end = -1;  // rows < expert_end belong to cur_expert
-  auto load_smooth = [&](int e) {
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const int64_t vi = lane_g + static_cast<int64_t>(k) * tpr;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        sm[k][j] = vi < nvec ? load_param(a.smooth, a.smooth_dtype, e * a.cols + vi * 8 + j) : 1.0f;
+  const size_t smooth_row_bytes = static_cast<size_t>(a.cols) * (SMK == kSmF32 ? 4 : 2);
+  const uint8_t* smooth_row = static_cast<const uint8_t*>(a.smooth);
+  int cur_expert = moe ? -1 : 0;
+  int64_t expert_end = moe ? -1 : INT64_MAX;
+  const int64_t y_row_bytes = OUT == kOutInt8 ? a.cols : (a.cols >> 1);
+  uint8_t* yrow = static_cast<uint8_t*>(a.y) + r_begin * y_row_bytes;
+
+  int st = 0;
+  uint32_t phase = 0;
+  for (int i = 0; i < n; ++i, yrow += y_row_bytes) {
+    const int64_t r = r_begin + i;
+    const bool arrived = mbar_wait_parity(bars + st, phase);
+    if (__any_sync(0xffffffffu, !arrived)) {
+      // A row copy never completed (not a data-dependent condition): mark this
+      // and the warp's remaining rows with NaN scales, drain, and stop.
+      for (int64_t rr = r + lane; rr < r_end; rr += 32) a.scale[rr] = __int_as_float(0x7fc00000);
+      if (lane == 0) {
+        int s2 = st;
+        uint32_t ph = phase;
+        for (int j = i + 1; j < issued; ++j) {
+          s2 = s2 + 1 == S ? 0 : s2 + 1;
+          if (s2 == 0) ph ^= 1u;
+          mbar_wait_parity(bars + s2, ph);
+        }
       }
+      return;
     }
-  };
-  if (has_smooth && !moe) load_smooth(0);
-
-  uint4 cur[VPT], nxt[VPT];
-  auto load_row = [&](int64_t r, uint4 (&buf)[VPT]) {
-    const uint4* p = xv + r * nvec;
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const int64_t vi = lane_g + static_cast<int64_t>(k) * tpr;
-      if (vi < nvec) buf[k] = __ldcs(p + vi);
-    }
-  };
-  load_row(r_begin, cur);
-
-  int parity = 0;
-  for (int64_t r = r_begin; r < r_end; ++r) {
-    if (r + 1 < r_end) load_row(r + 1, nxt);
+    const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(st) * stride);
 
     bool row_valid = true;
     if (moe) {
       if (r >= expert_end) {
-        const int e = expert_of(gi_smem, a.num_groups, r);
-        if (e >= a.num_groups) {
-          row_valid = false;
-          expert_end = INT64_MAX;
-          cur_expert = a.num_groups;
-        } else {
-          expert_end = gi_smem[e];
-          if (e != cur_expert) {
-            load_smooth(e);
-            cur_expert = e;
-          }
-        }
+        const int e = expert_of(gi_s, a.num_groups, r);
+        cur_expert = e;
+        expert_end = e < a.num_groups ? static_cast<int64_t>(gi_s[e]) : INT64_MAX;
+        smooth_row = static_cast<const uint8_t*>(a.smooth) + static_cast<size_t>(e < a.num_groups ? e : 0) *
+                                                                 smooth_row_bytes;
       }
       row_valid = cur_expert < a.num_groups;
     }
 
-    // widen (+ smooth multiply), reduce
-    float v[VPT][8];
-    float m0 = MODE == kSym ? 0.0f : -INFINITY;  // absmax or max
-    float m1 = INFINITY;                         // min (asymmetric)
+    // ---- pass 1: reduce
+    float m0, m1;
+    if (SMK != kSmNone) {
+      m0 = kA ? -INFINITY : 0.0f;
+      m1 = INFINITY;
+#pragma unroll 4
+      for (int vi = lane; vi < nvec; vi += 32) {
+        float v[8];
+        input8<InT, SMK>(srow[vi], smooth_row, vi, v);
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const int64_t vi = lane_g + static_cast<int64_t>(k) * tpr;
-      InTraits<InT>::widen8(cur[k], v[k]);
-      if (has_smooth) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[k][j] = __fmul_rn(v[k][j], sm[k][j]);
-      }
-      if (vi < nvec) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (MODE == kSym) {
-            m0 = fmaxf(m0, fabsf(v[k][j]));
+        for (int p = 0; p < 4; ++p) {
+          if (kA) {
+            m0 = fmaxf(m0, fmaxf(v[2 * p], v[2 * p + 1]));
+            m1 = fminf(m1, fminf(v[2 * p], v[2 * p + 1]));
           } else {
-            m0 = fmaxf(m0, v[k][j]);
-            m1 = fminf(m1, v[k][j]);
+            m0 = fmaxf(m0, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
           }
         }
       }
+    } else {
+      typename P::T2 hmax = kA ? P::lowest() : P::zero();
+      typename P::T2 hmin = P::highest();
+#pragma unroll 4
+      for (int vi = lane; vi < nvec; vi += 32) {
+        const uint4 raw = srow[vi];
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          if (kA) {
+            hmax = P::vmax(hmax, P::from_bits(w[p]));
+            hmin = P::vmin(hmin, P::from_bits(w[p]));
+          } else {
+            hmax = P::vmax(hmax, P::from_bits(w[p] & 0x7FFF7FFFu));
+          }
+        }
+      }
+      m0 = P::hi_lo_max(hmax);
+      m1 = kA ? P::hi_lo_min(hmin) : INFINITY;
     }
     m0 = warp_max(m0);
-    if (MODE == kAsym) m1 = warp_min(m1);
-    if (nwarps_g > 1) {
-      if (lane == 0) {
-        red[parity][warp][0] = m0;
-        red[parity][warp][1] = m1;
-      }
-      group_barrier(1 + g, tpr);
-      m0 = red[parity][warp_g0][0];
-      m1 = red[parity][warp_g0][1];
-      for (int w = 1; w < nwarps_g; ++w) {
-        m0 = fmaxf(m0, red[parity][warp_g0 + w][0]);
-        if (MODE == kAsym) m1 = fminf(m1, red[parity][warp_g0 + w][1]);
-      }
-      parity ^= 1;
-    }
+    if (kA) m1 = warp_min(m1);
 
-    RowQuant q = MODE == kSym ? make_sym(m0, C::kDivisor) : make_asym(m0, m1, C::kDivisor, C::kOffsetOpt);
+    RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
     if (!row_valid) {
       q.scale = 0.0f;
       q.offset = 0.0f;
     }
-    if (lane_g == 0) {
+    if (lane == 0) {
       __stcs(a.scale + r, q.scale);
-      if (MODE == kAsym) __stcs(a.offset + r, q.offset);
+      if (kA) __stcs(a.offset + r, q.offset);
     }
 
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const int64_t vi = lane_g + static_cast<int64_t>(k) * tpr;
-      if (vi >= nvec) continue;
-      float c[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (!row_valid) {
-          c[j] = 0.0f;
-        } else if (q.zero_scale) {
-          c[j] = C::kOffsetOpt;
-        } else if (MODE == kSym) {
-          c[j] = sym_code(v[k][j], q, C::kLo, C::kHi);
+    // ---- pass 2: quantize and store
+    if (!row_valid || q.zero_scale) {
+      const uint32_t cb = __float_as_uint(__fadd_rn(row_valid ? C::kOffsetOpt : 0.0f, kRoundMagic));
+      const uint32_t bits[8] = {cb, cb, cb, cb, cb, cb, cb, cb};
+      for (int vi = lane; vi < nvec; vi += 32) {
+        if (OUT == kOutInt8) {
+          __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
         } else {
-          c[j] = asym_code(v[k][j], q, C::kLo, C::kHi);
+          __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
         }
       }
-      if (OUT == kOutInt8) {
-        uint2* yp = reinterpret_cast<uint2*>(static_cast<int8_t*>(a.y) + r * a.cols) + vi;
-        __stcs(yp, pack_int8x8(c));
+    } else if (q.exact_row) {
+      quantize_row_exact<InT, MODE, OUT, SMK>(srow, smooth_row, q, lane, nvec, yrow);
+    } else {
+      auto pass2 = [&](auto clamp_tag) {
+        constexpr bool kClamp = decltype(clamp_tag)::value;
+#pragma unroll 4
+        for (int vi = lane; vi < nvec; vi += 32) {
+          float v[8];
+          input8<InT, SMK>(srow[vi], smooth_row, vi, v);
+          uint32_t bits[8];
+          quant8<kA, kClamp>(v, q, C::kLo, C::kHi, bits);
+          if (OUT == kOutInt8) {
+            __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
+          } else {
+            __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
+          }
+        }
+      };
+      if (kA && q.clamp) {
+        pass2(BoolTag<true>{});
       } else {
-        uint32_t* yp = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(a.y) + r * (a.cols >> 1)) + vi;
-        __stcs(reinterpret_cast<unsigned int*>(yp), pack_int4x8(c));
+        pass2(BoolTag<false>{});
       }
     }
 
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) cur[k] = nxt[k];
+    // The warp is done with this stage: refill it with the warp's next row.
+    __syncwarp();
+    if (lane == 0 && issued < n) {
+      fence_proxy_async_smem();
+      issue_into(st);
+    }
+    st = st + 1 == S ? 0 : st + 1;
+    if (st == 0) phase ^= 1u;
   }
 }
 
@@ -248,6 +348,7 @@ template <typename InT, int MODE, int OUT>
 __global__ void __launch_bounds__(kGenericBlock)
 dynamic_quant_generic_kernel(const RowQuantArgs a) {
   using C = QuantConsts<MODE, OUT>;
+  constexpr bool kA = MODE == kAsym;
   __shared__ float red[kGenericBlock / 32][2];
   write_group_status(a);
   const bool moe = a.group_index != nullptr;
@@ -269,21 +370,21 @@ dynamic_quant_generic_kernel(const RowQuantArgs a) {
       if (a.smooth != nullptr) v = __fmul_rn(v, load_param(a.smooth, a.smooth_dtype, srow * a.cols + c));
       return v;
     };
-    float m0 = MODE == kSym ? 0.0f : -INFINITY;
+    float m0 = kA ? -INFINITY : 0.0f;
     float m1 = INFINITY;
     if (row_valid) {
       for (int64_t c = threadIdx.x; c < a.cols; c += kGenericBlock) {
         const float v = input(c);
-        if (MODE == kSym) {
-          m0 = fmaxf(m0, fabsf(v));
-        } else {
+        if (kA) {
           m0 = fmaxf(m0, v);
           m1 = fminf(m1, v);
+        } else {
+          m0 = fmaxf(m0, fabsf(v));
         }
       }
     }
     m0 = warp_max(m0);
-    if (MODE == kAsym) m1 = warp_min(m1);
+    if (kA) m1 = warp_min(m1);
     if (lane == 0) {
       red[warp][0] = m0;
       red[warp][1] = m1;
@@ -293,24 +394,23 @@ dynamic_quant_generic_kernel(const RowQuantArgs a) {
     m1 = red[0][1];
     for (int w = 1; w < kWarps; ++w) {
       m0 = fmaxf(m0, red[w][0]);
-      if (MODE == kAsym) m1 = fminf(m1, red[w][1]);
+      if (kA) m1 = fminf(m1, red[w][1]);
     }
     __syncthreads();  // red[] is rewritten by the next row
 
-    RowQuant q = MODE == kSym ? make_sym(m0, C::kDivisor) : make_asym(m0, m1, C::kDivisor, C::kOffsetOpt);
+    RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
     if (!row_valid) {
       q.scale = 0.0f;
       q.offset = 0.0f;
     }
     if (threadIdx.x == 0) {
       a.scale[r] = q.scale;
-      if (MODE == kAsym) a.offset[r] = q.offset;
+      if (kA) a.offset[r] = q.offset;
     }
     auto code = [&](int64_t c) -> int {
       if (!row_valid) return 0;
       if (q.zero_scale) return static_cast<int>(C::kOffsetOpt);
-      const float v = input(c);
-      return __float2int_rn(MODE == kSym ? sym_code(v, q, C::kLo, C::kHi) : asym_code(v, q, C::kLo, C::kHi));
+      return code_exact<kA>(input(c), q, C::kLo, C::kHi);
     };
     if (OUT == kOutInt8) {
       int8_t* yr = static_cast<int8_t*>(a.y) + base;

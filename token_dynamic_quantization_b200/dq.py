@@ -53,6 +53,8 @@ _lib.dq_get_workspace_size.restype = _ci
 _lib.dq_dynamic_quant.argtypes = [_vp, _ci, _i64, _i64, _vp, _ci, _vp, _i32, _ci, _ci, _vp, _vp, _vp, _vp, _sz,
                                   _vp]
 _lib.dq_dynamic_quant.restype = _ci
+_lib.dq_ada_layernorm_quant_get_workspace_size.argtypes = [_i64, _i64, _i64, _ci, _ci, ctypes.POINTER(_sz)]
+_lib.dq_ada_layernorm_quant_get_workspace_size.restype = _ci
 _lib.dq_ada_layernorm_quant.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp, _vp,
                                         _vp, _sz, _vp]
 _lib.dq_ada_layernorm_quant.restype = _ci
@@ -75,6 +77,15 @@ def dq_status_string(status: int) -> str:
 def dq_get_workspace_size(rows: int, cols: int, x_dtype: int, mode: int, y_dtype: int, num_groups: int) -> int:
     out = _sz(0)
     st = _lib.dq_get_workspace_size(rows, cols, x_dtype, mode, y_dtype, num_groups, ctypes.byref(out))
+    if st != DQ_OK:
+        raise DQError(st)
+    return int(out.value)
+
+
+def dq_ada_layernorm_quant_get_workspace_size(batch: int, seq: int, hidden: int, x_dtype: int,
+                                              param_dtype: int) -> int:
+    out = _sz(0)
+    st = _lib.dq_ada_layernorm_quant_get_workspace_size(batch, seq, hidden, x_dtype, param_dtype, ctypes.byref(out))
     if st != DQ_OK:
         raise DQError(st)
     return int(out.value)
@@ -171,10 +182,12 @@ def dynamic_quant(x, smooth=None, group_index=None, mode: str = "symmetric", y_d
 
 
 def ada_layernorm_quant(x, ada_scale, ada_shift, weight=None, bias=None, smooth=None, epsilon: float = 1e-6,
-                        out=None, stream=None, check: bool = True):
+                        out=None, workspace=None, stream=None, check: bool = True):
     """Fused AdaLayerNorm + symmetric INT8 quantization of CUDA tensor ``x`` [batch, seq, hidden].
 
     Returns ``(out int8 [batch, seq, hidden], quant_scale float32 [batch, seq])``.
+    ``workspace``: optional preallocated CUDA tensor of at least
+    ``dq_ada_layernorm_quant_get_workspace_size`` bytes (16-byte aligned).
     """
     torch = _torch()
     if x.dim() != 3:
@@ -184,18 +197,22 @@ def ada_layernorm_quant(x, ada_scale, ada_shift, weight=None, bias=None, smooth=
     for name, p in (("ada_shift", ada_shift), ("weight", weight), ("bias", bias), ("smooth", smooth)):
         if p is not None and _dtype_code(p) != pdt:
             raise TypeError(f"{name} must have the dtype of ada_scale")
+    ws_bytes = dq_ada_layernorm_quant_get_workspace_size(batch, seq, hidden, _dtype_code(x), pdt)
     if out is None:
         o = torch.empty((batch, seq, hidden), dtype=torch.int8, device=x.device)
         qs = torch.empty((batch, seq), dtype=torch.float32, device=x.device)
     else:
         o, qs = out
+    if workspace is None and ws_bytes:
+        workspace = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=x.device)
     if stream is None:
         stream = torch.cuda.current_stream(x.device).cuda_stream
     st = dq_ada_layernorm_quant(_dev_ptr(x, "x"), _dtype_code(x), batch, seq, hidden,
                                 _dev_ptr(ada_scale, "ada_scale"), _dev_ptr(ada_shift, "ada_shift"),
                                 _dev_ptr(weight, "weight"), _dev_ptr(bias, "bias"), _dev_ptr(smooth, "smooth"),
                                 pdt, float(epsilon), _dev_ptr(o, "out"), _dev_ptr(qs, "quant_scale"),
-                                None, 0, stream)
+                                _dev_ptr(workspace, "workspace"),
+                                ws_bytes if workspace is not None else 0, stream)
     if check and st != DQ_OK:
         raise DQError(st)
     return o, qs
