@@ -168,32 +168,72 @@ bool allow_smem(const void* kernel, int device) {
     cudaGetLastError();
     return false;
   }
+  // prefer the largest shared-memory carveout: these kernels hold their row
+  // rings there and use little L1 beyond it
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
+    cudaGetLastError();
+  }
   if (used < 256) done[used++] = Entry{kernel, device};
   return true;
 }
 
 // ---------------------------------------------------------------- dynamic quant dispatch
 
-// Warp-per-row ring geometry: DQ_WARP_STAGES row buffers per warp, warps per
-// CTA so that a CTA holds about DQ_WARP_CTA_BYTES of rows.
+// Row-group geometry of the bulk-copy DynamicQuant kernel: a group of
+// tpr = 32 * G threads owns a row, VPT in {2, 4, 8} vectors per thread; the
+// shape wasting the fewest lanes wins, then the one whose VPT is closest to
+// DQ_TARGET_VPT. DQ_WARP_STAGES row buffers per group; groups per CTA so that
+// a CTA holds about DQ_WARP_CTA_BYTES of rows.
+#ifndef DQ_TARGET_VPT
+#define DQ_TARGET_VPT 8
+#endif
 #ifndef DQ_WARP_STAGES
 #define DQ_WARP_STAGES 2
 #endif
 #ifndef DQ_WARP_CTA_BYTES
-#define DQ_WARP_CTA_BYTES 98304
+#define DQ_WARP_CTA_BYTES 65536
 #endif
 
-template <typename InT, int MODE, int OUT, int SMK>
-dq_status launch_dq_warp(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
-  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK>);
+GroupShape pick_dq_shape(int64_t nvec) {
+  GroupShape best{0, 0};
+  double best_eff = -1.0;
+  static const int kVpts[3] = {2, 4, 8};
+  for (int vpt : kVpts) {
+    const int64_t warps = (nvec + 32 * vpt - 1) / (32 * vpt);
+    if (warps > 16) continue;
+    const int64_t tpr = warps * 32;
+    const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
+    const bool better = eff > best_eff + 1e-9 ||
+                        (eff > best_eff - 1e-9 && std::abs(vpt - DQ_TARGET_VPT) < std::abs(best.vpt - DQ_TARGET_VPT));
+    if (better) {
+      best_eff = eff;
+      best = GroupShape{vpt, static_cast<int>(tpr)};
+    }
+  }
+  return best;
+}
+
+template <typename InT, int MODE, int OUT, int SMK, int VPT>
+dq_status launch_dq_tma(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
+  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT>);
   const size_t smem = dq::dq_smem_bytes(a.groups, a.stages, a.stage_stride, a.group_index ? a.num_groups : 0);
   if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
-  const int block = 32 * a.groups;
+  const int block = a.tpr * a.groups;
   const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
   const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK><<<grid, block, smem, stream>>>(a);
+  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT><<<grid, block, smem, stream>>>(a);
   return launch_status();
+}
+
+template <typename InT, int MODE, int OUT, int SMK>
+dq_status launch_dq_vpt(dq::RowQuantArgs a, int vpt, int device, int sms, cudaStream_t stream) {
+  switch (vpt) {
+    case 2: return launch_dq_tma<InT, MODE, OUT, SMK, 2>(a, device, sms, stream);
+    case 4: return launch_dq_tma<InT, MODE, OUT, SMK, 4>(a, device, sms, stream);
+    default: return launch_dq_tma<InT, MODE, OUT, SMK, 8>(a, device, sms, stream);
+  }
 }
 
 template <typename InT, int MODE, int OUT>
@@ -201,21 +241,26 @@ dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t 
   const int device = current_device();
   const int sms = sm_count(device);
   if (vector_ok) {
-    const int64_t row_bytes = a.cols * 2;
-    const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
-    const int stages = DQ_WARP_STAGES;
-    int64_t warps = DQ_WARP_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
-    warps = warps < 1 ? 1 : (warps > 16 ? 16 : warps);
-    a.groups = static_cast<int>(warps);
-    a.stages = stages;
-    a.stage_stride = stride;
-    a.tpr = 32;
-    if (dq::dq_smem_bytes(a.groups, stages, stride, a.group_index ? a.num_groups : 0) <= kMaxDynamicSmem) {
-      if (a.smooth == nullptr) return launch_dq_warp<InT, MODE, OUT, dq::kSmNone>(a, device, sms, stream);
-      switch (a.smooth_dtype) {
-        case dq::kF32: return launch_dq_warp<InT, MODE, OUT, dq::kSmF32>(a, device, sms, stream);
-        case dq::kF16: return launch_dq_warp<InT, MODE, OUT, dq::kSmF16>(a, device, sms, stream);
-        default: return launch_dq_warp<InT, MODE, OUT, dq::kSmBF16>(a, device, sms, stream);
+    const GroupShape gs = pick_dq_shape(a.cols >> 3);
+    if (gs.vpt > 0) {
+      const int64_t row_bytes = a.cols * 2;
+      const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
+      const int stages = DQ_WARP_STAGES;
+      int64_t groups = DQ_WARP_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
+      const int64_t max_groups = dq::kWarpKernelMaxThreads / gs.tpr;
+      groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
+      groups = groups > 15 ? 15 : groups;  // named barriers 1..15
+      a.groups = static_cast<int>(groups);
+      a.stages = stages;
+      a.stage_stride = stride;
+      a.tpr = gs.tpr;
+      if (dq::dq_smem_bytes(a.groups, stages, stride, a.group_index ? a.num_groups : 0) <= kMaxDynamicSmem) {
+        if (a.smooth == nullptr) return launch_dq_vpt<InT, MODE, OUT, dq::kSmNone>(a, gs.vpt, device, sms, stream);
+        switch (a.smooth_dtype) {
+          case dq::kF32: return launch_dq_vpt<InT, MODE, OUT, dq::kSmF32>(a, gs.vpt, device, sms, stream);
+          case dq::kF16: return launch_dq_vpt<InT, MODE, OUT, dq::kSmF16>(a, gs.vpt, device, sms, stream);
+          default: return launch_dq_vpt<InT, MODE, OUT, dq::kSmBF16>(a, gs.vpt, device, sms, stream);
+        }
       }
     }
   }

@@ -122,10 +122,10 @@ __device__ __forceinline__ void input8(const uint4& raw, const void* smooth_row,
 // offset): every element of the row with the IEEE division. Out of line and
 // reached only for such rows.
 template <typename InT, int MODE, int OUT, int SMK>
-__device__ __noinline__ void quantize_row_exact(const uint4* srow, const void* smooth_row, RowQuant q, int lane,
-                                                int nvec, uint8_t* yrow) {
+__device__ __noinline__ void quantize_row_exact(const uint4* srow, const void* smooth_row, RowQuant q, int lane_g,
+                                                int tpr, int nvec, uint8_t* yrow) {
   using C = QuantConsts<MODE, OUT>;
-  for (int vi = lane; vi < nvec; vi += 32) {
+  for (int vi = lane_g; vi < nvec; vi += tpr) {
     float v[8];
     input8<InT, SMK>(srow[vi], smooth_row, vi, v);
     uint32_t bits[8];
@@ -138,38 +138,53 @@ __device__ __noinline__ void quantize_row_exact(const uint4* srow, const void* s
   }
 }
 
-// One warp per row. Each warp owns a ring of `stages` shared-memory row
-// buffers that its lane 0 keeps filled with cp.async.bulk (TMA) copies of the
-// warp's next rows; a stage is refilled as soon as the warp has finished with
-// its row. Per row: pass 1 reads the row from shared memory and reduces it
-// (packed 16-bit pairs without smooth scales), the warp reduces with shuffles,
-// one lane derives the row constants, and pass 2 reads the row again,
-// quantizes (Markstein division, magic rounding) and stores 8 codes per lane
-// and vector. No block-level barrier is used after set-up.
+// Row groups of tpr = 32 * G threads, `groups` row groups per CTA. Each group
+// owns a ring of `stages` shared-memory row buffers that its first lane keeps
+// filled with cp.async.bulk (TMA) copies of the group's next rows. A thread
+// owns VPT 16-byte vectors of the row (vector vi = lane_g + k * tpr):
+//   pass 1: copy them from the stage into registers (raw 16-bit values) and
+//     reduce (packed 16-bit pairs without smooth scales; fp32 products with);
+//     the group reduces through warp shuffles and, for G > 1, shared memory
+//     behind its named barrier. That barrier also tells the leader that the
+//     stage has been read by every thread, so the stage is refilled right
+//     away: while a group quantizes one row, its next `stages` rows are in
+//     flight.
+//   pass 2: from registers only: widen (* smooth), Markstein division, magic
+//     rounding, byte-permute packing, one 8-byte (int8) or 4-byte (int4)
+//     store per vector.
 constexpr int kWarpKernelMaxThreads = 512;
+#ifndef DQ_MAX_REGS
+#define DQ_MAX_REGS 96  // registers per thread: leaves room for enough resident warps
+#endif
 
-template <typename InT, int MODE, int OUT, int SMK>
-__global__ void __launch_bounds__(kWarpKernelMaxThreads, 1)
+template <typename InT, int MODE, int OUT, int SMK, int VPT>
+__global__ void __maxnreg__(DQ_MAX_REGS)
 dynamic_quant_tma_kernel(const RowQuantArgs a) {
   using C = QuantConsts<MODE, OUT>;
   using P = Packed<InT>;
   constexpr bool kA = MODE == kAsym;
   extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float red[2][kWarpKernelMaxThreads / 32][2];
 
+  const int tpr = a.tpr;
+  const int g = threadIdx.x / tpr;
+  const int lane_g = threadIdx.x - g * tpr;
   const int warp = threadIdx.x >> 5;
+  const int warp_g0 = (g * tpr) >> 5;
+  const int nwarps_g = tpr >> 5;
   const int lane = threadIdx.x & 31;
   const int S = a.stages;
-  const int W = a.groups;  // warps per CTA
+  const int NG = a.groups;
   const uint32_t stride = a.stage_stride;
-  const size_t ring_bytes = static_cast<size_t>(W) * S * stride;
-  uint8_t* ring = smem + static_cast<size_t>(warp) * S * stride;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes) + warp * S;
-  int32_t* gi_s = reinterpret_cast<int32_t*>(smem + ring_bytes + static_cast<size_t>(W) * S * 8);
+  const size_t ring_bytes = static_cast<size_t>(NG) * S * stride;
+  uint8_t* ring = smem + static_cast<size_t>(g) * S * stride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ring_bytes) + g * S;
+  int32_t* gi_s = reinterpret_cast<int32_t*>(smem + ring_bytes + static_cast<size_t>(NG) * S * 8);
 
   const bool moe = a.group_index != nullptr;
   if (threadIdx.x == 0) {
     uint64_t* all = reinterpret_cast<uint64_t*>(smem + ring_bytes);
-    for (int i = 0; i < W * S; ++i) mbar_init(all + i, 1);
+    for (int i = 0; i < NG * S; ++i) mbar_init(all + i, 1);
     fence_mbarrier_init();
   }
   if (moe) {
@@ -178,25 +193,26 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
   __syncthreads();
   write_group_status(a);
 
-  const int64_t workers = static_cast<int64_t>(gridDim.x) * W;
-  const int64_t worker = static_cast<int64_t>(blockIdx.x) * W + warp;
+  const int64_t workers = static_cast<int64_t>(gridDim.x) * NG;
+  const int64_t worker = static_cast<int64_t>(blockIdx.x) * NG + g;
   const int64_t r_begin = worker * a.rows / workers;
   const int64_t r_end = (worker + 1) * a.rows / workers;
-  const int n = static_cast<int>(r_end - r_begin);  // rows of this warp (< 2^31 by validation)
-  if (n <= 0) return;
+  const int n = static_cast<int>(r_end - r_begin);  // rows of this group (< 2^31 by validation)
+  if (n <= 0) return;  // whole group idle (its barriers are group-local)
 
   const int nvec = static_cast<int>(a.cols >> 3);
   const uint32_t row_bytes = static_cast<uint32_t>(a.cols) * 2u;
-  const uint64_t policy = lane == 0 ? l2_evict_first_policy() : 0;
+  const bool leader = lane_g == 0;
+  const uint64_t policy = leader ? l2_evict_first_policy() : 0;
   const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   int issued = 0;
-  auto issue_into = [&](int st) {  // lane 0 only
+  auto issue_into = [&](int st) {  // leader only
     mbar_arrive_expect_tx(bars + st, row_bytes);
     bulk_copy_g2s(ring + static_cast<size_t>(st) * stride, x_next, row_bytes, bars + st, policy);
     x_next += row_bytes;
     ++issued;
   };
-  if (lane == 0) {
+  if (leader) {
     for (int st = 0; st < S && st < n; ++st) issue_into(st);
   }
 
@@ -209,24 +225,10 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
 
   int st = 0;
   uint32_t phase = 0;
+  int parity = 0;
   for (int i = 0; i < n; ++i, yrow += y_row_bytes) {
     const int64_t r = r_begin + i;
     const bool arrived = mbar_wait_parity(bars + st, phase);
-    if (__any_sync(0xffffffffu, !arrived)) {
-      // A row copy never completed (not a data-dependent condition): mark this
-      // and the warp's remaining rows with NaN scales, drain, and stop.
-      for (int64_t rr = r + lane; rr < r_end; rr += 32) a.scale[rr] = __int_as_float(0x7fc00000);
-      if (lane == 0) {
-        int s2 = st;
-        uint32_t ph = phase;
-        for (int j = i + 1; j < issued; ++j) {
-          s2 = s2 + 1 == S ? 0 : s2 + 1;
-          if (s2 == 0) ph ^= 1u;
-          mbar_wait_parity(bars + s2, ph);
-        }
-      }
-      return;
-    }
     const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(st) * stride);
 
     bool row_valid = true;
@@ -241,39 +243,49 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       row_valid = cur_expert < a.num_groups;
     }
 
-    // ---- pass 1: reduce
+    // ---- pass 1: this thread's vectors into registers, reduce
+    uint4 raw[VPT];
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int vi = lane_g + k * tpr;
+      raw[k] = vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0);
+    }
     float m0, m1;
     if (SMK != kSmNone) {
       m0 = kA ? -INFINITY : 0.0f;
       m1 = INFINITY;
-#pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) {
-        float v[8];
-        input8<InT, SMK>(srow[vi], smooth_row, vi, v);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          if (kA) {
-            m0 = fmaxf(m0, fmaxf(v[2 * p], v[2 * p + 1]));
-            m1 = fminf(m1, fminf(v[2 * p], v[2 * p + 1]));
-          } else {
-            m0 = fmaxf(m0, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
+      for (int k = 0; k < VPT; ++k) {
+        const int vi = lane_g + k * tpr;
+        if (vi < nvec) {
+          float v[8];
+          input8<InT, SMK>(raw[k], smooth_row, vi, v);
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            if (kA) {
+              m0 = fmaxf(m0, fmaxf(v[2 * p], v[2 * p + 1]));
+              m1 = fminf(m1, fminf(v[2 * p], v[2 * p + 1]));
+            } else {
+              m0 = fmaxf(m0, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
+            }
           }
         }
       }
     } else {
       typename P::T2 hmax = kA ? P::lowest() : P::zero();
       typename P::T2 hmin = P::highest();
-#pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) {
-        const uint4 raw = srow[vi];
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          if (kA) {
-            hmax = P::vmax(hmax, P::from_bits(w[p]));
-            hmin = P::vmin(hmin, P::from_bits(w[p]));
-          } else {
-            hmax = P::vmax(hmax, P::from_bits(w[p] & 0x7FFF7FFFu));
+      for (int k = 0; k < VPT; ++k) {
+        if (lane_g + k * tpr < nvec) {
+          const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            if (kA) {
+              hmax = P::vmax(hmax, P::from_bits(w[p]));
+              hmin = P::vmin(hmin, P::from_bits(w[p]));
+            } else {
+              hmax = P::vmax(hmax, P::from_bits(w[p] & 0x7FFF7FFFu));
+            }
           }
         }
       }
@@ -282,61 +294,93 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
     }
     m0 = warp_max(m0);
     if (kA) m1 = warp_min(m1);
+    bool failed;
+    if (nwarps_g > 1) {
+      if (lane == 0) {
+        red[parity][warp][0] = m0;
+        red[parity][warp][1] = m1;
+      }
+      failed = group_barrier_or(1 + g, tpr, !arrived);
+      m0 = red[parity][warp_g0][0];
+      m1 = red[parity][warp_g0][1];
+      for (int w = 1; w < nwarps_g; ++w) {
+        m0 = fmaxf(m0, red[parity][warp_g0 + w][0]);
+        if (kA) m1 = fminf(m1, red[parity][warp_g0 + w][1]);
+      }
+      parity ^= 1;
+    } else {
+      failed = __any_sync(0xffffffffu, !arrived);
+    }
+    if (failed) {
+      // A row copy never completed (not a data-dependent condition): mark this
+      // and the group's remaining rows with NaN scales, drain, and stop.
+      for (int64_t rr = r + lane_g; rr < r_end; rr += tpr) a.scale[rr] = __int_as_float(0x7fc00000);
+      if (leader) {
+        int s2 = st;
+        uint32_t ph = phase;
+        for (int j = i + 1; j < issued; ++j) {
+          s2 = s2 + 1 == S ? 0 : s2 + 1;
+          if (s2 == 0) ph ^= 1u;
+          mbar_wait_parity(bars + s2, ph);
+        }
+      }
+      return;
+    }
 
     RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
+    if (q.exact_row && row_valid && !q.zero_scale) {
+      // rare: the stage is still needed by the out-of-line exact path
+      quantize_row_exact<InT, MODE, OUT, SMK>(srow, smooth_row, q, lane_g, tpr, nvec, yrow);
+      if (nwarps_g > 1) group_barrier(1 + g, tpr); else __syncwarp();
+    }
+    // Every thread of the group has its share of the row in registers (and the
+    // exact path, if taken, is done): refill this stage with the group's next row.
+    if (leader && issued < n) {
+      fence_proxy_async_smem();
+      issue_into(st);
+    }
+    st = st + 1 == S ? 0 : st + 1;
+    if (st == 0) phase ^= 1u;
     if (!row_valid) {
       q.scale = 0.0f;
       q.offset = 0.0f;
     }
-    if (lane == 0) {
+    if (leader) {
       __stcs(a.scale + r, q.scale);
       if (kA) __stcs(a.offset + r, q.offset);
     }
+    if (q.exact_row && row_valid && !q.zero_scale) continue;
 
-    // ---- pass 2: quantize and store
-    if (!row_valid || q.zero_scale) {
-      const uint32_t cb = __float_as_uint(__fadd_rn(row_valid ? C::kOffsetOpt : 0.0f, kRoundMagic));
-      const uint32_t bits[8] = {cb, cb, cb, cb, cb, cb, cb, cb};
-      for (int vi = lane; vi < nvec; vi += 32) {
+    // ---- pass 2: quantize from registers and store
+    const bool constant = !row_valid || q.zero_scale;
+    const uint32_t cb = __float_as_uint(__fadd_rn(row_valid ? C::kOffsetOpt : 0.0f, kRoundMagic));
+    auto pass2 = [&](auto clamp_tag) {
+      constexpr bool kClamp = decltype(clamp_tag)::value;
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        const int vi = lane_g + k * tpr;
+        if (vi >= nvec) continue;
+        uint32_t bits[8];
+        if (constant) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) bits[j] = cb;
+        } else {
+          float v[8];
+          input8<InT, SMK>(raw[k], smooth_row, vi, v);
+          quant8<kA, kClamp>(v, q, C::kLo, C::kHi, bits);
+        }
         if (OUT == kOutInt8) {
           __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
         } else {
           __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
         }
       }
-    } else if (q.exact_row) {
-      quantize_row_exact<InT, MODE, OUT, SMK>(srow, smooth_row, q, lane, nvec, yrow);
+    };
+    if (kA && q.clamp) {
+      pass2(BoolTag<true>{});
     } else {
-      auto pass2 = [&](auto clamp_tag) {
-        constexpr bool kClamp = decltype(clamp_tag)::value;
-#pragma unroll 4
-        for (int vi = lane; vi < nvec; vi += 32) {
-          float v[8];
-          input8<InT, SMK>(srow[vi], smooth_row, vi, v);
-          uint32_t bits[8];
-          quant8<kA, kClamp>(v, q, C::kLo, C::kHi, bits);
-          if (OUT == kOutInt8) {
-            __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
-          } else {
-            __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
-          }
-        }
-      };
-      if (kA && q.clamp) {
-        pass2(BoolTag<true>{});
-      } else {
-        pass2(BoolTag<false>{});
-      }
+      pass2(BoolTag<false>{});
     }
-
-    // The warp is done with this stage: refill it with the warp's next row.
-    __syncwarp();
-    if (lane == 0 && issued < n) {
-      fence_proxy_async_smem();
-      issue_into(st);
-    }
-    st = st + 1 == S ? 0 : st + 1;
-    if (st == 0) phase ^= 1u;
   }
 }
 
