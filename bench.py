@@ -298,7 +298,7 @@ def run_ours(args, world, rank, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    wl = workloads.make(args.workload)
+    wl = workloads.make(args.workload, rows=args.rows)
     nbytes = algorithmic_bytes(wl)
     per_set = wl.tensors["x"].numel() * wl.tensors["x"].element_size() + nbytes
     sets = max(2, math.ceil(3 * L2_BYTES / per_set))
@@ -505,7 +505,7 @@ def run_reference(args, world, rank):
 
     if rank != 0:
         return None
-    wl = workloads.make(args.workload)
+    wl = workloads.make(args.workload, rows=args.rows)
     nbytes = algorithmic_bytes(wl)
     rows = wl.rows
     bytes_per_row = nbytes / rows
@@ -554,6 +554,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--rows", type=int, default=None,
+                    help="smaller row count of the same workload (for quick profiler captures)")
     ap.add_argument("--graph", action="store_true", help="replay the K timed launches as one CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

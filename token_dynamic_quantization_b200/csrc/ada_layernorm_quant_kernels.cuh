@@ -110,13 +110,13 @@ __device__ __noinline__ void ada_quantize_row_exact(const uint4* srow, const flo
 
 // ============================================================ bulk-copy kernel
 
-constexpr int kAdaMaxBlock = 256;
-#ifndef DQ_ADA_MIN_BLOCKS
-#define DQ_ADA_MIN_BLOCKS 3
+constexpr int kAdaMaxBlock = 512;
+#ifndef DQ_ADA_MAX_REGS
+#define DQ_ADA_MAX_REGS 128  // the row share stays in registers across four passes
 #endif
 
 template <typename InT, int VPT>
-__global__ void __launch_bounds__(kAdaMaxBlock, DQ_ADA_MIN_BLOCKS)
+__global__ void __maxnreg__(DQ_ADA_MAX_REGS)
 ada_layernorm_quant_tma_kernel(const AdaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ double red_d[2][2][kAdaMaxBlock / 32];  // [parity][sum|sq][warp]
@@ -196,15 +196,22 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(c_stage) * stride);
 
     // ---- pass 1: load, widen, E(x)
+    constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
     float v[VPT][8];
-    float2 s1 = make_float2(0.0f, 0.0f);
+    float2 acc[NACC];
+#pragma unroll
+    for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = lane_g + k * tpr;
       InTraits<InT>::widen8(vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0), v[k]);  // zero when inactive
-#pragma unroll
-      for (int p = 0; p < 4; ++p) s1 = __fadd2_rn(s1, make_float2(v[k][2 * p], v[k][2 * p + 1]));
+      const float2 s01 = __fadd2_rn(make_float2(v[k][0], v[k][1]), make_float2(v[k][2], v[k][3]));
+      const float2 s23 = __fadd2_rn(make_float2(v[k][4], v[k][5]), make_float2(v[k][6], v[k][7]));
+      acc[k % NACC] = __fadd2_rn(acc[k % NACC], __fadd2_rn(s01, s23));
     }
+#pragma unroll
+    for (int j = 1; j < NACC; ++j) acc[0] = __fadd2_rn(acc[0], acc[j]);
+    const float2 s1 = acc[0];
     double sum = warp_sum(static_cast<double>(s1.x) + static_cast<double>(s1.y));
     bool failed;
     if (nwarps_g > 1) {
@@ -239,7 +246,8 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const float mean_f = __double2float_rn(mean_d);
 
     // ---- pass 2: Var(x), biased, about the double mean
-    float2 s2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const bool active = lane_g + k * tpr < nvec;
@@ -249,9 +257,12 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
         if (!active) d = make_float2(0.0f, 0.0f);
         v[k][2 * p] = d.x;
         v[k][2 * p + 1] = d.y;
-        s2 = __ffma2_rn(d, d, s2);
+        acc[(k + p) % NACC] = __ffma2_rn(d, d, acc[(k + p) % NACC]);
       }
     }
+#pragma unroll
+    for (int j = 1; j < NACC; ++j) acc[0] = __fadd2_rn(acc[0], acc[j]);
+    const float2 s2 = acc[0];
     double sq = warp_sum(static_cast<double>(s2.x) + static_cast<double>(s2.y));
     if (nwarps_g > 1) {
       if (lane == 0) red_d[parity][1][warp] = sq;
@@ -266,7 +277,9 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
 
     // ---- pass 3: y = n * A + B, absmax
-    float amax = 0.0f;
+    float amx[NACC];
+#pragma unroll
+    for (int j = 0; j < NACC; ++j) amx[j] = 0.0f;
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const int vi = lane_g + k * tpr;
@@ -282,10 +295,11 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
               __ffma2_rn(nn, make_float2(Av[2 * p], Av[2 * p + 1]), make_float2(Bv[2 * p], Bv[2 * p + 1]));
           v[k][2 * p] = y.x;
           v[k][2 * p + 1] = y.y;
-          amax = fmaxf(amax, fmaxf(fabsf(y.x), fabsf(y.y)));
         }
+        amx[k % NACC] = fmaxf(amx[k % NACC], absmax8(v[k]));
       }
     }
+    float amax = tree<NACC, true>(amx);
     amax = warp_max(amax);
     if (nwarps_g > 1) {
       if (lane == 0) red_f[parity][warp] = amax;

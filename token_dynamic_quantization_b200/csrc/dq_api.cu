@@ -168,12 +168,8 @@ bool allow_smem(const void* kernel, int device) {
     cudaGetLastError();
     return false;
   }
-  // prefer the largest shared-memory carveout: these kernels hold their row
-  // rings there and use little L1 beyond it
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared) != cudaSuccess) {
-    cudaGetLastError();
-  }
+  // (the shared-memory carveout is left to the driver: the smooth-scale
+  // tables are read through L1 and need it to stay resident)
   if (used < 256) done[used++] = Entry{kernel, device};
   return true;
 }
@@ -328,24 +324,59 @@ dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream
   return launch_status();
 }
 
+// AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8}, fewest wasted lanes,
+// then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
+// three row reductions; the row share stays in registers).
+#ifndef DQ_ADA_TARGET_VPT
+#define DQ_ADA_TARGET_VPT 6
+#endif
+#ifndef DQ_ADA_CTA_BYTES
+#define DQ_ADA_CTA_BYTES 65536
+#endif
+
+GroupShape pick_ada_shape(int64_t nvec) {
+  GroupShape best{0, 0};
+  double best_eff = -1.0;
+  static const int kVpts[5] = {2, 3, 4, 6, 8};
+  for (int vpt : kVpts) {
+    const int64_t warps = (nvec + 32 * vpt - 1) / (32 * vpt);
+    if (warps > 16) continue;
+    const int64_t tpr = warps * 32;
+    const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
+    const bool better = eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && std::abs(vpt - DQ_ADA_TARGET_VPT) <
+                                                                             std::abs(best.vpt - DQ_ADA_TARGET_VPT));
+    if (better) {
+      best_eff = eff;
+      best = GroupShape{vpt, static_cast<int>(tpr)};
+    }
+  }
+  return best;
+}
+
 template <typename InT>
 dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
   const int device = current_device();
   const int sms = sm_count(device);
   if (vector_ok) {
-    const GroupShape gs = pick_shape(a.hidden >> 3, dq::kAdaMaxBlock, 4);
+    const GroupShape gs = pick_ada_shape(a.hidden >> 3);
     if (gs.vpt > 0) {
-      const RingShape rs = pick_ring(gs.tpr, a.hidden * 2, dq::kAdaMaxBlock);
+      const uint32_t stride = static_cast<uint32_t>((a.hidden * 2 + 127) / 128 * 128);
+      const int stages = 2;
+      int64_t groups = DQ_ADA_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
+      const int64_t max_groups = dq::kAdaMaxBlock / gs.tpr;
+      groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
+      groups = groups > 15 ? 15 : groups;
       a.tpr = gs.tpr;
-      a.groups = rs.groups;
-      a.stages = rs.stages;
-      a.stage_stride = rs.stride;
-      if (dq::ada_smem_bytes(rs.groups, rs.stages, rs.stride) <= kMaxDynamicSmem) {
+      a.groups = static_cast<int>(groups);
+      a.stages = stages;
+      a.stage_stride = stride;
+      if (dq::ada_smem_bytes(a.groups, stages, stride) <= kMaxDynamicSmem) {
         switch (gs.vpt) {
-          case 1: return launch_ada_tma<InT, 1>(a, device, sms, stream);
           case 2: return launch_ada_tma<InT, 2>(a, device, sms, stream);
           case 3: return launch_ada_tma<InT, 3>(a, device, sms, stream);
-          default: return launch_ada_tma<InT, 4>(a, device, sms, stream);
+          case 4: return launch_ada_tma<InT, 4>(a, device, sms, stream);
+          case 6: return launch_ada_tma<InT, 6>(a, device, sms, stream);
+          default: return launch_ada_tma<InT, 8>(a, device, sms, stream);
         }
       }
     }

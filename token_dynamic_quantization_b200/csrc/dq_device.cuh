@@ -96,6 +96,43 @@ __device__ __forceinline__ void group_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---------------------------------------------------------------- tree reductions
+
+// Three-input max / min (sm_100a). max and min are exact in any order, so the
+// row reductions use shallow trees instead of one serial chain.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// max |v| of 8 values (depth 3)
+__device__ __forceinline__ float absmax8(const float (&v)[8]) {
+  const float a = fmaxf(fabsf(v[0]), fabsf(v[1])), b = fmaxf(fabsf(v[2]), fabsf(v[3]));
+  const float c = fmaxf(fabsf(v[4]), fabsf(v[5])), d = fmaxf(fabsf(v[6]), fabsf(v[7]));
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+__device__ __forceinline__ float max8(const float (&v)[8]) {
+  return fmaxf(max3(v[0], v[1], v[2]), max3(v[3], v[4], max3(v[5], v[6], v[7])));
+}
+__device__ __forceinline__ float min8(const float (&v)[8]) {
+  return fminf(min3(v[0], v[1], v[2]), min3(v[3], v[4], min3(v[5], v[6], v[7])));
+}
+// combine N partials with a tree
+template <int N, bool kMax>
+__device__ __forceinline__ float tree(float (&p)[N]) {
+#pragma unroll
+  for (int w = 1; w < N; w *= 2) {
+#pragma unroll
+    for (int i = 0; i + w < N; i += 2 * w) p[i] = kMax ? fmaxf(p[i], p[i + w]) : fminf(p[i], p[i + w]);
+  }
+  return p[0];
+}
+
 // ---------------------------------------------------------------- packed reductions
 
 // Row max / absmax / min on the raw 16-bit values, two per instruction

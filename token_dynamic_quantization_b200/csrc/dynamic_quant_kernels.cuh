@@ -251,46 +251,63 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       raw[k] = vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0);
     }
     float m0, m1;
+    constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
     if (SMK != kSmNone) {
-      m0 = kA ? -INFINITY : 0.0f;
-      m1 = INFINITY;
+      float amx[NACC], amn[NACC];
+#pragma unroll
+      for (int j = 0; j < NACC; ++j) {
+        amx[j] = kA ? -INFINITY : 0.0f;
+        amn[j] = INFINITY;
+      }
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
         const int vi = lane_g + k * tpr;
         if (vi < nvec) {
           float v[8];
           input8<InT, SMK>(raw[k], smooth_row, vi, v);
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            if (kA) {
-              m0 = fmaxf(m0, fmaxf(v[2 * p], v[2 * p + 1]));
-              m1 = fminf(m1, fminf(v[2 * p], v[2 * p + 1]));
-            } else {
-              m0 = fmaxf(m0, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
-            }
+          if (kA) {
+            amx[k % NACC] = fmaxf(amx[k % NACC], max8(v));
+            amn[k % NACC] = fminf(amn[k % NACC], min8(v));
+          } else {
+            amx[k % NACC] = fmaxf(amx[k % NACC], absmax8(v));
           }
         }
       }
+      m0 = tree<NACC, true>(amx);
+      m1 = kA ? tree<NACC, false>(amn) : INFINITY;
     } else {
-      typename P::T2 hmax = kA ? P::lowest() : P::zero();
-      typename P::T2 hmin = P::highest();
+      typename P::T2 hmax[NACC], hmin[NACC];
+#pragma unroll
+      for (int j = 0; j < NACC; ++j) {
+        hmax[j] = kA ? P::lowest() : P::zero();
+        hmin[j] = P::highest();
+      }
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
         if (lane_g + k * tpr < nvec) {
           const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            if (kA) {
-              hmax = P::vmax(hmax, P::from_bits(w[p]));
-              hmin = P::vmin(hmin, P::from_bits(w[p]));
-            } else {
-              hmax = P::vmax(hmax, P::from_bits(w[p] & 0x7FFF7FFFu));
-            }
+          if (kA) {
+            hmax[k % NACC] = P::vmax(hmax[k % NACC], P::vmax(P::vmax(P::from_bits(w[0]), P::from_bits(w[1])),
+                                                              P::vmax(P::from_bits(w[2]), P::from_bits(w[3]))));
+            hmin[k % NACC] = P::vmin(hmin[k % NACC], P::vmin(P::vmin(P::from_bits(w[0]), P::from_bits(w[1])),
+                                                              P::vmin(P::from_bits(w[2]), P::from_bits(w[3]))));
+          } else {
+            hmax[k % NACC] = P::vmax(hmax[k % NACC],
+                                     P::vmax(P::vmax(P::from_bits(w[0] & 0x7FFF7FFFu), P::from_bits(w[1] & 0x7FFF7FFFu)),
+                                             P::vmax(P::from_bits(w[2] & 0x7FFF7FFFu), P::from_bits(w[3] & 0x7FFF7FFFu))));
           }
         }
       }
-      m0 = P::hi_lo_max(hmax);
-      m1 = kA ? P::hi_lo_min(hmin) : INFINITY;
+#pragma unroll
+      for (int w = 1; w < NACC; w *= 2) {
+#pragma unroll
+        for (int i = 0; i + w < NACC; i += 2 * w) {
+          hmax[i] = P::vmax(hmax[i], hmax[i + w]);
+          if (kA) hmin[i] = P::vmin(hmin[i], hmin[i + w]);
+        }
+      }
+      m0 = P::hi_lo_max(hmax[0]);
+      m1 = kA ? P::hi_lo_min(hmin[0]) : INFINITY;
     }
     m0 = warp_max(m0);
     if (kA) m1 = warp_min(m1);

@@ -105,24 +105,33 @@ WORKLOADS = (
 )
 
 
-def make(name: str) -> Workload:
-    """Build one of the named workloads (CPU tensors)."""
+def make(name: str, rows: int | None = None) -> Workload:
+    """Build one of the named workloads (CPU tensors).
+
+    ``rows``: optional smaller row count drawn the same way (for quick
+    captures of the same kernel configuration); the MoE group index is drawn
+    for that row count, and for the AdaLayerNorm workload the sequence length
+    shrinks (rows = batch * seq).
+    """
     if name == "sym_int8_f16_64x1024":
-        return Workload(name, "dynamic_quant", {"x": normal((64, 1024), torch.float16, 0)})
+        return Workload(name, "dynamic_quant", {"x": normal((rows or 64, 1024), torch.float16, 0)})
     if name == "sym_int8_smooth_bf16_8192x4096":
-        x = with_outlier_columns(normal((8192, 4096), torch.bfloat16, 0), 0.01, 20.0, 1)
+        r = rows or 8192
+        x = with_outlier_columns(normal((r, 4096), torch.bfloat16, 0), 0.01, 20.0, 1)
         smooth = uniform((4096,), torch.float32, 2, 0.5, 2.0)
         return Workload(name, "dynamic_quant", {"x": x, "smooth": smooth})
     if name == "moe_sym_int8_bf16_32768x7168_e64":
-        x = normal((32768, 7168), torch.bfloat16, 0)
+        r = rows or 32768
+        x = normal((r, 7168), torch.bfloat16, 0)
         smooth = uniform((64, 7168), torch.float32, 2, 0.5, 2.0)
-        gi = moe_group_index(32768, 64, 3)
+        gi = moe_group_index(r, 64, 3)
         return Workload(name, "dynamic_quant", {"x": x, "smooth": smooth, "group_index": gi})
     if name == "asym_int4_f16_16384x8192":
-        x = normal((16384, 8192), torch.float16, 0, mean=0.5, std=2.0)
+        x = normal((rows or 16384, 8192), torch.float16, 0, mean=0.5, std=2.0)
         return Workload(name, "dynamic_quant", {"x": x}, mode="asymmetric", y_dtype="int4")
     if name == "ada_layernorm_quant_bf16_4x4096x3072":
-        b, s, h = 4, 4096, 3072
+        b, h = 4, 3072
+        s = max(1, (rows or 4 * 4096) // b)
         t = {
             "x": normal((b, s, h), torch.bfloat16, 0),
             "ada_scale": normal((b, h), torch.bfloat16, 4, std=0.1),
