@@ -71,6 +71,12 @@ def algorithmic_bytes(wl) -> int:
     return int(total)
 
 
+def launches_per_call(wl) -> int:
+    """Kernels one C-ABI call launches: DynamicQuant one; AdaLayerNormQuant two
+    (the per-batch affine table, then the row kernel)."""
+    return 1 if wl.kind == "dynamic_quant" else 2
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -368,10 +374,11 @@ def run_ours(args, world, rank, local):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if "bf16" in args.workload else "f16",
+            "dtype": "f32",
             "data": "synthetic",
             "config": {
                 "workload": args.workload,
+                "x_dtype": "bf16" if "bf16" in args.workload else "f16",
                 "rows": wl.rows,
                 "cols": wl.cols,
                 "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric",
@@ -391,11 +398,11 @@ def run_ours(args, world, rank, local):
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy kernel)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s",
                 "traffic": traffic,
-                "kernel": "dynamic_quant_vec_kernel" if wl.kind == "dynamic_quant" else
-                "ada_layernorm_quant_vec_kernel",
+                "kernel": "dynamic_quant_tma_kernel" if wl.kind == "dynamic_quant" else
+                "ada_layernorm_quant_tma_kernel (time of the whole call: affine-table kernel included)",
             },
             "clocks": clocks,
-            "gpu_launches": args.steps * world,
+            "gpu_launches": args.steps * launches_per_call(wl),
         }
         if e2e is not None:
             result["e2e"] = e2e
@@ -537,10 +544,11 @@ def run_reference(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16" if "bf16" in args.workload else "f16",
+        "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "rows": rows, "cols": wl.cols,
-                   "rows_per_step": n, "rows_per_s": round(n * args.steps / elapsed, 1)},
+        "config": {"workload": args.workload, "x_dtype": "bf16" if "bf16" in args.workload else "f16",
+                   "rows": rows, "cols": wl.cols, "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric",
+                   "y_dtype": wl.y_dtype, "rows_per_step": n, "rows_per_s": round(n * args.steps / elapsed, 1)},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "reference arm = the CPU oracle (the pages ship no runnable implementation)",

@@ -328,7 +328,7 @@ dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream
 // then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
 // three row reductions; the row share stays in registers).
 #ifndef DQ_ADA_TARGET_VPT
-#define DQ_ADA_TARGET_VPT 6
+#define DQ_ADA_TARGET_VPT 4
 #endif
 #ifndef DQ_ADA_CTA_BYTES
 #define DQ_ADA_CTA_BYTES 65536
