@@ -31,7 +31,9 @@
 //     symmetric INT4 [-7, 7], asymmetric INT8 [-128, 127], asymmetric INT4
 //     [-8, 7] (saturation only removes rounding noise for finite inputs);
 //   * symmetric quantization to INT4/INT32 divides by 7 (= offset_opt of the
-//     4-bit type) rather than 127, since 127 cannot be held in four bits;
+//     4-bit type) rather than 127, since 127 cannot be held in four bits.
+//     The pages fix no value here: parity unpinned for that case (the tests
+//     pin the arithmetic given the divisor, not the divisor itself);
 //   * a symmetric row whose absmax is 0 gets scale 0 and all codes 0; an
 //     asymmetric row whose max equals its min gets scale 0, offset offset_opt
 //     and all codes offset_opt (the row max maps to offset_opt, as the
