@@ -211,6 +211,36 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype,
                                  int8_t* out, float* quant_scale,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Largest batch * hidden that dq_ada_layernorm_quant_noalloc accepts (its
+ * fixed table holds this many 8-byte entries: 1 MiB per device). */
+#define DQ_ADA_NOALLOC_MAX_TABLE 131072
+
+/* dq_ada_layernorm_quant without a workspace argument: the same computation,
+ * results and errors, with the scratch table kept in a fixed device array
+ * inside the library. The pages have no counterpart to this entry point (their
+ * two-phase calls always take a workspace); it exists for callers that cannot
+ * allocate device memory: a plain C host program that links only this
+ * library, or code that runs where allocating would re-enter the caller's own
+ * allocator (for example an out-of-memory handler).
+ *   - Allocates nothing: no cudaMalloc/cudaFree, no library allocation.
+ *   - batch * hidden <= DQ_ADA_NOALLOC_MAX_TABLE, else DQ_ERR_UNSUPPORTED and
+ *     nothing is launched.
+ *   - The first call on each device (with that device current) looks up the
+ *     array's address with cudaGetSymbolAddress and caches it; make that first
+ *     call before any stream capture. A failed lookup returns DQ_ERR_CUDA.
+ *   - Nothing needs clearing beforehand: each call writes every table entry it
+ *     reads.
+ *   - The array is shared by all calls on a device: calls whose executions
+ *     overlap (other streams, other host threads) race on it and must use
+ *     dq_ada_layernorm_quant with separate workspaces instead.
+ * batch * seq == 0 returns DQ_OK without any CUDA call. */
+dq_status dq_ada_layernorm_quant_noalloc(const void* x, dq_dtype x_dtype,
+                                         int64_t batch, int64_t seq, int64_t hidden,
+                                         const void* ada_scale, const void* ada_shift,
+                                         const void* weight, const void* bias, const void* smooth,
+                                         dq_dtype param_dtype, float epsilon,
+                                         int8_t* out, float* quant_scale, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,85 @@
+// dq_ada_layernorm_quant_noalloc: AdaLayerNormQuant with its scratch table in
+// a fixed device array instead of a caller-provided workspace.
+//
+// The AdaLayerNormQuant path needs batch * hidden pairs of fp32 (the folded
+// affine table A, B that the row kernel reads). The regular entry point takes
+// that scratch from the caller. Some callers have no device allocator to get
+// it from: a plain C host program that links only this library, or a hook
+// that runs where allocating would re-enter the caller's own allocator (for
+// example inside an out-of-memory handler). This entry point serves them: the
+// table lives in a file-scope __device__ array of DQ_ADA_NOALLOC_MAX_TABLE
+// entries (8 bytes each, 1 MiB), and the call allocates nothing, neither
+// through CUDA nor through any library.
+//
+// Set-up: the array's device address is looked up with cudaGetSymbolAddress
+// once per device, on the first call made while that device is current, and
+// cached. Every other call only reads the cache.
+//
+// Nothing in the array has to start at zero: every call writes each table
+// entry it reads (the table kernel runs first on the same stream and the row
+// kernel waits for it). The array is shared by all calls on a device, so two
+// calls whose executions overlap (different streams, or different host
+// threads) race on it; such callers use the regular entry point with
+// separate workspaces.
+
+#include <atomic>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "dq.h"
+
+namespace {
+
+// The array has one instance per device (each device loads its own copy of
+// the module); its address is therefore looked up per device.
+static __device__ __align__(256) float2 g_ada_noalloc_table[DQ_ADA_NOALLOC_MAX_TABLE];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_table_addr[kMaxDevices];
+std::mutex g_setup_mutex;
+
+// Device address of this device's table (set up on first use).
+dq_status noalloc_table(void** addr) {
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) {
+    cudaGetLastError();
+    return DQ_ERR_CUDA;
+  }
+  if (device < 0 || device >= kMaxDevices) return DQ_ERR_UNSUPPORTED;
+  void* p = g_table_addr[device].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    p = g_table_addr[device].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      if (cudaGetSymbolAddress(&p, g_ada_noalloc_table) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return DQ_ERR_CUDA;
+      }
+      g_table_addr[device].store(p, std::memory_order_release);
+    }
+  }
+  *addr = p;
+  return DQ_OK;
+}
+
+}  // namespace
+
+extern "C" dq_status dq_ada_layernorm_quant_noalloc(const void* x, dq_dtype x_dtype, int64_t batch, int64_t seq,
+                                                    int64_t hidden, const void* ada_scale, const void* ada_shift,
+                                                    const void* weight, const void* bias, const void* smooth,
+                                                    dq_dtype param_dtype, float epsilon, int8_t* out,
+                                                    float* quant_scale, cudaStream_t stream) {
+  size_t needed = 0;
+  const dq_status st = dq_ada_layernorm_quant_get_workspace_size(batch, seq, hidden, x_dtype, param_dtype, &needed);
+  if (st != DQ_OK) return st;
+  if (needed == 0) return DQ_OK;  // batch * seq == 0: nothing to do, no set-up
+  if (batch > DQ_ADA_NOALLOC_MAX_TABLE / hidden) return DQ_ERR_UNSUPPORTED;  // table larger than the array
+  void* table = nullptr;
+  const dq_status ts = noalloc_table(&table);
+  if (ts != DQ_OK) return ts;
+  return dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias, smooth,
+                                param_dtype, epsilon, out, quant_scale, table,
+                                sizeof(float2) * static_cast<size_t>(DQ_ADA_NOALLOC_MAX_TABLE), stream);
+}

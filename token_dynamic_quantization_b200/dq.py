@@ -42,6 +42,7 @@ DQ_SYMMETRIC, DQ_ASYMMETRIC = 0, 1
 DQ_WS_ROWS_PAST_LAST_GROUP = 0x1
 DQ_WS_GROUP_INDEX_INVALID = 0x2
 DQ_MAX_GROUPS = 1024
+DQ_ADA_NOALLOC_MAX_TABLE = 131072
 
 _vp, _i64, _i32, _f32, _sz, _ci = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float,
                                    ctypes.c_size_t, ctypes.c_int)
@@ -58,6 +59,9 @@ _lib.dq_ada_layernorm_quant_get_workspace_size.restype = _ci
 _lib.dq_ada_layernorm_quant.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp, _vp,
                                         _vp, _sz, _vp]
 _lib.dq_ada_layernorm_quant.restype = _ci
+_lib.dq_ada_layernorm_quant_noalloc.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp,
+                                                _vp, _vp]
+_lib.dq_ada_layernorm_quant_noalloc.restype = _ci
 
 LIBRARY_PATH = _LIB_PATH
 
@@ -104,6 +108,13 @@ def dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift,
     return _lib.dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias,
                                        smooth, param_dtype, epsilon, out, quant_scale, workspace,
                                        workspace_bytes, stream)
+
+
+def dq_ada_layernorm_quant_noalloc(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias, smooth,
+                                   param_dtype, epsilon, out, quant_scale, stream) -> int:
+    """Raw call (no workspace: the library's fixed table). Returns the dq_status."""
+    return _lib.dq_ada_layernorm_quant_noalloc(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias,
+                                               smooth, param_dtype, epsilon, out, quant_scale, stream)
 
 
 # ---------------------------------------------------------------- tensor-level helpers
