@@ -1,12 +1,15 @@
 /* Property check of the division method the CUDA quantizer uses.
  *
- * With y = RN(1/s) (IEEE reciprocal), q0 = RN(v*y) and two FMA corrections
- * q <- RN(q + RN(v - s*q) * y) (P. Markstein, IBM J. Res. Dev. 34(1), 1990),
+ * With the two-term reciprocal y = RN(1/s), y_lo = RN(RN(1 - s*y) * y) (the
+ * residual 1 - s*y is exact; it is checked here too), the first quotient
+ * q0 = RN(v*y + RN(v*y_lo)) and one Markstein correction
+ * q = RN(q0 + RN(v - s*q0) * y) (P. Markstein, IBM J. Res. Dev. 34(1), 1990),
  * the result must equal the IEEE quotient RN(v/s) whenever |v| >= 2^-100 and
  * s >= 2^-40 (the kernel's domain; smaller scales use the IEEE division).
- * Where |v| < 2^-100 the remainder may underflow; there the true quotient must
- * be below 2^-60 in magnitude, and adding any offset with 1/4 < |offset| < 2^20
- * must round the same way for both quotients (so no code can change).
+ * Where |v| < 2^-100 a product or the remainder may underflow; there the true
+ * quotient must be below 2^-60 in magnitude, and adding any offset with
+ * 1/4 < |offset| < 2^20 must round the same way for both quotients (so no
+ * code can change).
  * Samples: uniform quotients, quotients within a few ulps of half-integers and
  * of integers, large quotients, and random bit patterns. The host's binary32
  * division and fmaf are IEEE, as on the GPU.
@@ -26,12 +29,10 @@ static float nudge(float v, int k) {
   for (; k < 0; ++k) v = nextafterf(v, -INFINITY);
   return v;
 }
-static float markstein(float v, float s, float y) {
-  float q = v * y;
-  float r = fmaf(-s, q, v);
-  q = fmaf(r, y, q);
-  r = fmaf(-s, q, v);
-  return fmaf(r, y, q);
+static float quotient(float v, float s, float y, float y_lo) {
+  const float q0 = fmaf(v, y, v * y_lo);
+  const float r = fmaf(-s, q0, v);
+  return fmaf(r, y, q0);
 }
 
 int main(int argc, char** argv) {
@@ -40,6 +41,12 @@ int main(int argc, char** argv) {
   for (long i = 0; i < n; ++i) {
     const float s = from_bits(((87u + (uint32_t)(rnd() % 140)) << 23) | (uint32_t)(rnd() & 0x7FFFFF));
     const float y = 1.0f / s;
+    const float e = fmaf(-s, y, 1.0f);
+    if ((double)e != 1.0 - (double)s * (double)y) {
+      printf("violation: residual 1 - s*y not exact for s=%a\n", s);
+      ++violations;
+    }
+    const float y_lo = e * y;
     float v;
     switch (rnd() % 5) {
       case 0: v = (float)((unit() * 512.0 - 256.0) * s); break;
@@ -54,7 +61,7 @@ int main(int argc, char** argv) {
     if (!isfinite(v)) continue;
     ++checked;
     const float want = v / s;
-    const float got = markstein(v, s, y);
+    const float got = quotient(v, s, y, y_lo);
     if (memcmp(&want, &got, 4) == 0) continue;
     if (fabsf(v) >= 0x1p-100f) {
       if (violations < 5) printf("violation: v=%a s=%a want=%a got=%a\n", v, s, want, got);

@@ -1,7 +1,7 @@
 """Pin of the division method of the CUDA quantizer (no GPU needed).
 
-The kernels compute x / scale as Markstein's two-step FMA refinement of
-x * RN(1/scale) instead of an IEEE division. tests/division_method_check.c
+The kernels compute x / scale from a two-term reciprocal of the scale and one
+Markstein FMA correction instead of an IEEE division. tests/division_method_check.c
 checks, with the host's IEEE binary32 arithmetic, that this equals the IEEE
 quotient on the kernels' domain (scale >= 2^-40, |x| >= 2^-100), and that
 where it may not (underflowing remainders) no quantization code can change.
@@ -14,7 +14,7 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-def test_markstein_division_is_exact_on_the_kernel_domain(tmp_path):
+def test_fma_division_is_exact_on_the_kernel_domain(tmp_path):
     exe = str(tmp_path / "division_method_check")
     subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-o", exe, os.path.join(HERE, "division_method_check.c"),
                     "-lm"], check=True)

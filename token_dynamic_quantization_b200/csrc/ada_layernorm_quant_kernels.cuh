@@ -115,7 +115,11 @@ constexpr int kAdaMaxBlock = 512;
 #define DQ_ADA_MAX_REGS 128  // the row share stays in registers across four passes
 #endif
 
-template <typename InT, int VPT>
+// Warp w of a row group owns the contiguous chunk of 32 * VPT vectors starting
+// at w * 32 * VPT; lane l owns vectors chunk + l + 32 * k (k < VPT), so every
+// per-k offset is a compile-time constant. kRagged: the row is not exactly
+// G * 32 * VPT vectors, so vectors past the row end are skipped.
+template <typename InT, int VPT, bool kRagged>
 __global__ void __maxnreg__(DQ_ADA_MAX_REGS)
 ada_layernorm_quant_tma_kernel(const AdaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -130,6 +134,7 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
   const int warp_g0 = (g * tpr) >> 5;
   const int nwarps_g = tpr >> 5;
   const int lane = threadIdx.x & 31;
+  const int vbase = (lane_g >> 5) * (32 * VPT) + lane;  // this thread's vector k is vbase + 32 * k
   const uint32_t stride = a.stage_stride;
   const size_t ring_bytes = static_cast<size_t>(a.groups) * S * stride;
   uint8_t* ring = smem + static_cast<size_t>(g) * S * stride;
@@ -171,14 +176,15 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
   if (leader) {
     while (issued < n && issued < S - 1) issue_next();
   }
+  auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
 
   pdl_wait_primary();  // the affine table is complete and visible from here on
 
   // batch of the current row, tracked without division
   int64_t b = r_begin / a.seq;
   int64_t b_end = (b + 1) * a.seq;
-  const float4* A4 = reinterpret_cast<const float4*>(a.table + b * H);
-  const float4* B4 = reinterpret_cast<const float4*>(a.table + a.batch * H + b * H);
+  const float4* A4 = reinterpret_cast<const float4*>(a.table + b * H) + 2 * vbase;
+  const float4* B4 = reinterpret_cast<const float4*>(a.table + a.batch * H + b * H) + 2 * vbase;
   const int64_t table_b_stride4 = H / 4;
   int8_t* orow = a.out + r_begin * H;
 
@@ -203,8 +209,7 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      const int vi = lane_g + k * tpr;
-      InTraits<InT>::widen8(vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0), v[k]);  // zero when inactive
+      InTraits<InT>::widen8(in_row(k) ? srow[vbase + 32 * k] : make_uint4(0, 0, 0, 0), v[k]);  // zero when inactive
       const float2 s01 = __fadd2_rn(make_float2(v[k][0], v[k][1]), make_float2(v[k][2], v[k][3]));
       const float2 s23 = __fadd2_rn(make_float2(v[k][4], v[k][5]), make_float2(v[k][6], v[k][7]));
       acc[k % NACC] = __fadd2_rn(acc[k % NACC], __fadd2_rn(s01, s23));
@@ -236,6 +241,8 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
       }
       return;
     }
+    // refill the stage of the previous row (S - 1 copies stay in flight; the
+    // current row's stage is kept for the out-of-line exact path)
     if (leader && issued < n) {
       fence_proxy_async_smem();
       issue_next();
@@ -250,11 +257,11 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      const bool active = lane_g + k * tpr < nvec;
+      const bool active = in_row(k);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         float2 d = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-mean_f));
-        if (!active) d = make_float2(0.0f, 0.0f);
+        if (kRagged && !active) d = make_float2(0.0f, 0.0f);
         v[k][2 * p] = d.x;
         v[k][2 * p + 1] = d.y;
         acc[(k + p) % NACC] = __ffma2_rn(d, d, acc[(k + p) % NACC]);
@@ -282,10 +289,9 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     for (int j = 0; j < NACC; ++j) amx[j] = 0.0f;
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      const int vi = lane_g + k * tpr;
-      if (vi < nvec) {
-        const float4 a0 = __ldg(A4 + 2 * vi), a1 = __ldg(A4 + 2 * vi + 1);
-        const float4 b0 = __ldg(B4 + 2 * vi), b1 = __ldg(B4 + 2 * vi + 1);
+      if (in_row(k)) {
+        const float4 a0 = __ldg(A4 + 64 * k), a1 = __ldg(A4 + 64 * k + 1);
+        const float4 b0 = __ldg(B4 + 64 * k), b1 = __ldg(B4 + 64 * k + 1);
         const float Av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
         const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -299,13 +305,12 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
         amx[k % NACC] = fmaxf(amx[k % NACC], absmax8(v[k]));
       }
     }
-    float amax = tree<NACC, true>(amx);
-    amax = warp_max(amax);
+    float amax = warp_max(tree<NACC, true>(amx));
     if (nwarps_g > 1) {
       if (lane == 0) red_f[parity][warp] = amax;
       group_barrier(1 + g, tpr);
-      amax = red_f[parity][warp_g0];
-      for (int w = 1; w < nwarps_g; ++w) amax = fmaxf(amax, red_f[parity][warp_g0 + w]);
+      // lane j takes warp j's partial; one more warp reduction combines them
+      amax = warp_max(lane < nwarps_g ? red_f[parity][warp_g0 + lane] : 0.0f);
       parity ^= 1;
     }
 
@@ -313,21 +318,24 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const RowQuant q = make_sym(amax, 127.0f);
     if (lane_g == 0) __stcs(a.quant_scale + r, q.scale);
     if (q.exact_row) {
-      ada_quantize_row_exact<InT>(srow, A4, B4, mean_f, rstd, q, lane_g, tpr, nvec, orow);
+      ada_quantize_row_exact<InT>(srow, A4 - 2 * vbase, B4 - 2 * vbase, mean_f, rstd, q, lane_g, tpr, nvec, orow);
+      continue;
+    }
+    uint2* ov = reinterpret_cast<uint2*>(orow) + vbase;
+    if (q.zero_scale) {
+      const uint2 zeros = make_uint2(0u, 0u);
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        if (in_row(k)) __stcs(ov + 32 * k, zeros);
+      }
       continue;
     }
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
-      const int vi = lane_g + k * tpr;
-      if (vi >= nvec) continue;
+      if (!in_row(k)) continue;
       uint32_t bits[8];
-      if (q.zero_scale) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) bits[j] = __float_as_uint(kRoundMagic);
-      } else {
-        quant8<false, false>(v[k], q, -127.0f, 127.0f, bits);
-      }
-      __stcs(reinterpret_cast<uint2*>(orow) + vi, pack8_int8(bits));
+      quant8<false, false>(v[k], q, -127.0f, 127.0f, bits);
+      __stcs(ov + 32 * k, pack8_int8(bits));
     }
   }
 }

@@ -87,66 +87,11 @@ dq_status launch_status() {
 
 // ---------------------------------------------------------------- launch shapes
 
-// Launch-shape targets (compile-time, so a build can be tuned without any
-// runtime switch).
-#ifndef DQ_TARGET_TPR
-#define DQ_TARGET_TPR 128  // preferred threads per row group
-#endif
-#ifndef DQ_CTA_THREADS
-#define DQ_CTA_THREADS 256  // row groups per CTA = DQ_CTA_THREADS / tpr
-#endif
-#ifndef DQ_RING_BYTES
-#define DQ_RING_BYTES 65536  // shared-memory row ring per CTA
-#endif
-
-// Row-group shape: VPT 16-byte vectors per thread, tpr threads per row. Picks
-// the VPT in {1, 2, 3, 4, 6, 8} (up to max_vpt) that wastes the fewest lanes, then the tpr closest to the
-// target (at most max_tpr).
+// Row-group shape: VPT 16-byte vectors per thread, tpr = 32 * G threads per row.
 struct GroupShape {
   int vpt;
   int tpr;
 };
-
-GroupShape pick_shape(int64_t nvec, int max_tpr, int max_vpt) {
-  GroupShape best{0, 0};
-  double best_eff = -1.0;
-  static const int kVpts[6] = {1, 2, 3, 4, 6, 8};
-  for (int vpt : kVpts) {
-    if (vpt > max_vpt) continue;
-    const int64_t tpr = ((nvec + vpt - 1) / vpt + 31) / 32 * 32;
-    if (tpr > max_tpr) continue;
-    const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
-    const bool better = eff > best_eff + 1e-9 ||
-                        (eff > best_eff - 1e-9 &&
-                         std::llabs(tpr - DQ_TARGET_TPR) < std::llabs(best.tpr - DQ_TARGET_TPR));
-    if (better) {
-      best_eff = eff;
-      best = GroupShape{vpt, static_cast<int>(tpr)};
-    }
-  }
-  return best;
-}
-
-// Ring geometry: `groups` row groups per CTA, `stages` row buffers per group,
-// about DQ_RING_BYTES of rows per CTA (so several CTAs fit on an SM and each
-// keeps rows in flight while it computes).
-struct RingShape {
-  int groups;
-  int stages;
-  uint32_t stride;
-};
-
-RingShape pick_ring(int tpr, int64_t row_bytes, int max_block) {
-  RingShape r;
-  const int cta = DQ_CTA_THREADS < max_block ? DQ_CTA_THREADS : max_block;
-  r.groups = tpr >= cta ? 1 : cta / tpr;
-  if (r.groups > 15) r.groups = 15;  // named barriers 1..15
-  r.stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
-  int64_t s = DQ_RING_BYTES / (static_cast<int64_t>(r.groups) * r.stride);
-  s = s < 2 ? 2 : (s > 8 ? 8 : s);
-  r.stages = static_cast<int>(s);
-  return r;
-}
 
 constexpr size_t kMaxDynamicSmem = 200 * 1024;
 
@@ -179,10 +124,15 @@ bool allow_smem(const void* kernel, int device) {
 // Row-group geometry of the bulk-copy DynamicQuant kernel: a group of
 // tpr = 32 * G threads owns a row, VPT in {2, 4, 8} vectors per thread; the
 // shape wasting the fewest lanes wins, then the one whose VPT is closest to
-// DQ_TARGET_VPT. DQ_WARP_STAGES row buffers per group; groups per CTA so that
+// the target: 4 with smooth scales (the fp32 products of pass 1 then stay in
+// registers for pass 2), 8 without (more elements per thread amortize the
+// per-row work). DQ_WARP_STAGES row buffers per group; groups per CTA so that
 // a CTA holds about DQ_WARP_CTA_BYTES of rows.
-#ifndef DQ_TARGET_VPT
-#define DQ_TARGET_VPT 8
+#ifndef DQ_TARGET_VPT_SMOOTH
+#define DQ_TARGET_VPT_SMOOTH 4
+#endif
+#ifndef DQ_TARGET_VPT_PLAIN
+#define DQ_TARGET_VPT_PLAIN 8
 #endif
 #ifndef DQ_WARP_STAGES
 #define DQ_WARP_STAGES 2
@@ -191,7 +141,7 @@ bool allow_smem(const void* kernel, int device) {
 #define DQ_WARP_CTA_BYTES 65536
 #endif
 
-GroupShape pick_dq_shape(int64_t nvec) {
+GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
   GroupShape best{0, 0};
   double best_eff = -1.0;
   static const int kVpts[3] = {2, 4, 8};
@@ -201,7 +151,7 @@ GroupShape pick_dq_shape(int64_t nvec) {
     const int64_t tpr = warps * 32;
     const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
     const bool better = eff > best_eff + 1e-9 ||
-                        (eff > best_eff - 1e-9 && std::abs(vpt - DQ_TARGET_VPT) < std::abs(best.vpt - DQ_TARGET_VPT));
+                        (eff > best_eff - 1e-9 && std::abs(vpt - target_vpt) < std::abs(best.vpt - target_vpt));
     if (better) {
       best_eff = eff;
       best = GroupShape{vpt, static_cast<int>(tpr)};
@@ -210,25 +160,33 @@ GroupShape pick_dq_shape(int64_t nvec) {
   return best;
 }
 
-template <typename InT, int MODE, int OUT, int SMK, int VPT>
+template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged>
 dq_status launch_dq_tma(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
-  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT>);
+  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>);
   const size_t smem = dq::dq_smem_bytes(a.groups, a.stages, a.stage_stride, a.group_index ? a.num_groups : 0);
   if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
   const int block = a.tpr * a.groups;
   const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
   const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT><<<grid, block, smem, stream>>>(a);
+  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged><<<grid, block, smem, stream>>>(a);
   return launch_status();
+}
+
+template <typename InT, int MODE, int OUT, int SMK, int VPT>
+dq_status launch_dq_ragged(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
+  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds checks
+  if ((a.cols >> 3) == static_cast<int64_t>(a.tpr) * VPT)
+    return launch_dq_tma<InT, MODE, OUT, SMK, VPT, false>(a, device, sms, stream);
+  return launch_dq_tma<InT, MODE, OUT, SMK, VPT, true>(a, device, sms, stream);
 }
 
 template <typename InT, int MODE, int OUT, int SMK>
 dq_status launch_dq_vpt(dq::RowQuantArgs a, int vpt, int device, int sms, cudaStream_t stream) {
   switch (vpt) {
-    case 2: return launch_dq_tma<InT, MODE, OUT, SMK, 2>(a, device, sms, stream);
-    case 4: return launch_dq_tma<InT, MODE, OUT, SMK, 4>(a, device, sms, stream);
-    default: return launch_dq_tma<InT, MODE, OUT, SMK, 8>(a, device, sms, stream);
+    case 2: return launch_dq_ragged<InT, MODE, OUT, SMK, 2>(a, device, sms, stream);
+    case 4: return launch_dq_ragged<InT, MODE, OUT, SMK, 4>(a, device, sms, stream);
+    default: return launch_dq_ragged<InT, MODE, OUT, SMK, 8>(a, device, sms, stream);
   }
 }
 
@@ -237,7 +195,8 @@ dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t 
   const int device = current_device();
   const int sms = sm_count(device);
   if (vector_ok) {
-    const GroupShape gs = pick_dq_shape(a.cols >> 3);
+    const GroupShape gs =
+        pick_dq_shape(a.cols >> 3, a.smooth != nullptr ? DQ_TARGET_VPT_SMOOTH : DQ_TARGET_VPT_PLAIN);
     if (gs.vpt > 0) {
       const int64_t row_bytes = a.cols * 2;
       const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
@@ -294,9 +253,9 @@ dq_status launch_ada_table(const dq::AdaArgs& a, int sms, cudaStream_t stream) {
   return launch_status();
 }
 
-template <typename InT, int VPT>
+template <typename InT, int VPT, bool kRagged>
 dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream) {
-  void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_tma_kernel<InT, VPT>;
+  void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_tma_kernel<InT, VPT, kRagged>;
   const void* k = reinterpret_cast<const void*>(kfn);
   const size_t smem = dq::ada_smem_bytes(a.groups, a.stages, a.stage_stride);
   if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
@@ -324,14 +283,25 @@ dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream
   return launch_status();
 }
 
+template <typename InT, int VPT>
+dq_status launch_ada_ragged(dq::AdaArgs a, int device, int sms, cudaStream_t stream) {
+  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds checks
+  if ((a.hidden >> 3) == static_cast<int64_t>(a.tpr) * VPT) return launch_ada_tma<InT, VPT, false>(a, device, sms, stream);
+  return launch_ada_tma<InT, VPT, true>(a, device, sms, stream);
+}
+
 // AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8}, fewest wasted lanes,
 // then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
-// three row reductions; the row share stays in registers).
+// three row reductions; the row share stays in registers). DQ_ADA_STAGES row
+// buffers per group, one of them holding the row being processed.
 #ifndef DQ_ADA_TARGET_VPT
 #define DQ_ADA_TARGET_VPT 4
 #endif
 #ifndef DQ_ADA_CTA_BYTES
-#define DQ_ADA_CTA_BYTES 65536
+#define DQ_ADA_CTA_BYTES 98304
+#endif
+#ifndef DQ_ADA_STAGES
+#define DQ_ADA_STAGES 3
 #endif
 
 GroupShape pick_ada_shape(int64_t nvec) {
@@ -361,7 +331,7 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
     const GroupShape gs = pick_ada_shape(a.hidden >> 3);
     if (gs.vpt > 0) {
       const uint32_t stride = static_cast<uint32_t>((a.hidden * 2 + 127) / 128 * 128);
-      const int stages = 2;
+      const int stages = DQ_ADA_STAGES;
       int64_t groups = DQ_ADA_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
       const int64_t max_groups = dq::kAdaMaxBlock / gs.tpr;
       groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
@@ -372,11 +342,11 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
       a.stage_stride = stride;
       if (dq::ada_smem_bytes(a.groups, stages, stride) <= kMaxDynamicSmem) {
         switch (gs.vpt) {
-          case 2: return launch_ada_tma<InT, 2>(a, device, sms, stream);
-          case 3: return launch_ada_tma<InT, 3>(a, device, sms, stream);
-          case 4: return launch_ada_tma<InT, 4>(a, device, sms, stream);
-          case 6: return launch_ada_tma<InT, 6>(a, device, sms, stream);
-          default: return launch_ada_tma<InT, 8>(a, device, sms, stream);
+          case 2: return launch_ada_ragged<InT, 2>(a, device, sms, stream);
+          case 3: return launch_ada_ragged<InT, 3>(a, device, sms, stream);
+          case 4: return launch_ada_ragged<InT, 4>(a, device, sms, stream);
+          case 6: return launch_ada_ragged<InT, 6>(a, device, sms, stream);
+          default: return launch_ada_ragged<InT, 8>(a, device, sms, stream);
         }
       }
     }

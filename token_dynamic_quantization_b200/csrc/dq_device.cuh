@@ -2,13 +2,17 @@
 //
 // The quantization arithmetic follows the formulas of aclnnDynamicQuantV2
 // ("Formula") bit for bit: IEEE binary32, one rounding per operation,
-// round-half-to-even. The division by the row scale is evaluated with
-// Markstein's method (P. Markstein, "Computation of elementary functions on
-// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with
-// y = RN(1/s), q0 = RN(v*y) and two FMA corrections q <- RN(q + RN(v - s*q)*y)
-// the result is the correctly rounded RN(v/s) whenever the remainder v - s*q
-// does not underflow. The rows that could break that precondition in a way
-// that matters are sent to the IEEE division instead (see RowQuant).
+// round-half-to-even. The division by the row scale uses a two-term
+// reciprocal y + y_lo of s (y = RN(1/s); the residual 1 - s*y is exact, and
+// y_lo = RN((1 - s*y) * y), as in multiplication by a constant written as a
+// sum of two floats: N. Brisebarre, J.-M. Muller, S. K. Raina, IEEE Trans.
+// Computers 53(8), 2004). q0 = RN(v*y + RN(v*y_lo)) is then within one ulp of
+// v/s, and one correction step of Markstein's method (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990), q = RN(q0 + RN(v - s*q0)*y),
+// gives the correctly rounded RN(v/s) whenever nothing underflows. The rows
+// that could break that precondition in a way that matters are sent to the
+// IEEE division instead (see RowQuant).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -74,15 +78,19 @@ __device__ __forceinline__ float load_param(const void* p, int dtype, int64_t i)
 
 // ---------------------------------------------------------------- reductions
 
+// Warp-wide max / min of a float in one instruction (sm_100a redux.sync on
+// f32). Max and min are exact, so the result does not depend on the order;
+// NaN lanes are ignored like fmaxf/fminf do (NaN inputs are outside the
+// contract anyway).
 __device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 __device__ __forceinline__ float warp_min(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+  float r;
+  asm volatile("redux.sync.min.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -172,12 +180,12 @@ struct Packed<__nv_bfloat16> {
 // Per-row quantization constants.
 //   exact_row: use the IEEE division for every element of the row. Set when
 //     scale < 2^-40 or the offset is not finite. Otherwise (scale >= 2^-40) an
-//     element whose remainder can underflow has |v| < 2^-100, hence a quotient
-//     below 2^-60 in magnitude: it rounds to code 0 (symmetric), or it cannot
-//     move fl(q + offset) across a rounding midpoint that decides a code
-//     (asymmetric: a decisive z needs |offset| > 1/4, whose neighbouring
-//     midpoints are at least 2^-27 away), so Markstein's result is exact
-//     wherever it is used.
+//     element whose remainder or v*y_lo can underflow has |v| < 2^-100 or a
+//     quotient below 2^-100, hence a quotient below 2^-60 in magnitude: it
+//     rounds to code 0 (symmetric), or it cannot move fl(q + offset) across a
+//     rounding midpoint that decides a code (asymmetric: a decisive z needs
+//     |offset| > 1/4, whose neighbouring midpoints are at least 2^-27 away),
+//     so the computed quotient is exact wherever it is used.
 //   clamp: saturate before rounding (asymmetric rows with |offset| >= 2^20,
 //     where rounding noise of the offset can push the row's extremes past the
 //     code range; below 2^20 every code provably lies in range).
@@ -185,12 +193,21 @@ struct RowQuant {
   float scale;   // written to scale[r]
   float offset;  // asymmetric only
   float rcp;     // RN(1 / scale) (IEEE reciprocal)
+  float rcp_lo;  // RN((1 - scale * rcp) * rcp): 1 / scale ~ rcp + rcp_lo
   bool zero_scale;
   bool exact_row;
   bool clamp;
 };
 
 constexpr float kMarksteinMinScale = 9.094947017729282e-13f;  // 2^-40
+
+// The two-term reciprocal of `scale` used by quant8. The residual
+// 1 - scale * rcp of a correctly rounded reciprocal is exact in binary32, so
+// rcp + rcp_lo carries 1 / scale to about 2^-47 relative.
+__device__ __forceinline__ void set_reciprocal(RowQuant& q) {
+  q.rcp = __frcp_rn(q.scale);
+  q.rcp_lo = __fmul_rn(__fmaf_rn(-q.scale, q.rcp, 1.0f), q.rcp);
+}
 
 // symmetric: scale = absmax / D (IEEE division)
 __device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
@@ -199,7 +216,9 @@ __device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
   q.offset = 0.0f;
   q.zero_scale = (q.scale == 0.0f);
   q.exact_row = !q.zero_scale && !(q.scale >= kMarksteinMinScale);
-  q.rcp = (q.zero_scale || q.exact_row) ? 0.0f : __frcp_rn(q.scale);
+  q.rcp = 0.0f;
+  q.rcp_lo = 0.0f;
+  if (!q.zero_scale && !q.exact_row) set_reciprocal(q);
   q.clamp = false;
   return q;
 }
@@ -213,12 +232,15 @@ __device__ __forceinline__ RowQuant make_asym(float mx, float mn, float scale_op
   if (q.zero_scale) {
     q.offset = offset_opt;
     q.rcp = 0.0f;
+    q.rcp_lo = 0.0f;
     q.exact_row = false;
     return q;
   }
   q.offset = __fsub_rn(offset_opt, __fdiv_rn(mx, q.scale));
   q.exact_row = !(q.scale >= kMarksteinMinScale) || !isfinite(q.offset);
-  q.rcp = q.exact_row ? 0.0f : __frcp_rn(q.scale);
+  q.rcp = 0.0f;
+  q.rcp_lo = 0.0f;
+  if (!q.exact_row) set_reciprocal(q);
   q.clamp = !(fabsf(q.offset) < 1048576.0f);  // 2^20
   return q;
 }
@@ -237,7 +259,8 @@ __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
 // Codes of 8 elements (magic-sum patterns, see kRoundMagic) on a row whose
 // RowQuant has neither zero_scale nor exact_row set:
-//   q = RN(v / scale) by Markstein's method (5 FMA-pipe operations),
+//   q = RN(v / scale) from the two-term reciprocal and one Markstein
+//   correction (4 FMA-pipe operations per element pair),
 //   z = RN(q + offset) (asymmetric), optional saturation, then RNE via the
 //   magic add. Branch-free; every element gets the formulas' exact result.
 template <bool kAsym, bool kClamp>
@@ -246,11 +269,9 @@ __device__ __forceinline__ void quant8(const float (&v)[8], const RowQuant& q, f
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
     const float2 vv = make_float2(v[2 * p], v[2 * p + 1]);
-    const float2 q0 = __fmul2_rn(vv, f2(q.rcp));
-    const float2 r0 = __ffma2_rn(f2(-q.scale), q0, vv);
-    const float2 q1 = __ffma2_rn(r0, f2(q.rcp), q0);
-    const float2 r1 = __ffma2_rn(f2(-q.scale), q1, vv);
-    float2 z = __ffma2_rn(r1, f2(q.rcp), q1);  // RN(v / scale)
+    const float2 q0 = __ffma2_rn(vv, f2(q.rcp), __fmul2_rn(vv, f2(q.rcp_lo)));  // faithful v / scale
+    const float2 r0 = __ffma2_rn(f2(-q.scale), q0, vv);                         // exact remainder
+    float2 z = __ffma2_rn(r0, f2(q.rcp), q0);                                    // RN(v / scale)
     if (kAsym) z = __fadd2_rn(z, f2(q.offset));
     if (kClamp) {
       z.x = fminf(fmaxf(z.x, lo), hi);

@@ -5,11 +5,13 @@
 // bounded by HBM bandwidth if each element costs only a handful of
 // instructions. Two kernels:
 //   * bulk-copy kernel (rows whose bytes, smooth-scale rows and code rows are
-//     suitably aligned): one warp per row, persistent grid. Each warp keeps a
-//     ring of shared-memory row buffers filled with cp.async.bulk (TMA)
-//     copies of its next rows, reduces the row (warp shuffles only), derives
-//     the row constants, then quantizes the row with Markstein's division
-//     (branch-free, exact) and packs codes with byte permutes.
+//     suitably aligned): a row group of one or more warps per row, persistent
+//     grid. Each group keeps a ring of shared-memory row buffers filled with
+//     cp.async.bulk (TMA) copies of its next rows, reduces the row (one-
+//     instruction warp reductions, then a shared-memory combine across the
+//     group's warps), derives the row constants, then quantizes the row with an exact FMA division
+//     (two-term reciprocal, one Markstein correction; branch-free) and packs
+//     codes with byte permutes.
 //   * generic kernel: any cols / alignment; one CTA per row (grid-strided),
 //     two passes over the row (the second one mostly hits L2).
 #pragma once
@@ -140,31 +142,38 @@ __device__ __noinline__ void quantize_row_exact(const uint4* srow, const void* s
 
 // Row groups of tpr = 32 * G threads, `groups` row groups per CTA. Each group
 // owns a ring of `stages` shared-memory row buffers that its first lane keeps
-// filled with cp.async.bulk (TMA) copies of the group's next rows. A thread
-// owns VPT 16-byte vectors of the row (vector vi = lane_g + k * tpr):
-//   pass 1: copy them from the stage into registers (raw 16-bit values) and
-//     reduce (packed 16-bit pairs without smooth scales; fp32 products with);
+// filled with cp.async.bulk (TMA) copies of the group's next rows. Warp w of a
+// group owns the contiguous chunk of 32 * VPT 16-byte vectors starting at
+// w * 32 * VPT; lane l of it owns vectors chunk + l + 32 * k (k < VPT), so
+// consecutive lanes touch consecutive 16-byte vectors (conflict-free shared
+// loads, coalesced stores) and every per-k offset is a compile-time constant.
+// kRagged: the row is not exactly G * 32 * VPT vectors, so vectors past the
+// row end are skipped.
+//   pass 1: copy the thread's vectors from the stage into registers (raw
+//     16-bit values) and reduce (packed 16-bit pairs without smooth scales;
+//     fp32 products with them, kept in registers for pass 2 when VPT <= 4);
 //     the group reduces through warp shuffles and, for G > 1, shared memory
 //     behind its named barrier. That barrier also tells the leader that the
 //     stage has been read by every thread, so the stage is refilled right
 //     away: while a group quantizes one row, its next `stages` rows are in
 //     flight.
-//   pass 2: from registers only: widen (* smooth), Markstein division, magic
-//     rounding, byte-permute packing, one 8-byte (int8) or 4-byte (int4)
-//     store per vector.
+//   pass 2: from registers only: widen (* smooth) unless kept, exact FMA
+//     division, magic rounding, byte-permute packing, one 8-byte (int8) or
+//     4-byte (int4) store per vector.
 constexpr int kWarpKernelMaxThreads = 512;
 #ifndef DQ_MAX_REGS
-#define DQ_MAX_REGS 96  // registers per thread: leaves room for enough resident warps
+#define DQ_MAX_REGS 128  // registers per thread: 2 CTAs of 256 threads per SM
 #endif
 
-template <typename InT, int MODE, int OUT, int SMK, int VPT>
+template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged>
 __global__ void __maxnreg__(DQ_MAX_REGS)
 dynamic_quant_tma_kernel(const RowQuantArgs a) {
   using C = QuantConsts<MODE, OUT>;
   using P = Packed<InT>;
   constexpr bool kA = MODE == kAsym;
+  constexpr bool kKeep = SMK != kSmNone && VPT <= 4;  // fp32 products stay in registers
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float red[2][kWarpKernelMaxThreads / 32][2];
+  __shared__ float red[2][2][kWarpKernelMaxThreads / 32];  // [parity][max, min][warp]
 
   const int tpr = a.tpr;
   const int g = threadIdx.x / tpr;
@@ -173,6 +182,7 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
   const int warp_g0 = (g * tpr) >> 5;
   const int nwarps_g = tpr >> 5;
   const int lane = threadIdx.x & 31;
+  const int vbase = (lane_g >> 5) * (32 * VPT) + lane;  // this thread's vector k is vbase + 32 * k
   const int S = a.stages;
   const int NG = a.groups;
   const uint32_t stride = a.stage_stride;
@@ -222,6 +232,7 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
   int64_t expert_end = moe ? -1 : INT64_MAX;
   const int64_t y_row_bytes = OUT == kOutInt8 ? a.cols : (a.cols >> 1);
   uint8_t* yrow = static_cast<uint8_t*>(a.y) + r_begin * y_row_bytes;
+  auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
 
   int st = 0;
   uint32_t phase = 0;
@@ -246,12 +257,10 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
     // ---- pass 1: this thread's vectors into registers, reduce
     uint4 raw[VPT];
 #pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const int vi = lane_g + k * tpr;
-      raw[k] = vi < nvec ? srow[vi] : make_uint4(0, 0, 0, 0);
-    }
+    for (int k = 0; k < VPT; ++k) raw[k] = in_row(k) ? srow[vbase + 32 * k] : make_uint4(0, 0, 0, 0);
     float m0, m1;
     constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
+    float prod[kKeep ? VPT : 1][8];
     if (SMK != kSmNone) {
       float amx[NACC], amn[NACC];
 #pragma unroll
@@ -261,10 +270,13 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       }
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
-        const int vi = lane_g + k * tpr;
-        if (vi < nvec) {
+        if (in_row(k)) {
           float v[8];
-          input8<InT, SMK>(raw[k], smooth_row, vi, v);
+          input8<InT, SMK>(raw[k], smooth_row, vbase + 32 * k, v);
+          if (kKeep) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) prod[kKeep ? k : 0][j] = v[j];
+          }
           if (kA) {
             amx[k % NACC] = fmaxf(amx[k % NACC], max8(v));
             amn[k % NACC] = fminf(amn[k % NACC], min8(v));
@@ -284,7 +296,7 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       }
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
-        if (lane_g + k * tpr < nvec) {
+        if (in_row(k)) {
           const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
           if (kA) {
             hmax[k % NACC] = P::vmax(hmax[k % NACC], P::vmax(P::vmax(P::from_bits(w[0]), P::from_bits(w[1])),
@@ -314,16 +326,14 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
     bool failed;
     if (nwarps_g > 1) {
       if (lane == 0) {
-        red[parity][warp][0] = m0;
-        red[parity][warp][1] = m1;
+        red[parity][0][warp] = m0;
+        if (kA) red[parity][1][warp] = m1;
       }
       failed = group_barrier_or(1 + g, tpr, !arrived);
-      m0 = red[parity][warp_g0][0];
-      m1 = red[parity][warp_g0][1];
-      for (int w = 1; w < nwarps_g; ++w) {
-        m0 = fmaxf(m0, red[parity][warp_g0 + w][0]);
-        if (kA) m1 = fminf(m1, red[parity][warp_g0 + w][1]);
-      }
+      // lane j takes warp j's partial; one more warp reduction combines them
+      const bool has = lane < nwarps_g;
+      m0 = warp_max(has ? red[parity][0][warp_g0 + lane] : (kA ? -INFINITY : 0.0f));
+      if (kA) m1 = warp_min(has ? red[parity][1][warp_g0 + lane] : INFINITY);
       parity ^= 1;
     } else {
       failed = __any_sync(0xffffffffu, !arrived);
@@ -345,7 +355,8 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
     }
 
     RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
-    if (q.exact_row && row_valid && !q.zero_scale) {
+    const bool exact = q.exact_row && row_valid && !q.zero_scale;
+    if (exact) {
       // rare: the stage is still needed by the out-of-line exact path
       quantize_row_exact<InT, MODE, OUT, SMK>(srow, smooth_row, q, lane_g, tpr, nvec, yrow);
       if (nwarps_g > 1) group_barrier(1 + g, tpr); else __syncwarp();
@@ -366,31 +377,45 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       __stcs(a.scale + r, q.scale);
       if (kA) __stcs(a.offset + r, q.offset);
     }
-    if (q.exact_row && row_valid && !q.zero_scale) continue;
+    if (exact) continue;
 
     // ---- pass 2: quantize from registers and store
-    const bool constant = !row_valid || q.zero_scale;
-    const uint32_t cb = __float_as_uint(__fadd_rn(row_valid ? C::kOffsetOpt : 0.0f, kRoundMagic));
+    auto store8 = [&](int k, const uint32_t (&bits)[8]) {
+      const int vi = vbase + 32 * k;
+      if (OUT == kOutInt8) {
+        __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
+      } else {
+        __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
+      }
+    };
+    if (!row_valid || q.zero_scale) {
+      // every code of the row is the same: 0, or offset_opt for a constant
+      // asymmetric row (rows past the last group get 0)
+      const uint32_t cb = __float_as_uint(__fadd_rn(row_valid ? C::kOffsetOpt : 0.0f, kRoundMagic));
+      uint32_t bits[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) bits[j] = cb;
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        if (in_row(k)) store8(k, bits);
+      }
+      continue;
+    }
     auto pass2 = [&](auto clamp_tag) {
       constexpr bool kClamp = decltype(clamp_tag)::value;
 #pragma unroll
       for (int k = 0; k < VPT; ++k) {
-        const int vi = lane_g + k * tpr;
-        if (vi >= nvec) continue;
-        uint32_t bits[8];
-        if (constant) {
+        if (!in_row(k)) continue;
+        float v[8];
+        if (kKeep) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) bits[j] = cb;
+          for (int j = 0; j < 8; ++j) v[j] = prod[kKeep ? k : 0][j];
         } else {
-          float v[8];
-          input8<InT, SMK>(raw[k], smooth_row, vi, v);
-          quant8<kA, kClamp>(v, q, C::kLo, C::kHi, bits);
+          input8<InT, SMK>(raw[k], smooth_row, vbase + 32 * k, v);
         }
-        if (OUT == kOutInt8) {
-          __stcs(reinterpret_cast<uint2*>(yrow) + vi, pack8_int8(bits));
-        } else {
-          __stcs(reinterpret_cast<unsigned int*>(yrow) + vi, pack8_int4(bits));
-        }
+        uint32_t bits[8];
+        quant8<kA, kClamp>(v, q, C::kLo, C::kHi, bits);
+        store8(k, bits);
       }
     };
     if (kA && q.clamp) {
