@@ -14,7 +14,9 @@
 //      registers between its passes. It is launched as a programmatic
 //      dependent of the table kernel: it sets up its ring and starts copying
 //      rows while the table is still being written, and waits for the table
-//      (griddepcontrol.wait) just before first reading it.
+//      (griddepcontrol.wait) just before first reading it. The table kernel
+//      is itself a programmatic dependent of the work before it and releases
+//      the row kernel only after that work has completed.
 //
 // Arithmetic:
 //   * E(x), Var(x): the row is resident, so a two-pass mean / centred
@@ -60,15 +62,17 @@ __host__ __device__ inline size_t ada_smem_bytes(int groups, int stages, uint32_
   return static_cast<size_t>(groups) * stages * stride + static_cast<size_t>(groups) * stages * 8;
 }
 
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ============================================================ affine table
 
 constexpr int kTableBlock = 256;
 
 __global__ void __launch_bounds__(kTableBlock) ada_affine_table_kernel(const AdaArgs a) {
-  pdl_launch_dependents();  // the main kernel may start its row copies now
+  // launched as a programmatic dependent of the previous work in the stream:
+  // wait for it, then let the row kernel start (it copies rows of x before
+  // its own wait, which is safe once the work before this kernel is done)
+  pdl_wait_primary();
+  pdl_launch_dependents();
   const int64_t H = a.hidden;
   const int64_t total = a.batch * H;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;

@@ -119,6 +119,29 @@ bool allow_smem(const void* kernel, int device) {
   return true;
 }
 
+// Launch `kernel` as a programmatic dependent of the previous work in
+// `stream`: it may start before that work finishes and waits for it
+// (griddepcontrol.wait) before touching global memory.
+template <typename Args>
+dq_status launch_programmatic(void (*kernel)(const Args), const Args& a, int grid, int block, size_t smem,
+                              cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, a) != cudaSuccess) {
+    cudaGetLastError();
+    return DQ_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // ---------------------------------------------------------------- dynamic quant dispatch
 
 // Row-group geometry of the bulk-copy DynamicQuant kernel: a group of
@@ -127,7 +150,9 @@ bool allow_smem(const void* kernel, int device) {
 // the target: 4 with smooth scales (the fp32 products of pass 1 then stay in
 // registers for pass 2), 8 without (more elements per thread amortize the
 // per-row work). DQ_WARP_STAGES row buffers per group; groups per CTA so that
-// a CTA holds about DQ_WARP_CTA_BYTES of rows.
+// a CTA holds about DQ_WARP_CTA_BYTES_SMOOTH / _PLAIN of rows (measured: the
+// smooth-scale path prefers several groups sharing a CTA, the plain path
+// smaller CTAs).
 #ifndef DQ_TARGET_VPT_SMOOTH
 #define DQ_TARGET_VPT_SMOOTH 4
 #endif
@@ -137,8 +162,11 @@ bool allow_smem(const void* kernel, int device) {
 #ifndef DQ_WARP_STAGES
 #define DQ_WARP_STAGES 2
 #endif
-#ifndef DQ_WARP_CTA_BYTES
-#define DQ_WARP_CTA_BYTES 65536
+#ifndef DQ_WARP_CTA_BYTES_SMOOTH
+#define DQ_WARP_CTA_BYTES_SMOOTH 65536
+#endif
+#ifndef DQ_WARP_CTA_BYTES_PLAIN
+#define DQ_WARP_CTA_BYTES_PLAIN 32768
 #endif
 
 GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
@@ -169,8 +197,8 @@ dq_status launch_dq_tma(dq::RowQuantArgs a, int device, int sms, cudaStream_t st
   const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
   const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-  dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged><<<grid, block, smem, stream>>>(a);
-  return launch_status();
+  return launch_programmatic(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>, a, grid, block, smem,
+                             stream);
 }
 
 template <typename InT, int MODE, int OUT, int SMK, int VPT>
@@ -201,7 +229,8 @@ dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t 
       const int64_t row_bytes = a.cols * 2;
       const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
       const int stages = DQ_WARP_STAGES;
-      int64_t groups = DQ_WARP_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
+      const int64_t cta_bytes = a.smooth != nullptr ? DQ_WARP_CTA_BYTES_SMOOTH : DQ_WARP_CTA_BYTES_PLAIN;
+      int64_t groups = cta_bytes / (static_cast<int64_t>(stages) * stride);
       const int64_t max_groups = dq::kWarpKernelMaxThreads / gs.tpr;
       groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
       groups = groups > 15 ? 15 : groups;  // named barriers 1..15
@@ -249,8 +278,7 @@ dq_status launch_ada_table(const dq::AdaArgs& a, int sms, cudaStream_t stream) {
   const int64_t total = a.batch * a.hidden;
   int64_t grid = (total + dq::kTableBlock - 1) / dq::kTableBlock;
   if (grid > 2 * sms) grid = 2 * sms;
-  dq::ada_affine_table_kernel<<<static_cast<int>(grid), dq::kTableBlock, 0, stream>>>(a);
-  return launch_status();
+  return launch_programmatic(dq::ada_affine_table_kernel, a, static_cast<int>(grid), dq::kTableBlock, 0, stream);
 }
 
 template <typename InT, int VPT, bool kRagged>
@@ -266,21 +294,7 @@ dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
   dq_status st = launch_ada_table(a, sms, stream);
   if (st != DQ_OK) return st;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kfn, a) != cudaSuccess) {
-    cudaGetLastError();
-    return DQ_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_programmatic(kfn, a, grid, block, smem, stream);
 }
 
 template <typename InT, int VPT>

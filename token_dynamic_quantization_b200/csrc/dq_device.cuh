@@ -30,6 +30,17 @@ struct BoolTag {
   static constexpr bool value = B;
 };
 
+// ---------------------------------------------------------------- launch overlap
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still
+// running. launch_dependents lets the next such kernel start early;
+// wait_primary blocks until the previous kernel has completed and its memory
+// is visible (a no-op for an ordinary launch), so no global memory may be
+// touched before it.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- widening
 
 template <typename T>

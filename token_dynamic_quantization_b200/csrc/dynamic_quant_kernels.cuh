@@ -171,7 +171,10 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
   using C = QuantConsts<MODE, OUT>;
   using P = Packed<InT>;
   constexpr bool kA = MODE == kAsym;
-  constexpr bool kKeep = SMK != kSmNone && VPT <= 4;  // fp32 products stay in registers
+#ifndef DQ_KEEP_MAX_VPT
+#define DQ_KEEP_MAX_VPT 8
+#endif
+  constexpr bool kKeep = SMK != kSmNone && VPT <= DQ_KEEP_MAX_VPT;  // fp32 products stay in registers
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[2][2][kWarpKernelMaxThreads / 32];  // [parity][max, min][warp]
 
@@ -197,6 +200,10 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
     for (int i = 0; i < NG * S; ++i) mbar_init(all + i, 1);
     fence_mbarrier_init();
   }
+  // launched as a programmatic dependent: the set-up above overlaps the tail
+  // of the previous kernel; every global memory access comes after the wait
+  pdl_launch_dependents();
+  pdl_wait_primary();
   if (moe) {
     for (int i = threadIdx.x; i < a.num_groups; i += blockDim.x) gi_s[i] = a.group_index[i];
   }
