@@ -114,7 +114,10 @@ __device__ __noinline__ void ada_quantize_row_exact(const uint4* srow, const flo
 
 // ============================================================ bulk-copy kernel
 
-constexpr int kAdaMaxBlock = 512;
+#ifndef DQ_ADA_MAX_BLOCK
+#define DQ_ADA_MAX_BLOCK 512
+#endif
+constexpr int kAdaMaxBlock = DQ_ADA_MAX_BLOCK;
 #ifndef DQ_ADA_MAX_REGS
 #define DQ_ADA_MAX_REGS 128  // the row share stays in registers across four passes
 #endif
@@ -319,7 +322,7 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     }
 
     // ---- steps 4-5
-    const RowQuant q = make_sym(amax, 127.0f);
+    const RowQuant q = make_sym<127>(amax);
     if (lane_g == 0) __stcs(a.quant_scale + r, q.scale);
     if (q.exact_row) {
       ada_quantize_row_exact<InT>(srow, A4 - 2 * vbase, B4 - 2 * vbase, mean_f, rstd, q, lane_g, tpr, nvec, orow);
@@ -398,7 +401,7 @@ ada_layernorm_quant_generic_kernel(const AdaArgs a) {
     amax = red_f[0];
     for (int i = 1; i < kWarps; ++i) amax = fmaxf(amax, red_f[i]);
     __syncthreads();
-    const RowQuant q = make_sym(amax, 127.0f);
+    const RowQuant q = make_sym<127>(amax);
     if (threadIdx.x == 0) a.quant_scale[r] = q.scale;
     for (int64_t c = threadIdx.x; c < H; c += kAdaGenericBlock) {
       a.out[base + c] = static_cast<int8_t>(q.zero_scale ? 0 : code_exact<false>(value(c), q, -127.0f, 127.0f));

@@ -188,14 +188,19 @@ GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
   return best;
 }
 
+// Internal status of the bulk-copy launchers: the configuration cannot run on
+// this device (shared memory or occupancy); the caller uses the generic kernel.
+constexpr dq_status kNotLaunchable = static_cast<dq_status>(-1);
+
 template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged>
 dq_status launch_dq_tma(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
   const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>);
   const size_t smem = dq::dq_smem_bytes(a.groups, a.stages, a.stage_stride, a.group_index ? a.num_groups : 0);
-  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
+  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return kNotLaunchable;
   const int block = a.tpr * a.groups;
   const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
   const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
+  if (resident < 1) return kNotLaunchable;
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
   return launch_programmatic(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>, a, grid, block, smem,
                              stream);
@@ -239,12 +244,17 @@ dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t 
       a.stage_stride = stride;
       a.tpr = gs.tpr;
       if (dq::dq_smem_bytes(a.groups, stages, stride, a.group_index ? a.num_groups : 0) <= kMaxDynamicSmem) {
-        if (a.smooth == nullptr) return launch_dq_vpt<InT, MODE, OUT, dq::kSmNone>(a, gs.vpt, device, sms, stream);
-        switch (a.smooth_dtype) {
-          case dq::kF32: return launch_dq_vpt<InT, MODE, OUT, dq::kSmF32>(a, gs.vpt, device, sms, stream);
-          case dq::kF16: return launch_dq_vpt<InT, MODE, OUT, dq::kSmF16>(a, gs.vpt, device, sms, stream);
-          default: return launch_dq_vpt<InT, MODE, OUT, dq::kSmBF16>(a, gs.vpt, device, sms, stream);
+        dq_status st;
+        if (a.smooth == nullptr) {
+          st = launch_dq_vpt<InT, MODE, OUT, dq::kSmNone>(a, gs.vpt, device, sms, stream);
+        } else if (a.smooth_dtype == dq::kF32) {
+          st = launch_dq_vpt<InT, MODE, OUT, dq::kSmF32>(a, gs.vpt, device, sms, stream);
+        } else if (a.smooth_dtype == dq::kF16) {
+          st = launch_dq_vpt<InT, MODE, OUT, dq::kSmF16>(a, gs.vpt, device, sms, stream);
+        } else {
+          st = launch_dq_vpt<InT, MODE, OUT, dq::kSmBF16>(a, gs.vpt, device, sms, stream);
         }
+        if (st != kNotLaunchable) return st;
       }
     }
   }
@@ -286,11 +296,12 @@ dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream
   void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_tma_kernel<InT, VPT, kRagged>;
   const void* k = reinterpret_cast<const void*>(kfn);
   const size_t smem = dq::ada_smem_bytes(a.groups, a.stages, a.stage_stride);
-  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return DQ_ERR_UNSUPPORTED;
+  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return kNotLaunchable;
   const int block = a.tpr * a.groups;
   const int64_t rows = a.batch * a.seq;
   const int64_t wanted = (rows + a.groups - 1) / a.groups;
   const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
+  if (resident < 1) return kNotLaunchable;
   const int grid = static_cast<int>(wanted < resident ? wanted : resident);
   dq_status st = launch_ada_table(a, sms, stream);
   if (st != DQ_OK) return st;
@@ -355,13 +366,15 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
       a.stages = stages;
       a.stage_stride = stride;
       if (dq::ada_smem_bytes(a.groups, stages, stride) <= kMaxDynamicSmem) {
+        dq_status st;
         switch (gs.vpt) {
-          case 2: return launch_ada_ragged<InT, 2>(a, device, sms, stream);
-          case 3: return launch_ada_ragged<InT, 3>(a, device, sms, stream);
-          case 4: return launch_ada_ragged<InT, 4>(a, device, sms, stream);
-          case 6: return launch_ada_ragged<InT, 6>(a, device, sms, stream);
-          default: return launch_ada_ragged<InT, 8>(a, device, sms, stream);
+          case 2: st = launch_ada_ragged<InT, 2>(a, device, sms, stream); break;
+          case 3: st = launch_ada_ragged<InT, 3>(a, device, sms, stream); break;
+          case 4: st = launch_ada_ragged<InT, 4>(a, device, sms, stream); break;
+          case 6: st = launch_ada_ragged<InT, 6>(a, device, sms, stream); break;
+          default: st = launch_ada_ragged<InT, 8>(a, device, sms, stream); break;
         }
+        if (st != kNotLaunchable) return st;
       }
     }
   }

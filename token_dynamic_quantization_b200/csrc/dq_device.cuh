@@ -190,7 +190,7 @@ struct Packed<__nv_bfloat16> {
 
 // Per-row quantization constants.
 //   exact_row: use the IEEE division for every element of the row. Set when
-//     scale < 2^-40 or the offset is not finite. Otherwise (scale >= 2^-40) an
+//     scale is outside [2^-40, 2^100] or the offset is not finite. Otherwise an
 //     element whose remainder or v*y_lo can underflow has |v| < 2^-100 or a
 //     quotient below 2^-100, hence a quotient below 2^-60 in magnitude: it
 //     rounds to code 0 (symmetric), or it cannot move fl(q + offset) across a
@@ -210,7 +210,8 @@ struct RowQuant {
   bool clamp;
 };
 
-constexpr float kMarksteinMinScale = 9.094947017729282e-13f;  // 2^-40
+constexpr float kMarksteinMinScale = 0x1p-40f;  // scales outside [2^-40, 2^100] use the IEEE division
+constexpr float kMarksteinMaxScale = 0x1p100f;
 
 // The two-term reciprocal of `scale` used by quant8. The residual
 // 1 - scale * rcp of a correctly rounded reciprocal is exact in binary32, so
@@ -220,13 +221,51 @@ __device__ __forceinline__ void set_reciprocal(RowQuant& q) {
   q.rcp_lo = __fmul_rn(__fmaf_rn(-q.scale, q.rcp, 1.0f), q.rcp);
 }
 
-// symmetric: scale = absmax / D (IEEE division)
-__device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
+// RN(v / scale) from the row's two-term reciprocal and one Markstein
+// correction (the method of quant8, for one value).
+__device__ __forceinline__ float div_split(float v, const RowQuant& q) {
+  const float q0 = __fmaf_rn(v, q.rcp, __fmul_rn(v, q.rcp_lo));
+  return __fmaf_rn(__fmaf_rn(-q.scale, q0, v), q.rcp, q0);
+}
+
+// Two-term reciprocals of the quantizers' constant divisors: y = RN(1/D) and
+// lo = RN((1 - D*y) * y), as exact binary32 literals.
+template <int D>
+struct ConstRecip;
+template <>
+struct ConstRecip<7> {
+  static constexpr float y = 0x1.24924ap-3f, lo = -0x1.b6db7p-28f;
+};
+template <>
+struct ConstRecip<15> {
+  static constexpr float y = 0x1.111112p-4f, lo = -0x1.ddddep-29f;
+};
+template <>
+struct ConstRecip<127> {
+  static constexpr float y = 0x1.020408p-7f, lo = 0x1.020408p-35f;
+};
+template <>
+struct ConstRecip<255> {
+  static constexpr float y = 0x1.010102p-8f, lo = -0x1.fdfep-33f;
+};
+
+// RN(a / D) for D in {7, 15, 127, 255} with three FMA-pipe operations and no
+// branch: exact for every finite binary32 a (checked exhaustively on the host
+// against the IEEE division).
+template <int D>
+__device__ __forceinline__ float div_const(float a) {
+  const float q0 = __fmaf_rn(a, ConstRecip<D>::y, __fmul_rn(a, ConstRecip<D>::lo));
+  return __fmaf_rn(__fmaf_rn(-static_cast<float>(D), q0, a), ConstRecip<D>::y, q0);
+}
+
+// symmetric: scale = absmax / D
+template <int D>
+__device__ __forceinline__ RowQuant make_sym(float absmax) {
   RowQuant q;
-  q.scale = __fdiv_rn(absmax, divisor);
+  q.scale = div_const<D>(absmax);
   q.offset = 0.0f;
   q.zero_scale = (q.scale == 0.0f);
-  q.exact_row = !q.zero_scale && !(q.scale >= kMarksteinMinScale);
+  q.exact_row = !q.zero_scale && !(q.scale >= kMarksteinMinScale && q.scale <= kMarksteinMaxScale);
   q.rcp = 0.0f;
   q.rcp_lo = 0.0f;
   if (!q.zero_scale && !q.exact_row) set_reciprocal(q);
@@ -234,24 +273,35 @@ __device__ __forceinline__ RowQuant make_sym(float absmax, float divisor) {
   return q;
 }
 
-// asymmetric: scale = (max - min) / scale_opt; offset = offset_opt - max / scale
-__device__ __forceinline__ RowQuant make_asym(float mx, float mn, float scale_opt, float offset_opt) {
+// asymmetric: scale = (max - min) / D; offset = OFF - max / scale
+template <int D, int OFF>
+__device__ __forceinline__ RowQuant make_asym(float mx, float mn) {
   RowQuant q;
-  q.scale = __fdiv_rn(__fsub_rn(mx, mn), scale_opt);
+  q.scale = div_const<D>(__fsub_rn(mx, mn));
   q.zero_scale = (q.scale == 0.0f);
   q.clamp = false;
+  q.rcp = 0.0f;
+  q.rcp_lo = 0.0f;
   if (q.zero_scale) {
-    q.offset = offset_opt;
-    q.rcp = 0.0f;
-    q.rcp_lo = 0.0f;
+    q.offset = static_cast<float>(OFF);
     q.exact_row = false;
     return q;
   }
-  q.offset = __fsub_rn(offset_opt, __fdiv_rn(mx, q.scale));
-  q.exact_row = !(q.scale >= kMarksteinMinScale) || !isfinite(q.offset);
-  q.rcp = 0.0f;
-  q.rcp_lo = 0.0f;
-  if (!q.exact_row) set_reciprocal(q);
+  const bool in_range = q.scale >= kMarksteinMinScale && q.scale <= kMarksteinMaxScale;
+  float mq;
+  if (in_range) {
+    set_reciprocal(q);
+    // the split division is exact for |max| >= 2^-100 (and for 0)
+    mq = (fabsf(mx) >= 0x1p-100f || mx == 0.0f) ? div_split(mx, q) : __fdiv_rn(mx, q.scale);
+  } else {
+    mq = __fdiv_rn(mx, q.scale);
+  }
+  q.offset = __fsub_rn(static_cast<float>(OFF), mq);
+  q.exact_row = !in_range || !isfinite(q.offset);
+  if (q.exact_row) {
+    q.rcp = 0.0f;
+    q.rcp_lo = 0.0f;
+  }
   q.clamp = !(fabsf(q.offset) < 1048576.0f);  // 2^20
   return q;
 }

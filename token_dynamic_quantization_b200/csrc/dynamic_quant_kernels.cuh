@@ -45,8 +45,9 @@ struct RowQuantArgs {
 template <int MODE, int OUT>
 struct QuantConsts {
   static constexpr bool kFour = OUT == kOutInt4;
-  static constexpr float kDivisor = MODE == kSym ? (kFour ? 7.0f : 127.0f) : (kFour ? 15.0f : 255.0f);
-  static constexpr float kOffsetOpt = MODE == kSym ? 0.0f : (kFour ? 7.0f : 127.0f);
+  static constexpr int kDivisor = MODE == kSym ? (kFour ? 7 : 127) : (kFour ? 15 : 255);
+  static constexpr int kOffsetOptInt = MODE == kSym ? 0 : (kFour ? 7 : 127);
+  static constexpr float kOffsetOpt = static_cast<float>(kOffsetOptInt);
   static constexpr float kLo = MODE == kSym ? (kFour ? -7.0f : -127.0f) : (kFour ? -8.0f : -128.0f);
   static constexpr float kHi = kFour ? 7.0f : 127.0f;
 };
@@ -361,7 +362,7 @@ dynamic_quant_tma_kernel(const RowQuantArgs a) {
       return;
     }
 
-    RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
+    RowQuant q = kA ? make_asym<C::kDivisor, C::kOffsetOptInt>(m0, m1) : make_sym<C::kDivisor>(m0);
     const bool exact = q.exact_row && row_valid && !q.zero_scale;
     if (exact) {
       // rare: the stage is still needed by the out-of-line exact path
@@ -491,7 +492,7 @@ dynamic_quant_generic_kernel(const RowQuantArgs a) {
     }
     __syncthreads();  // red[] is rewritten by the next row
 
-    RowQuant q = kA ? make_asym(m0, m1, C::kDivisor, C::kOffsetOpt) : make_sym(m0, C::kDivisor);
+    RowQuant q = kA ? make_asym<C::kDivisor, C::kOffsetOptInt>(m0, m1) : make_sym<C::kDivisor>(m0);
     if (!row_valid) {
       q.scale = 0.0f;
       q.offset = 0.0f;
