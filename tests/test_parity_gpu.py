@@ -357,8 +357,8 @@ def _ada_inputs(b, s, h, dtype, pdtype, seed, x_mean=0.0, x_std=1.0):
     return x, sc, sh, w, bias, sm
 
 
-ADA_SHAPES = [(1, 1, 8), (2, 3, 64), (3, 17, 1000), (2, 9, 3072), (1, 5, 4096), (2, 3, 4104), (1, 2, 8192),
-              (2, 3, 77)]
+ADA_SHAPES = [(1, 1, 8), (2, 3, 64), (1, 3, 256), (1, 3, 512), (2, 7, 1024), (3, 11, 2048), (3, 17, 1000),
+              (2, 9, 3072), (1, 5, 4096), (2, 3, 4104), (1, 2, 8192), (2, 3, 77)]
 
 
 @pytest.mark.parametrize("shape", ADA_SHAPES, ids=[f"{b}x{s}x{h}" for b, s, h in ADA_SHAPES])
@@ -385,6 +385,17 @@ def test_ada_optional_parameters(dq, opt):
         kw["sm"] = sm
     want = oracle.ada_layernorm_quant(x, sc, sh, kw["w"], kw["b"], kw["sm"], epsilon=1e-5)
     got = run_ada_gpu(dq, x, sc, sh, kw["w"], kw["b"], kw["sm"], 1e-5, misalign=opt == "misaligned")
+    assert_ada_close(got, want)
+
+
+@pytest.mark.parametrize("h", [3072, 1000, 1024])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_ada_large_mean_rows(dq, h, dtype):
+    """Rows with mean far above their spread (1000 +- 3): E(x) must be accurate
+    to well below the spread, or most codes move."""
+    x, sc, sh, w, bias, sm = _ada_inputs(3, 13, h, dtype, torch.bfloat16, seed=h + 5, x_mean=1000.0, x_std=3.0)
+    want = oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6)
+    got = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
     assert_ada_close(got, want)
 
 
