@@ -147,14 +147,14 @@ dq_status launch_programmatic(void (*kernel)(const Args), const Args& a, int gri
 // Row-group geometry of the bulk-copy DynamicQuant kernel: a group of
 // tpr = 32 * G threads owns a row, VPT in {2, 4, 8} vectors per thread; the
 // shape wasting the fewest lanes wins, then the one whose VPT is closest to
-// the target: 4 with smooth scales (the fp32 products of pass 1 then stay in
-// registers for pass 2), 8 without (more elements per thread amortize the
-// per-row work). DQ_WARP_STAGES row buffers per group; groups per CTA so that
+// the target VPT (8 by default: more elements per thread amortize the
+// per-row work; with smooth scales the fp32 products of pass 1 stay in
+// registers for pass 2). DQ_WARP_STAGES row buffers per group; groups per CTA so that
 // a CTA holds about DQ_WARP_CTA_BYTES_SMOOTH / _PLAIN of rows (measured: the
 // smooth-scale path prefers several groups sharing a CTA, the plain path
 // smaller CTAs).
 #ifndef DQ_TARGET_VPT_SMOOTH
-#define DQ_TARGET_VPT_SMOOTH 4
+#define DQ_TARGET_VPT_SMOOTH 8
 #endif
 #ifndef DQ_TARGET_VPT_PLAIN
 #define DQ_TARGET_VPT_PLAIN 8
