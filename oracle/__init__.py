@@ -4,7 +4,8 @@ A plain, single-threaded C++ implementation (``dq_oracle.cpp``) of the
 formulas on the aclnnDynamicQuantV2 page ("Formula": symmetric and
 asymmetric quantization, with and without smooth scales; MoE smooth-scale
 selection from "Description") and the aclnnAdaLayerNormQuant page
-("Formula", steps 1-5), wrapped here with ctypes + numpy.
+("Formula", steps 1-5), plus the PER_TOKEN dequantizer of the AntiQuantize
+page (one scale and offset per row), wrapped here with ctypes + numpy.
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package. It shares nothing with the CUDA library: no
@@ -75,6 +76,12 @@ def _load():
             lib.oracle_ada_layernorm_quant.argtypes = [vp, ci, i64, i64, i64, vp, vp, vp, vp, vp, ci, f32,
                                                        vp, vp]
             lib.oracle_ada_layernorm_quant.restype = ci
+            lib.oracle_dequant_per_token.argtypes = [vp, ci, i64, i64, vp, vp, ci, ci, vp]
+            lib.oracle_dequant_per_token.restype = ci
+            lib.oracle_float_to_half_bits.argtypes = [f32]
+            lib.oracle_float_to_half_bits.restype = ctypes.c_uint16
+            lib.oracle_float_to_bfloat16_bits.argtypes = [f32]
+            lib.oracle_float_to_bfloat16_bits.restype = ctypes.c_uint16
             _lib = lib
     return _lib
 
@@ -195,6 +202,45 @@ def ada_layernorm_quant(x, ada_scale, ada_shift, weight=None, bias=None, smooth=
     _check(lib.oracle_ada_layernorm_quant(_ptr(xb), xc, batch, seq, hidden, _ptr(a), _ptr(s), _ptr(w), _ptr(b),
                                           _ptr(sm), pc, ctypes.c_float(epsilon), _ptr(out), _ptr(qs)))
     return out, qs
+
+
+def dequant_per_token(codes, scale, offset=None, y_dtype: str = "int8", cols: int | None = None,
+                      out_dtype: str = "f32", scale_dtype: str | None = None):
+    """Per-token dequantization (AntiQuantize, PER_TOKEN policy), read as the
+    inverse of the quantizer: out = (code - offset) * scale in binary32, then
+    rounded to ``out_dtype`` ("f32" | "f16" | "bf16").
+
+    ``codes``: int8 [rows, cols], packed uint8 [rows, cols/2] ("int4") or
+    uint32 [rows, cols/8] ("int32"); ``scale``, ``offset``: [rows] floats.
+    Returns float32 for "f32", float16 for "f16" and the uint16 bit patterns
+    for "bf16".
+    """
+    lib = _load()
+    yc = {"int8": Y_INT8, "int4": Y_INT4X2, "int32": Y_INT32}[y_dtype]
+    cb = np.ascontiguousarray(codes)
+    rows = int(cb.shape[0])
+    if cols is None:
+        cols = int(cb.shape[1]) * {Y_INT8: 1, Y_INT4X2: 2, Y_INT32: 8}[yc]
+    sb, sc = _float_buffer(scale, scale_dtype)
+    ob = None
+    if offset is not None:
+        ob, oc = _float_buffer(offset, scale_dtype)
+        if oc != sc:
+            raise TypeError("oracle: offset must have the dtype of scale")
+    oc_out = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
+    out = np.zeros((rows, cols), dtype=np.float32 if oc_out == F32 else np.uint16)
+    _check(lib.oracle_dequant_per_token(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, oc_out, _ptr(out)))
+    return out.view(np.float16) if oc_out == F16 else out
+
+
+def float_to_half_bits(v: float) -> int:
+    """binary32 -> binary16 bit pattern, round to nearest even."""
+    return int(_load().oracle_float_to_half_bits(ctypes.c_float(v)))
+
+
+def float_to_bfloat16_bits(v: float) -> int:
+    """binary32 -> bfloat16 bit pattern, round to nearest even."""
+    return int(_load().oracle_float_to_bfloat16_bits(ctypes.c_float(v)))
 
 
 def unpack_int4(packed: np.ndarray, cols: int) -> np.ndarray:

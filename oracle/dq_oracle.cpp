@@ -44,6 +44,13 @@
 //   * packed INT4: element 2j goes to bits 0-3 and element 2j+1 to bits 4-7 of
 //     byte j (two's-complement nibbles); INT32: element 8j+k goes to bits
 //     4k..4k+3 of word j;
+//   * AntiQuantize, PER_TOKEN policy (one scale and offset per row): the
+//     formula was lost from the page; the dequantizer is read as the inverse
+//     of the quantizer above, out = (code - offset) * scale in binary32, then
+//     rounded once to the output type (round to nearest even). Only the
+//     page's printed example (scale 1, offset 0: output = input) pins it
+//     directly; the sign of the offset is parity unpinned by the pages (the
+//     tests pin it against the quantizer, whose inverse it is read to be);
 //   * AdaLayerNormQuant: the mean and the biased variance (divide by H) are
 //     accumulated in double over the fp32-widened row and rounded to float
 //     once; epsilon is added inside the square root; x - E(x) is divided by
@@ -101,6 +108,69 @@ float load_element(const void* base, int dtype, int64_t index) {
     default:
       return NAN;
   }
+}
+
+// ---- narrowing of binary32 to the 16-bit storage types (round to nearest even)
+
+// A finite value v > 0 with 2^e <= v < 2^(e+1) is written with `fraction_bits`
+// bits after the leading one: scaling by 2^(fraction_bits - e) makes the
+// significand an integer in [2^fraction_bits, 2^(fraction_bits+1)) plus a
+// fraction, which nearbyint rounds to nearest even (exact scaling by powers of
+// two in double). Below the smallest normal exponent the spacing stays fixed
+// (subnormals). Returns the rounded significand and updates e.
+double round_significand(double v, int fraction_bits, int min_exponent, int* e) {
+  int exp2;
+  std::frexp(v, &exp2);  // v = m * 2^exp2, m in [0.5, 1)
+  int ee = exp2 - 1;     // 2^ee <= v < 2^(ee+1)
+  if (ee < min_exponent) ee = min_exponent;  // subnormal: fixed spacing 2^(min_exponent - fraction_bits)
+  double q = std::nearbyint(std::ldexp(v, fraction_bits - ee));
+  if (q >= std::ldexp(1.0, fraction_bits + 1)) {  // rounded up into the next binade
+    q = std::ldexp(1.0, fraction_bits);
+    ++ee;
+  }
+  *e = ee;
+  return q;
+}
+
+uint16_t narrow_to_half(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, sizeof x);
+  const uint16_t sign = static_cast<uint16_t>((x >> 16) & 0x8000u);
+  if (std::isnan(f)) return static_cast<uint16_t>(sign | 0x7E00u);
+  if (std::isinf(f)) return static_cast<uint16_t>(sign | 0x7C00u);
+  const double v = std::fabs(static_cast<double>(f));
+  if (v == 0.0) return sign;
+  int e;
+  const double q = round_significand(v, 10, -14, &e);  // binary16: 10 fraction bits, exponents -14..15
+  if (e > 15) return static_cast<uint16_t>(sign | 0x7C00u);  // overflow: infinity
+  const uint32_t sig = static_cast<uint32_t>(q);
+  if (sig < 1024u) return static_cast<uint16_t>(sign | sig);  // subnormal (e == -14, no leading one)
+  return static_cast<uint16_t>(sign | (static_cast<uint32_t>(e + 15) << 10) | (sig - 1024u));
+}
+
+uint16_t narrow_to_bfloat16(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, sizeof x);
+  const uint16_t sign = static_cast<uint16_t>((x >> 16) & 0x8000u);
+  if (std::isnan(f)) return static_cast<uint16_t>(sign | 0x7FC0u);
+  if (std::isinf(f)) return static_cast<uint16_t>(sign | 0x7F80u);
+  const double v = std::fabs(static_cast<double>(f));
+  if (v == 0.0) return sign;
+  int e;
+  const double q = round_significand(v, 7, -126, &e);  // bfloat16: 7 fraction bits, exponents -126..127
+  if (e > 127) return static_cast<uint16_t>(sign | 0x7F80u);
+  const uint32_t sig = static_cast<uint32_t>(q);
+  if (sig < 128u) return static_cast<uint16_t>(sign | sig);
+  return static_cast<uint16_t>(sign | (static_cast<uint32_t>(e + 127) << 7) | (sig - 128u));
+}
+
+// Signed code c of a container (ORACLE_Y_*): int8, or 4-bit two's complement
+// with element 2j in the low nibble of byte j (INT32 words hold the same bytes).
+int load_code(const void* y, int y_dtype, int64_t index) {
+  if (y_dtype == ORACLE_Y_INT8) return static_cast<const int8_t*>(y)[index];
+  const uint8_t byte = static_cast<const uint8_t*>(y)[index / 2];
+  const int nibble = (index % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+  return nibble >= 8 ? nibble - 16 : nibble;
 }
 
 bool is_float_dtype(int dtype) {
@@ -328,5 +398,37 @@ int oracle_ada_layernorm_quant(const void* x, int x_dtype, int64_t batch, int64_
   return oracle_dynamic_quant(y.data(), ORACLE_F32, rows, hidden, nullptr, ORACLE_F32, nullptr, 0,
                               ORACLE_SYMMETRIC, ORACLE_Y_INT8, out, quant_scale, nullptr);
 }
+
+int oracle_dequant_per_token(const void* y, int y_dtype, int64_t rows, int64_t cols,
+                             const void* scale, const void* offset, int scale_dtype,
+                             int out_dtype, void* out) {
+  if (rows < 0 || cols < 1) return ORACLE_ERR_SHAPE;
+  if (y_dtype != ORACLE_Y_INT8 && y_dtype != ORACLE_Y_INT4X2 && y_dtype != ORACLE_Y_INT32) return ORACLE_ERR_DTYPE;
+  if (y_dtype == ORACLE_Y_INT4X2 && cols % 2 != 0) return ORACLE_ERR_SHAPE;
+  if (y_dtype == ORACLE_Y_INT32 && cols % 8 != 0) return ORACLE_ERR_SHAPE;
+  if (!is_float_dtype(scale_dtype) || !is_float_dtype(out_dtype)) return ORACLE_ERR_DTYPE;
+  if (rows > 0 && (y == nullptr || scale == nullptr || out == nullptr)) return ORACLE_ERR_ARGUMENT;
+  for (int64_t r = 0; r < rows; ++r) {
+    const float s = load_element(scale, scale_dtype, r);
+    const float o = offset != nullptr ? load_element(offset, scale_dtype, r) : 0.0f;
+    for (int64_t c = 0; c < cols; ++c) {
+      const int64_t i = r * cols + c;
+      float v = static_cast<float>(load_code(y, y_dtype, i));
+      if (offset != nullptr) v = v - o;
+      v = v * s;
+      if (out_dtype == ORACLE_F32) {
+        static_cast<float*>(out)[i] = v;
+      } else if (out_dtype == ORACLE_F16) {
+        static_cast<uint16_t*>(out)[i] = narrow_to_half(v);
+      } else {
+        static_cast<uint16_t*>(out)[i] = narrow_to_bfloat16(v);
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+uint16_t oracle_float_to_half_bits(float f) { return narrow_to_half(f); }
+uint16_t oracle_float_to_bfloat16_bits(float f) { return narrow_to_bfloat16(f); }
 
 }  // extern "C"

@@ -51,6 +51,24 @@ int oracle_ada_layernorm_quant(const void* x, int x_dtype, int64_t batch, int64_
                                int param_dtype, float epsilon,
                                int8_t* out, float* quant_scale);
 
+/* Per-token dequantization (AntiQuantize, PER_TOKEN policy: one scale and
+ * offset per row of an [m, n] source). The pages print no formula for it; the
+ * reading is the inverse of aclnnDynamicQuantV2's quantizer:
+ *   out[r,c] = (code[r,c] - offset[r]) * scale[r]   (binary32, each operation
+ *   rounded; the subtraction only when offset is given), then rounded to
+ *   out_dtype (round to nearest even).
+ * y: codes in a container of y_dtype (ORACLE_Y_*), [rows, cols] codes;
+ * scale, offset (NULL allowed): [rows] of scale_dtype; out: [rows, cols] of
+ * out_dtype (float, or the uint16 bit patterns of binary16 / bfloat16). */
+int oracle_dequant_per_token(const void* y, int y_dtype, int64_t rows, int64_t cols,
+                             const void* scale, const void* offset, int scale_dtype,
+                             int out_dtype, void* out);
+
+/* binary32 -> binary16 / bfloat16 bit patterns, round to nearest even (the
+ * narrowing the dequantizer ends with; exported for its pins). */
+uint16_t oracle_float_to_half_bits(float f);
+uint16_t oracle_float_to_bfloat16_bits(float f);
+
 #ifdef __cplusplus
 }
 #endif

@@ -464,3 +464,137 @@ def test_symmetric_quotient_near_ties(oracle_mod):
     y, scale, _ = oracle_mod.dynamic_quant(row)
     want, _, _ = ex.exact_codes_row(row[0], "symmetric", False)
     assert list(y[0].astype(int)) == want
+
+
+# ---------------------------------------------------------------- PER_TOKEN dequantization (AntiQuantize)
+
+def _load_antiquant_golden():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "antiquant_per_token.txt")
+    recs = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        y_dtype, codes, scale, offset, out_dtype, want = (f.strip() for f in line.split("|"))
+        rows = lambda t, conv=float: [[conv(v) for v in r.split()] for r in t.split(";")]
+        recs.append(dict(y_dtype=y_dtype, codes=np.array(rows(codes, int), np.int64),
+                         scale=[float(v) for v in scale.split()],
+                         offset=None if offset == "-" else [float(v) for v in offset.split()],
+                         out_dtype=out_dtype, want=np.array(rows(want), np.float64)))
+    return recs
+
+
+def _pack_int4(codes):
+    c = (np.asarray(codes, np.int64) & 0xF).astype(np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def _as_float64(out, out_dtype):
+    if out_dtype == "bf16":
+        return (out.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return out.astype(np.float64)
+
+
+ANTIQUANT_RECORDS = _load_antiquant_golden()
+
+
+@pytest.mark.parametrize("rec", ANTIQUANT_RECORDS, ids=[f"antiquant{i + 1}" for i in range(len(ANTIQUANT_RECORDS))])
+def test_antiquant_worked_examples(oracle_mod, rec):
+    codes = rec["codes"]
+    y = codes.astype(np.int8) if rec["y_dtype"] == "int8" else _pack_int4(codes)
+    sdt = np.float16 if rec["out_dtype"] == "f16" else np.float32
+    scale = np.array(rec["scale"], sdt)
+    offset = None if rec["offset"] is None else np.array(rec["offset"], sdt)
+    out = oracle_mod.dequant_per_token(y, scale, offset, y_dtype=rec["y_dtype"], cols=codes.shape[1],
+                                       out_dtype=rec["out_dtype"])
+    np.testing.assert_array_equal(_as_float64(out, rec["out_dtype"]), rec["want"])
+
+
+def test_narrowing_matches_library_conversions(oracle_mod):
+    """binary32 -> binary16 (numpy) and -> bfloat16 (torch), round to nearest even:
+    random bit patterns plus ties, subnormals, overflow and specials. The values
+    go through the dequantizer as code 1 times a per-row scale (exact)."""
+    import torch
+
+    rng = np.random.default_rng(7)
+    bits = rng.integers(0, 2 ** 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    v = bits.view(np.float32)
+    ties_h = (np.arange(-3000, 3000, dtype=np.float64) + 0.5) * 2.0 ** -24       # subnormal half ties
+    ties_h2 = (np.arange(1024, 2048, dtype=np.float64) + 0.5) * 2.0 ** -10      # normal half ties in [1, 2)
+    ties_b = (np.arange(128, 256, dtype=np.float64) + 0.5) * 2.0 ** -7          # bfloat16 ties in [1, 2)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 65504.0, 65519.99, 65520.0, 65536.0, 6e-8, 3e-8,
+                        2.0 ** -149, 3.4e38, -3.4e38, 1e-40], np.float64)
+    v = np.concatenate([v, ties_h.astype(np.float32), ties_h2.astype(np.float32), ties_b.astype(np.float32),
+                        special.astype(np.float32)])
+    v = v[np.isfinite(v) | np.isinf(v)]
+    ones = np.ones((v.size, 1), np.int8)
+    got_h = oracle_mod.dequant_per_token(ones, v, out_dtype="f16")[:, 0]
+    with np.errstate(over="ignore"):
+        want_h = v.astype(np.float16)
+    assert np.array_equal(got_h.view(np.uint16), want_h.view(np.uint16))
+    got_b = oracle_mod.dequant_per_token(ones, v, out_dtype="bf16")[:, 0]
+    want_b = torch.from_numpy(v.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got_b, want_b)
+    nan = oracle_mod.dequant_per_token(np.ones((1, 1), np.int8), np.array([np.nan], np.float32), out_dtype="bf16")
+    assert (int(nan[0, 0]) & 0x7F80) == 0x7F80 and (int(nan[0, 0]) & 0x7F) != 0
+
+
+@pytest.mark.parametrize("mode,y_dtype", [("symmetric", "int8"), ("asymmetric", "int8"), ("symmetric", "int4"),
+                                          ("asymmetric", "int4"), ("asymmetric", "int32")])
+def test_dequant_inverts_the_quantizer(oracle_mod, mode, y_dtype):
+    """quant then dequant returns every element to within half a quantization
+    step (plus fp32 rounding): |x - (q - offset) * scale| <= scale / 2 * (1 + 2^-20).
+    Read with the other offset sign, asymmetric rows miss by ~2 * offset * scale."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((64, 96)) * rng.uniform(0.01, 50, size=(64, 1)) + rng.uniform(-5, 5, size=(64, 1)))
+    x = x.astype(np.float32)
+    y, scale, offset = oracle_mod.dynamic_quant(x, mode=mode, y_dtype=y_dtype)
+    back = oracle_mod.dequant_per_token(y, scale, offset, y_dtype=y_dtype, cols=96, out_dtype="f32")
+    err = np.abs(back.astype(np.float64) - x.astype(np.float64))
+    bound = scale.astype(np.float64)[:, None] / 2 * (1 + 2.0 ** -20) + 1e-30
+    assert np.all(err <= bound)
+    if offset is not None:
+        # the other sign moves every element of a row by 2 * offset * scale
+        wrong = ((_codes_signed(oracle_mod, y, y_dtype, 96) + offset[:, None]) * scale[:, None]).astype(np.float32)
+        far = np.abs(offset) >= 1
+        assert far.sum() > 10
+        miss = np.abs(wrong - x).max(axis=1)
+        assert np.all(miss[far] >= 1.5 * scale[far])
+
+
+def _codes_signed(oracle_mod, y, y_dtype, cols):
+    if y_dtype == "int8":
+        return y.astype(np.float64)
+    if y_dtype == "int4":
+        return oracle_mod.unpack_int4(y, cols).astype(np.float64)
+    return oracle_mod.unpack_int4(y.view(np.uint8).reshape(y.shape[0], -1), cols).astype(np.float64)
+
+
+def test_dequant_power_of_two_scales_are_exact(oracle_mod):
+    """scale 2^k and integer offsets: (q - o) * 2^k is exact in binary32."""
+    rng = np.random.default_rng(3)
+    codes = rng.integers(-128, 128, size=(40, 64)).astype(np.int8)
+    k = rng.integers(-20, 20, size=40)
+    scale = np.ldexp(np.ones(40), k).astype(np.float32)
+    off = rng.integers(-128, 128, size=40).astype(np.float32)
+    out = oracle_mod.dequant_per_token(codes, scale, off, out_dtype="f32")
+    want = (codes.astype(np.float64) - off[:, None]) * np.ldexp(1.0, k)[:, None]
+    np.testing.assert_array_equal(out.astype(np.float64), want)
+
+
+def test_dequant_int32_container_matches_int4(oracle_mod):
+    rng = np.random.default_rng(4)
+    codes = rng.integers(-8, 8, size=(5, 32))
+    packed = _pack_int4(codes)
+    scale = rng.uniform(0.1, 2, 5).astype(np.float32)
+    a = oracle_mod.dequant_per_token(packed, scale, y_dtype="int4", cols=32)
+    b = oracle_mod.dequant_per_token(packed.view(np.uint32), scale, y_dtype="int32", cols=32)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(a, (codes.astype(np.float32) * scale[:, None]).astype(np.float32))
+
+
+def test_dequant_shape_errors(oracle_mod):
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.dequant_per_token(np.zeros((2, 3), np.uint8), np.ones(2, np.float32), y_dtype="int4", cols=5)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.dequant_per_token(np.zeros((2, 1), np.uint32), np.ones(2, np.float32), y_dtype="int32", cols=4)
