@@ -53,8 +53,12 @@ FALLBACK_HBM_GBS = 6650.0
 def algorithmic_bytes(wl) -> int:
     """HBM bytes one call must move: x read, codes + per-row floats written, side tables read."""
     t = wl.tensors
-    x = t["x"]
     rows, cols = wl.rows, wl.cols
+    if wl.kind == "dequant_per_token":
+        # codes + per-row scale (and offset) read, [rows, cols] outputs written
+        total = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
+        return int(total + rows * cols * {"f32": 4, "f16": 2, "bf16": 2}[wl.out_dtype])
+    x = t["x"]
     total = x.numel() * x.element_size()
     if wl.kind == "dynamic_quant":
         code_bytes = rows * cols if wl.y_dtype == "int8" else rows * cols // 2
@@ -71,10 +75,20 @@ def algorithmic_bytes(wl) -> int:
     return int(total)
 
 
+def workload_config(wl) -> dict:
+    """The config keys that describe a workload's operation and types."""
+    if wl.kind == "dequant_per_token":
+        return {"operation": "dequant_per_token", "rows": wl.rows, "cols": wl.cols, "y_dtype": wl.y_dtype,
+                "scale_dtype": str(wl.tensors["scale"].dtype).replace("torch.", ""), "out_dtype": wl.out_dtype,
+                "offset": wl.tensors.get("offset") is not None}
+    return {"operation": wl.kind, "x_dtype": "bf16" if "bf16" in wl.name else "f16", "rows": wl.rows,
+            "cols": wl.cols, "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric", "y_dtype": wl.y_dtype}
+
+
 def launches_per_call(wl) -> int:
-    """Kernels one C-ABI call launches: DynamicQuant one; AdaLayerNormQuant two
-    (the per-batch affine table, then the row kernel)."""
-    return 1 if wl.kind == "dynamic_quant" else 2
+    """Kernels one C-ABI call launches: DynamicQuant and the dequantizer one;
+    AdaLayerNormQuant two (the per-batch affine table, then the row kernel)."""
+    return 2 if wl.kind == "ada_layernorm_quant" else 1
 
 
 def measured_peaks():
@@ -229,10 +243,14 @@ class Launcher:
         self.stream = torch.cuda.Stream(device)
         self.sptr = self.stream.cuda_stream
         self.sets = []
-        xs = t["x"].to(device)
+        xs = wl.primary.to(device)
         for i in range(sets):
             x = xs if i == 0 else xs.clone()
-            if wl.kind == "dynamic_quant":
+            if wl.kind == "dequant_per_token":
+                out = torch.empty((wl.rows, wl.cols), dtype={"f32": torch.float32, "f16": torch.float16,
+                                                              "bf16": torch.bfloat16}[wl.out_dtype], device=device)
+                self.sets.append(dict(x=x, out=out))
+            elif wl.kind == "dynamic_quant":
                 cols = wl.cols
                 ycols = cols if wl.y_dtype == "int8" else (cols // 2 if wl.y_dtype == "int4" else cols // 8)
                 ydt = {"int8": torch.int8, "int4": torch.uint8, "int32": torch.int32}[wl.y_dtype]
@@ -244,8 +262,10 @@ class Launcher:
                 out = torch.empty(tuple(t["x"].shape), dtype=torch.int8, device=device)
                 qs = torch.empty(tuple(t["x"].shape[:2]), dtype=torch.float32, device=device)
                 self.sets.append(dict(x=x, out=out, qs=qs))
-        self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k != "x"}
-        if wl.kind == "dynamic_quant":
+        self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k not in ("x", "y")}
+        if wl.kind == "dequant_per_token":
+            self.ws_bytes, self.ws = 0, None
+        elif wl.kind == "dynamic_quant":
             gi = self.side.get("group_index")
             self.ngroups = int(gi.numel()) if gi is not None else 0
             x_dt = dq.DQ_BF16 if t["x"].dtype == torch.bfloat16 else dq.DQ_F16
@@ -270,8 +290,14 @@ class Launcher:
         p = lambda t: None if t is None else t.data_ptr()
         code = {torch.float32: dq.DQ_F32, torch.float16: dq.DQ_F16, torch.bfloat16: dq.DQ_BF16}
         self.calls = []
+        ycode = {"int8": dq.DQ_INT8, "int4": dq.DQ_INT4X2, "int32": dq.DQ_INT32}
         for s in self.sets:
-            if wl.kind == "dynamic_quant":
+            if wl.kind == "dequant_per_token":
+                sc, off = self.side["scale"], self.side.get("offset")
+                args = (p(s["x"]), ycode[wl.y_dtype], wl.rows, wl.cols, p(sc), p(off), code[sc.dtype],
+                        p(s["out"]), code[s["out"].dtype], self.sptr)
+                self.calls.append((dq.dq_dequant_per_token, args))
+            elif wl.kind == "dynamic_quant":
                 sm = self.side.get("smooth")
                 gi = self.side.get("group_index")
                 args = (p(s["x"]), code[s["x"].dtype], wl.rows, wl.cols, p(sm), code[sm.dtype] if sm is not None
@@ -306,7 +332,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(device)
     wl = workloads.make(args.workload, rows=args.rows)
     nbytes = algorithmic_bytes(wl)
-    per_set = wl.tensors["x"].numel() * wl.tensors["x"].element_size() + nbytes
+    per_set = wl.primary.numel() * wl.primary.element_size() + nbytes
     sets = max(2, math.ceil(3 * L2_BYTES / per_set))
     L = Launcher(dq, wl, device, sets)
     torch.cuda.synchronize(device)
@@ -378,11 +404,7 @@ def run_ours(args, world, rank, local):
             "data": "synthetic",
             "config": {
                 "workload": args.workload,
-                "x_dtype": "bf16" if "bf16" in args.workload else "f16",
-                "rows": wl.rows,
-                "cols": wl.cols,
-                "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric",
-                "y_dtype": wl.y_dtype,
+                **workload_config(wl),
                 "algorithmic_bytes_per_step": nbytes,
                 "rows_per_s": round(rows_per_s, 1),
                 "parallelism": f"dp{world} (independent row batches, no collective)",
@@ -398,8 +420,10 @@ def run_ours(args, world, rank, local):
                 "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy kernel)" if peak_kind == "measured"
                 else "fallback 6.65 TB/s",
                 "traffic": traffic,
-                "kernel": "dynamic_quant_tma_kernel" if wl.kind == "dynamic_quant" else
-                "ada_layernorm_quant_tma_kernel (time of the whole call: affine-table kernel included)",
+                "kernel": {"dynamic_quant": "dynamic_quant_tma_kernel",
+                           "dequant_per_token": "dequant_per_token_vec_kernel",
+                           "ada_layernorm_quant": "ada_layernorm_quant_tma_kernel (time of the whole call: "
+                                                  "affine-table kernel included)"}[wl.kind],
             },
             "clocks": clocks,
             "gpu_launches": args.steps * launches_per_call(wl),
@@ -430,7 +454,12 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
     sets = []
     for _ in range(nsets):
         d_in = {k: (v.to(device) if v is not None else None) for k, v in host_in.items()}  # outputs sized by a real call
-        if wl.kind == "dynamic_quant":
+        if wl.kind == "dequant_per_token":
+            o = dq.dequant_per_token(d_in["y"], d_in["scale"], d_in.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
+                                     out_dtype={"f32": torch.float32, "f16": torch.float16,
+                                                "bf16": torch.bfloat16}[wl.out_dtype], stream=s_call.cuda_stream)
+            outs = (o,)
+        elif wl.kind == "dynamic_quant":
             y, sc, off, ws = dq.dynamic_quant(d_in["x"], d_in.get("smooth"), d_in.get("group_index"), mode=wl.mode,
                                               y_dtype=wl.y_dtype, check=False, stream=s_call.cuda_stream)
             outs = (y, sc, off, ws)
@@ -442,7 +471,8 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
                                                                      dq._dtype_code(d_in["ada_scale"]))
             ws = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=device) if ws_bytes else None
             outs = (y, sc, ws)
-        results = [o for o in (outs[:3] if wl.kind == "dynamic_quant" else outs[:2]) if o is not None]
+        keep = {"dynamic_quant": 3, "ada_layernorm_quant": 2, "dequant_per_token": 1}[wl.kind]
+        results = [o for o in outs[:keep] if o is not None]
         h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in results]
         ev = {n: torch.cuda.Event() for n in ("in", "call", "out")}
         sets.append({"in": d_in, "outs": outs, "results": results, "h_out": h_out, "ev": ev, "used": False})
@@ -461,7 +491,10 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
             ev["in"].record(s_in)
         s_call.wait_event(ev["in"])
         d = st["in"]
-        if wl.kind == "dynamic_quant":
+        if wl.kind == "dequant_per_token":
+            dq.dequant_per_token(d["y"], d["scale"], d.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
+                                 out=st["outs"][0], stream=s_call.cuda_stream)
+        elif wl.kind == "dynamic_quant":
             dq.dynamic_quant(d["x"], d.get("smooth"), d.get("group_index"), mode=wl.mode, y_dtype=wl.y_dtype,
                              out=st["outs"], stream=s_call.cuda_stream)
         else:
@@ -506,6 +539,11 @@ def _oracle_rows(wl, r0, r1):
     import oracle
 
     t = wl.tensors
+    if wl.kind == "dequant_per_token":
+        off = t.get("offset")
+        return oracle.dequant_per_token(t["y"][r0:r1].numpy(), t["scale"][r0:r1],
+                                        None if off is None else off[r0:r1], y_dtype=wl.y_dtype, cols=wl.cols,
+                                        out_dtype=wl.out_dtype)
     if wl.kind == "dynamic_quant":
         gi = t.get("group_index")
         smooth = t.get("smooth")
@@ -590,9 +628,8 @@ def run_reference(args, world, rank):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload, "x_dtype": "bf16" if "bf16" in args.workload else "f16",
-                   "rows": rows, "cols": wl.cols, "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric",
-                   "y_dtype": wl.y_dtype, "rows_per_step": n, "rows_per_s": round(n * args.steps / elapsed, 1)},
+        "config": {"workload": args.workload, **workload_config(wl), "rows_per_step": n,
+                   "rows_per_s": round(n * args.steps / elapsed, 1)},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "reference arm = the CPU oracle (the pages ship no runnable implementation)",

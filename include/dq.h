@@ -1,7 +1,7 @@
 /*
  * dq.h — C ABI of the B200 (sm_100a) per-token dynamic quantization library.
  *
- * Two operations, launched asynchronously on the caller's stream:
+ * Three operations, launched asynchronously on the caller's stream:
  *
  *   dq_dynamic_quant        aclnnDynamicQuantV2, "Formula" and "Description":
  *                           per-row (per-token) symmetric or asymmetric
@@ -12,6 +12,8 @@
  *                           LayerNorm with optional weight/bias, then
  *                           y * (1 + scale) + shift, optional smooth scales,
  *                           then symmetric INT8 dynamic quantization.
+ *   dq_dequant_per_token    AntiQuantize, PER_TOKEN policy: codes back to
+ *                           floats with one scale (and offset) per row.
  *
  * plus the workspace queries of the two-phase calling convention both pages
  * describe ("...GetWorkspaceSize" first, then the run): dq_get_workspace_size
@@ -31,8 +33,8 @@
  *     through the CUDA stream like any other kernel's.
  *   - Results are deterministic: the same inputs give the same bytes on
  *     every call (both pages state deterministic implementations).
- *   - Rows are streamed through shared memory with bulk (TMA) copies; every
- *     wait in the kernels is bounded. If a copy never completes (a device
+ *   - Quantization rows are streamed through shared memory with bulk (TMA)
+ *     copies; every wait in the kernels is bounded. If a copy never completes (a device
  *     fault, never a data-dependent condition) the affected rows get NaN
  *     scales instead of the kernel hanging.
  *
@@ -210,6 +212,35 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype,
                                  dq_dtype param_dtype, float epsilon,
                                  int8_t* out, float* quant_scale,
                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Per-token dequantization (AntiQuantize, PER_TOKEN policy: every row of an
+ * [m, n] code matrix shares one scale and one offset, shapes [m, 1]).
+ *
+ * The page's formula images were lost; the operation is read as the inverse
+ * of dq_dynamic_quant (whose codes are round(input / scale + offset)):
+ *   out[r,c] = (code[r,c] - offset[r]) * scale[r]
+ * evaluated in IEEE binary32 with one rounding per operation (the subtraction
+ * only when offset is given), then rounded to nearest even into out_dtype.
+ * Arguments
+ *   y            device codes: DQ_INT8 int8 [rows, cols]; DQ_INT4X2 uint8
+ *                [rows, cols/2] (element 2j in the low nibble of byte j);
+ *                DQ_INT32 int32 [rows, cols/8] (the same bytes).
+ *   scale        device [rows] of scale_dtype (DQ_F32, DQ_F16 or DQ_BF16).
+ *   offset       device [rows] of scale_dtype, or NULL for no offset.
+ *   out          device [rows, cols] of out_dtype (DQ_F32, DQ_F16, DQ_BF16).
+ * The page lists int8 codes with half scales to half output, bfloat16 to
+ * bfloat16, and float scales to float, half or bfloat16 output; every
+ * combination of the three float types is accepted here.
+ * Alignment: scale/offset to their element size, out to its element size,
+ * y 4-byte for DQ_INT32. Rows whose codes and outputs are 16-byte aligned
+ * and a whole number of 16-byte code vectors take a vectorised path; others
+ * a scalar one, with the same results. rows == 0 is a no-op.
+ * Errors: DQ_ERR_NULL_POINTER, DQ_ERR_BAD_SHAPE (cols < 1, odd cols for
+ * DQ_INT4X2, cols % 8 for DQ_INT32), DQ_ERR_BAD_DTYPE, DQ_ERR_MISALIGNED,
+ * DQ_ERR_CUDA. */
+dq_status dq_dequant_per_token(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols,
+                               const void* scale, const void* offset, dq_dtype scale_dtype,
+                               void* out, dq_dtype out_dtype, cudaStream_t stream);
 
 /* Largest batch * hidden that dq_ada_layernorm_quant_noalloc accepts (its
  * fixed table holds this many 8-byte entries: 1 MiB per device). */

@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant_get_workspace_size",
-              "dq_ada_layernorm_quant", "dq_status_string"):
+              "dq_ada_layernorm_quant", "dq_dequant_per_token", "dq_status_string"):
         assert n in names
 
 
@@ -166,6 +166,38 @@ def test_ada_layernorm_quant_validation(dq_lib):
     ]
     for kw, want in cases:
         assert _ada(d, **kw) == want, kw
+
+
+def _deq(d, **kw):
+    args = dict(y=FAKE, y_dtype=d.DQ_INT8, rows=4, cols=64, scale=FAKE, offset=None, scale_dtype=d.DQ_F32,
+                out=FAKE, out_dtype=d.DQ_BF16, stream=None)
+    args.update(kw)
+    return d.dq_dequant_per_token(**args)
+
+
+def test_dequant_per_token_validation(dq_lib):
+    """Every invalid call is rejected on the host before any launch."""
+    d = dq_lib
+    assert _deq(d, rows=0, y=None, out=None) == d.DQ_OK
+    cases = [
+        (dict(y=None), d.DQ_ERR_NULL_POINTER),
+        (dict(scale=None), d.DQ_ERR_NULL_POINTER),
+        (dict(out=None), d.DQ_ERR_NULL_POINTER),
+        (dict(rows=-1), d.DQ_ERR_BAD_SHAPE),
+        (dict(cols=0), d.DQ_ERR_BAD_SHAPE),
+        (dict(y_dtype=d.DQ_INT4X2, cols=63), d.DQ_ERR_BAD_SHAPE),
+        (dict(y_dtype=d.DQ_INT32, cols=60), d.DQ_ERR_BAD_SHAPE),
+        (dict(y_dtype=d.DQ_F16), d.DQ_ERR_BAD_DTYPE),
+        (dict(scale_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
+        (dict(out_dtype=d.DQ_INT32), d.DQ_ERR_BAD_DTYPE),
+        (dict(scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(offset=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(out=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(out_dtype=d.DQ_F32, out=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(y_dtype=d.DQ_INT32, y=FAKE + 2), d.DQ_ERR_MISALIGNED),
+    ]
+    for kw, want in cases:
+        assert _deq(d, **kw) == want, kw
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

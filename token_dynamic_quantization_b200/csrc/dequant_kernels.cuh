@@ -1,0 +1,214 @@
+// Per-token dequantization (AntiQuantize, PER_TOKEN policy), sm_100a.
+//
+// One scale and one optional offset per row of an [m, n] code matrix. The
+// page's formula images were lost; the operation is the inverse of the
+// aclnnDynamicQuantV2 quantizer (codes = round(x / scale + offset)):
+//   out[r,c] = (code[r,c] - offset[r]) * scale[r]
+// in binary32, one rounding per operation, then rounded to nearest even into
+// the output type.
+//
+// The work is 1 (int8) or 0.5 (int4) byte in and 2 or 4 bytes out per element,
+// so the kernel is HBM-bound. A warp takes one chunk of a row at a time; each
+// lane streams 16-byte vectors of codes (16 int8 or 32 int4 codes), four loads
+// in flight.
+// A code becomes a float without the conversion unit: XOR with the sign bit
+// makes it an unsigned byte u = code + 128 (u = code + 8 for nibbles), a byte
+// permute places u in the low byte of the pattern of 1.5 * 2^23, and one
+// subtraction of 1.5 * 2^23 + 128 (or + 8) leaves the code exactly. Then
+// (v - offset) * scale as packed f32x2 operations and one packed conversion
+// (cvt.rn.{bf16x2,f16x2}.f32) per pair of outputs.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "dq_device.cuh"
+
+namespace dq {
+
+struct DequantArgs {
+  const void* y;       // codes
+  int64_t rows, cols;
+  const void* scale;   // [rows] of scale_dtype
+  const void* offset;  // [rows] of scale_dtype or nullptr
+  int scale_dtype;     // kF32 / kF16 / kBF16
+  void* out;           // [rows, cols] of the output type
+};
+
+enum : int { kOutF32 = 0, kOutF16 = 1, kOutBF16 = 2 };
+
+// Output element storage and pair narrowing (round to nearest even).
+template <int OUT>
+struct OutTraits;
+template <>
+struct OutTraits<kOutF32> {
+  static constexpr int kBytes = 4;
+};
+template <>
+struct OutTraits<kOutF16> {
+  static constexpr int kBytes = 2;
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ void store1(void* p, int64_t i, float v) {
+    static_cast<__half*>(p)[i] = __float2half_rn(v);
+  }
+};
+template <>
+struct OutTraits<kOutBF16> {
+  static constexpr int kBytes = 2;
+  static __device__ __forceinline__ uint32_t pack(float a, float b) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ void store1(void* p, int64_t i, float v) {
+    static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  }
+};
+
+// 1.5 * 2^23 + bias as a binary32 value: the pattern 0x4B400000 | u reads as
+// 1.5 * 2^23 + u, so subtracting this gives u - bias exactly.
+constexpr float kCodeMagic8 = 12583040.0f;  // 1.5 * 2^23 + 128
+constexpr float kCodeMagic4 = 12582920.0f;  // 1.5 * 2^23 + 8
+
+// Value of byte j (0..3) of `u` placed in the low byte of 1.5 * 2^23's pattern.
+__device__ __forceinline__ float byte_as_float(uint32_t u, int j, float magic) {
+  return __uint_as_float(__byte_perm(u, 0x4B400000u, 0x7650u | static_cast<uint32_t>(j))) - magic;
+}
+
+// The 16 (int8) or 32 (int4) codes of one 16-byte vector as floats, in element order.
+template <bool kFour>
+__device__ __forceinline__ void codes_of(const uint4& w, float (&v)[kFour ? 32 : 16]) {
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (!kFour) {
+      const uint32_t u = ws[i] ^ 0x80808080u;  // signed byte -> code + 128
+#pragma unroll
+      for (int j = 0; j < 4; ++j) v[4 * i + j] = byte_as_float(u, j, kCodeMagic8);
+    } else {
+      const uint32_t u = ws[i] ^ 0x88888888u;  // signed nibble -> code + 8
+      const uint32_t lo = u & 0x0F0F0F0Fu;        // elements 8i + 0, 2, 4, 6
+      const uint32_t hi = (u >> 4) & 0x0F0F0F0Fu;  // elements 8i + 1, 3, 5, 7
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = byte_as_float(lo, j, kCodeMagic4);
+        v[8 * i + 2 * j + 1] = byte_as_float(hi, j, kCodeMagic4);
+      }
+    }
+  }
+}
+
+// (v - offset) * scale over the vector, as packed pairs.
+template <int N, bool kOff>
+__device__ __forceinline__ void apply_row_constants(float (&v)[N], float scale, float offset) {
+#pragma unroll
+  for (int p = 0; p < N / 2; ++p) {
+    float2 t = make_float2(v[2 * p], v[2 * p + 1]);
+    if (kOff) t = __fadd2_rn(t, f2(-offset));
+    t = __fmul2_rn(t, f2(scale));
+    v[2 * p] = t.x;
+    v[2 * p + 1] = t.y;
+  }
+}
+
+template <int OUT, int N>
+__device__ __forceinline__ void store_vector(void* out_row, int vi, const float (&v)[N]) {
+  if constexpr (OUT == kOutF32) {
+    float4* o = reinterpret_cast<float4*>(out_row) + static_cast<int64_t>(vi) * (N / 4);
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) __stcs(o + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+  } else {
+    uint4* o = reinterpret_cast<uint4*>(out_row) + static_cast<int64_t>(vi) * (N / 8);
+#pragma unroll
+    for (int q = 0; q < N / 8; ++q) {
+      uint4 w;
+      w.x = OutTraits<OUT>::pack(v[8 * q + 0], v[8 * q + 1]);
+      w.y = OutTraits<OUT>::pack(v[8 * q + 2], v[8 * q + 3]);
+      w.z = OutTraits<OUT>::pack(v[8 * q + 4], v[8 * q + 5]);
+      w.w = OutTraits<OUT>::pack(v[8 * q + 6], v[8 * q + 7]);
+      __stcs(o + q, w);
+    }
+  }
+}
+
+constexpr int kDequantBlock = 256;
+constexpr int kDequantUnroll = 4;  // 16-byte code vectors in flight per lane
+
+// Rows whose code bytes are a whole number of 16-byte vectors, 16-byte
+// aligned codes and output rows. A work item is one chunk of a row: 32 lanes
+// x kDequantUnroll vectors (2048 int8 or 4096 int4 codes). Items are many
+// and small, and the grid covers them all (a grid-stride loop only beyond
+// the grid limit), so the block scheduler balances the tail.
+template <int OUT, bool kFour, bool kOff>
+__global__ void __launch_bounds__(kDequantBlock) dequant_per_token_vec_kernel(const DequantArgs a) {
+  constexpr int N = kFour ? 32 : 16;  // codes per 16-byte vector
+  constexpr int kWarps = kDequantBlock / 32;
+  pdl_launch_dependents();
+  pdl_wait_primary();  // launched as a programmatic dependent: inputs are visible from here on
+  const int lane = threadIdx.x & 31;
+  const int nvec = static_cast<int>(a.cols / N);
+  const int64_t chunks = (nvec + 32 * kDequantUnroll - 1) / (32 * kDequantUnroll);  // per row
+  const int64_t items = a.rows * chunks;
+  const int64_t row_code_bytes = kFour ? a.cols / 2 : a.cols;
+  const int64_t row_out_bytes = a.cols * OutTraits<OUT>::kBytes;
+  for (int64_t item = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); item < items;
+       item += static_cast<int64_t>(gridDim.x) * kWarps) {
+    const int64_t r = item / chunks;
+    const int v0 = static_cast<int>(item - r * chunks) * (32 * kDequantUnroll) + lane;
+    const float scale = load_param(a.scale, a.scale_dtype, r);
+    const float offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.y) + r * row_code_bytes);
+    void* dst = static_cast<uint8_t*>(a.out) + r * row_out_bytes;
+    uint4 w[kDequantUnroll];
+#pragma unroll
+    for (int u = 0; u < kDequantUnroll; ++u) {
+      const int vi = v0 + 32 * u;
+      w[u] = vi < nvec ? __ldcs(src + vi) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kDequantUnroll; ++u) {
+      const int vi = v0 + 32 * u;
+      if (vi < nvec) {
+        float v[N];
+        codes_of<kFour>(w[u], v);
+        apply_row_constants<N, kOff>(v, scale, offset);
+        store_vector<OUT, N>(dst, vi, v);
+      }
+    }
+  }
+}
+
+// Any shape and alignment: one element per thread step, grid-strided rows.
+template <int OUT, bool kFour, bool kOff>
+__global__ void __launch_bounds__(kDequantBlock) dequant_per_token_generic_kernel(const DequantArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_primary();
+  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+    const float scale = load_param(a.scale, a.scale_dtype, r);
+    const float offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
+    for (int64_t c = threadIdx.x; c < a.cols; c += kDequantBlock) {
+      const int64_t i = r * a.cols + c;
+      int code;
+      if (kFour) {
+        const uint8_t byte = static_cast<const uint8_t*>(a.y)[i >> 1];
+        const int nib = (i & 1) ? (byte >> 4) : (byte & 0xF);
+        code = nib >= 8 ? nib - 16 : nib;
+      } else {
+        code = static_cast<const int8_t*>(a.y)[i];
+      }
+      float v = static_cast<float>(code);
+      if (kOff) v = __fsub_rn(v, offset);
+      v = __fmul_rn(v, scale);
+      if constexpr (OUT == kOutF32) {
+        static_cast<float*>(a.out)[i] = v;
+      } else {
+        OutTraits<OUT>::store1(a.out, i, v);
+      }
+    }
+  }
+}
+
+}  // namespace dq

@@ -59,6 +59,8 @@ _lib.dq_ada_layernorm_quant_get_workspace_size.restype = _ci
 _lib.dq_ada_layernorm_quant.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp, _vp,
                                         _vp, _sz, _vp]
 _lib.dq_ada_layernorm_quant.restype = _ci
+_lib.dq_dequant_per_token.argtypes = [_vp, _ci, _i64, _i64, _vp, _vp, _ci, _vp, _ci, _vp]
+_lib.dq_dequant_per_token.restype = _ci
 _lib.dq_ada_layernorm_quant_noalloc.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp,
                                                 _vp, _vp]
 _lib.dq_ada_layernorm_quant_noalloc.restype = _ci
@@ -108,6 +110,11 @@ def dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift,
     return _lib.dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias,
                                        smooth, param_dtype, epsilon, out, quant_scale, workspace,
                                        workspace_bytes, stream)
+
+
+def dq_dequant_per_token(y, y_dtype, rows, cols, scale, offset, scale_dtype, out, out_dtype, stream) -> int:
+    """Raw call: pointers are ints (0/None for NULL). Returns the dq_status."""
+    return _lib.dq_dequant_per_token(y, y_dtype, rows, cols, scale, offset, scale_dtype, out, out_dtype, stream)
 
 
 def dq_ada_layernorm_quant_noalloc(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias, smooth,
@@ -227,3 +234,33 @@ def ada_layernorm_quant(x, ada_scale, ada_shift, weight=None, bias=None, smooth=
     if check and st != DQ_OK:
         raise DQError(st)
     return o, qs
+
+
+def dequant_per_token(y, scale, offset=None, y_dtype: str = "int8", cols: int | None = None,
+                      out_dtype=None, out=None, stream=None, check: bool = True):
+    """Per-token dequantization of CUDA codes ``y`` (AntiQuantize, PER_TOKEN).
+
+    ``y``: int8 [rows, cols], uint8 [rows, cols/2] ("int4") or int32
+    [rows, cols/8] ("int32"); ``scale`` / ``offset``: CUDA [rows] float
+    tensors of one dtype; ``out_dtype``: torch.float32 / float16 / bfloat16
+    (default: the scale's dtype). Returns the [rows, cols] output tensor.
+    """
+    torch = _torch()
+    yc = _YTYPES[{"int8": "int8", "int4": "int4", "int32": "int32"}[y_dtype]]
+    rows = int(y.shape[0]) if y.dim() else 0
+    if cols is None:
+        cols = int(y.shape[-1]) * {DQ_INT8: 1, DQ_INT4X2: 2, DQ_INT32: 8}[yc]
+    sdt = _dtype_code(scale)
+    if offset is not None and _dtype_code(offset) != sdt:
+        raise TypeError("offset must have the dtype of scale")
+    if out_dtype is None:
+        out_dtype = scale.dtype
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=y.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(y.device).cuda_stream
+    st = dq_dequant_per_token(_dev_ptr(y, "y"), yc, rows, cols, _dev_ptr(scale, "scale"), _dev_ptr(offset, "offset"),
+                              sdt, _dev_ptr(out, "out"), _dtype_code(out), stream)
+    if check and st != DQ_OK:
+        raise DQError(st)
+    return out

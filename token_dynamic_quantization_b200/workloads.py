@@ -26,6 +26,10 @@ LayerNorm path):
   (seed 0); adaptive scale and shift bf16 [4, 3072] ~ N(0, 0.1) (seeds 4, 5);
   LayerNorm weight bf16 [3072] ~ N(1, 0.05) (seed 6), bias ~ N(0, 0.05)
   (seed 7); smooth bf16 [3072] ~ U(0.5, 2.0) (seed 2); epsilon 1e-6.
+* ``dequant_per_token_int8_bf16_8192x4096`` (AntiQuantize page, PER_TOKEN
+  policy; the inverse of the 8192 x 4096 quantization workload): codes int8
+  [8192, 4096] uniform in [-127, 127] (seed 8), per-row scale fp32 [8192]
+  ~ U(0.001, 0.05) (seed 9), no offset, bfloat16 output.
 """
 
 from __future__ import annotations
@@ -80,19 +84,27 @@ class Workload:
     """One synthetic workload: named tensors on the CPU plus the call's options."""
 
     name: str
-    kind: str                    # "dynamic_quant" | "ada_layernorm_quant"
+    kind: str                    # "dynamic_quant" | "ada_layernorm_quant" | "dequant_per_token"
     tensors: dict = field(default_factory=dict)
     mode: str = "symmetric"      # dynamic_quant only
-    y_dtype: str = "int8"        # dynamic_quant only
+    y_dtype: str = "int8"        # code container (dynamic_quant output, dequant_per_token input)
     epsilon: float = 1e-6        # ada_layernorm_quant only
+    out_dtype: str = "bf16"      # dequant_per_token only
+
+    @property
+    def primary(self):
+        """The per-row input: x, or the codes of a dequantization."""
+        return self.tensors["y"] if self.kind == "dequant_per_token" else self.tensors["x"]
 
     @property
     def rows(self) -> int:
-        x = self.tensors["x"]
-        return int(x.numel() // x.shape[-1])
+        t = self.primary
+        return int(t.numel() // t.shape[-1])
 
     @property
     def cols(self) -> int:
+        if self.kind == "dequant_per_token":
+            return int(self.tensors["y"].shape[-1]) * {"int8": 1, "int4": 2, "int32": 8}[self.y_dtype]
         return int(self.tensors["x"].shape[-1])
 
 
@@ -102,6 +114,7 @@ WORKLOADS = (
     "moe_sym_int8_bf16_32768x7168_e64",
     "asym_int4_f16_16384x8192",
     "ada_layernorm_quant_bf16_4x4096x3072",
+    "dequant_per_token_int8_bf16_8192x4096",
 )
 
 
@@ -141,4 +154,10 @@ def make(name: str, rows: int | None = None) -> Workload:
             "smooth": uniform((h,), torch.bfloat16, 2, 0.5, 2.0),
         }
         return Workload(name, "ada_layernorm_quant", t, epsilon=1e-6)
+    if name == "dequant_per_token_int8_bf16_8192x4096":
+        r = rows or 8192
+        g = _gen(8)
+        y = torch.randint(-127, 128, (r, 4096), generator=g, dtype=torch.int32).to(torch.int8)
+        scale = uniform((r,), torch.float32, 9, 0.001, 0.05)
+        return Workload(name, "dequant_per_token", {"y": y, "scale": scale}, y_dtype="int8", out_dtype="bf16")
     raise KeyError(f"unknown workload {name!r}; known: {', '.join(WORKLOADS)}")
