@@ -4,8 +4,8 @@ A plain, single-threaded C++ implementation (``dq_oracle.cpp``) of the
 formulas on the aclnnDynamicQuantV2 page ("Formula": symmetric and
 asymmetric quantization, with and without smooth scales; MoE smooth-scale
 selection from "Description") and the aclnnAdaLayerNormQuant page
-("Formula", steps 1-5), plus the PER_TOKEN dequantizer of the AntiQuantize
-page (one scale and offset per row), wrapped here with ctypes + numpy.
+("Formula", steps 1-5), plus the PER_TOKEN and PER_GROUP dequantizers of the
+AntiQuantize page, wrapped here with ctypes + numpy.
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package. It shares nothing with the CUDA library: no
@@ -78,6 +78,8 @@ def _load():
             lib.oracle_ada_layernorm_quant.restype = ci
             lib.oracle_dequant_per_token.argtypes = [vp, ci, i64, i64, vp, vp, ci, ci, vp]
             lib.oracle_dequant_per_token.restype = ci
+            lib.oracle_dequant_per_group.argtypes = [vp, ci, i64, i64, vp, vp, ci, i64, ci, ci, vp]
+            lib.oracle_dequant_per_group.restype = ci
             lib.oracle_float_to_half_bits.argtypes = [f32]
             lib.oracle_float_to_half_bits.restype = ctypes.c_uint16
             lib.oracle_float_to_bfloat16_bits.argtypes = [f32]
@@ -230,6 +232,31 @@ def dequant_per_token(codes, scale, offset=None, y_dtype: str = "int8", cols: in
     oc_out = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
     out = np.zeros((rows, cols), dtype=np.float32 if oc_out == F32 else np.uint16)
     _check(lib.oracle_dequant_per_token(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, oc_out, _ptr(out)))
+    return out.view(np.float16) if oc_out == F16 else out
+
+
+def dequant_per_group(codes, scale, offset=None, group_size: int = 32, k_dim: int = 1, y_dtype: str = "int8",
+                      cols: int | None = None, out_dtype: str = "f32", scale_dtype: str | None = None):
+    """Per-group dequantization (AntiQuantize, PER_GROUP policy): element (i, j)
+    uses scale/offset entry (i, j // g) when ``k_dim`` = 1 (table
+    [rows, ceil(cols/g)]) or (i // g, j) when ``k_dim`` = 0 (table
+    [ceil(rows/g), cols]); value as in ``dequant_per_token``."""
+    lib = _load()
+    yc = {"int8": Y_INT8, "int4": Y_INT4X2, "int32": Y_INT32}[y_dtype]
+    cb = np.ascontiguousarray(codes)
+    rows = int(cb.shape[0])
+    if cols is None:
+        cols = int(cb.shape[1]) * {Y_INT8: 1, Y_INT4X2: 2, Y_INT32: 8}[yc]
+    sb, sc = _float_buffer(scale, scale_dtype)
+    ob = None
+    if offset is not None:
+        ob, oc = _float_buffer(offset, scale_dtype)
+        if oc != sc:
+            raise TypeError("oracle: offset must have the dtype of scale")
+    oc_out = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
+    out = np.zeros((rows, cols), dtype=np.float32 if oc_out == F32 else np.uint16)
+    _check(lib.oracle_dequant_per_group(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, int(group_size),
+                                        int(k_dim), oc_out, _ptr(out)))
     return out.view(np.float16) if oc_out == F16 else out
 
 

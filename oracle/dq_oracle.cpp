@@ -51,6 +51,11 @@
 //     page's printed example (scale 1, offset 0: output = input) pins it
 //     directly; the sign of the offset is parity unpinned by the pages (the
 //     tests pin it against the quantizer, whose inverse it is read to be);
+//   * AntiQuantize, PER_GROUP policy: every groupSize elements along the k
+//     axis (kDim 1: along a row; kDim 0: down a column) share one scale and
+//     offset of a [rows, ceil(cols/g)] or [ceil(rows/g), cols] table (the
+//     page's shapes); the value is the PER_TOKEN reading with that element's
+//     scale and offset (the page's formula images were lost here too);
 //   * AdaLayerNormQuant: the mean and the biased variance (divide by H) are
 //     accumulated in double over the fp32-widened row and rounded to float
 //     once; epsilon is added inside the square root; x - E(x) is divided by
@@ -422,6 +427,37 @@ int oracle_dequant_per_token(const void* y, int y_dtype, int64_t rows, int64_t c
         static_cast<uint16_t*>(out)[i] = narrow_to_half(v);
       } else {
         static_cast<uint16_t*>(out)[i] = narrow_to_bfloat16(v);
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+int oracle_dequant_per_group(const void* y, int y_dtype, int64_t rows, int64_t cols,
+                             const void* scale, const void* offset, int scale_dtype,
+                             int64_t group_size, int k_dim, int out_dtype, void* out) {
+  if (rows < 0 || cols < 1) return ORACLE_ERR_SHAPE;
+  if (y_dtype != ORACLE_Y_INT8 && y_dtype != ORACLE_Y_INT4X2 && y_dtype != ORACLE_Y_INT32) return ORACLE_ERR_DTYPE;
+  if (y_dtype == ORACLE_Y_INT4X2 && cols % 2 != 0) return ORACLE_ERR_SHAPE;
+  if (y_dtype == ORACLE_Y_INT32 && cols % 8 != 0) return ORACLE_ERR_SHAPE;
+  if (!is_float_dtype(scale_dtype) || !is_float_dtype(out_dtype)) return ORACLE_ERR_DTYPE;
+  if (group_size <= 0 || group_size % 32 != 0 || (k_dim != 0 && k_dim != 1)) return ORACLE_ERR_ARGUMENT;
+  if (rows > 0 && (y == nullptr || scale == nullptr || out == nullptr)) return ORACLE_ERR_ARGUMENT;
+  const int64_t groups_per_row = (cols + group_size - 1) / group_size;  // k_dim 1: table width
+  for (int64_t i = 0; i < rows; ++i) {
+    for (int64_t j = 0; j < cols; ++j) {
+      const int64_t entry = k_dim == 1 ? i * groups_per_row + j / group_size : (i / group_size) * cols + j;
+      const float s = load_element(scale, scale_dtype, entry);
+      const int64_t e = i * cols + j;
+      float v = static_cast<float>(load_code(y, y_dtype, e));
+      if (offset != nullptr) v = v - load_element(offset, scale_dtype, entry);
+      v = v * s;
+      if (out_dtype == ORACLE_F32) {
+        static_cast<float*>(out)[e] = v;
+      } else if (out_dtype == ORACLE_F16) {
+        static_cast<uint16_t*>(out)[e] = narrow_to_half(v);
+      } else {
+        static_cast<uint16_t*>(out)[e] = narrow_to_bfloat16(v);
       }
     }
   }

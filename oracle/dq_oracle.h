@@ -64,6 +64,17 @@ int oracle_dequant_per_token(const void* y, int y_dtype, int64_t rows, int64_t c
                              const void* scale, const void* offset, int scale_dtype,
                              int out_dtype, void* out);
 
+/* Per-group dequantization (AntiQuantize, PER_GROUP policy, int8 source):
+ * every group_size elements along the k axis share one scale and offset.
+ * k_dim = 1 (k runs along a row): scale/offset [rows, ceil(cols/group_size)],
+ * element (i, j) uses entry (i, j / group_size); k_dim = 0 (k runs down a
+ * column): scale/offset [ceil(rows/group_size), cols], element (i, j) uses
+ * entry (i / group_size, j). group_size > 0 and a multiple of 32. The value is
+ * computed as in oracle_dequant_per_token with that element's scale/offset. */
+int oracle_dequant_per_group(const void* y, int y_dtype, int64_t rows, int64_t cols,
+                             const void* scale, const void* offset, int scale_dtype,
+                             int64_t group_size, int k_dim, int out_dtype, void* out);
+
 /* binary32 -> binary16 / bfloat16 bit patterns, round to nearest even (the
  * narrowing the dequantizer ends with; exported for its pins). */
 uint16_t oracle_float_to_half_bits(float f);

@@ -600,3 +600,83 @@ def test_dequant_shape_errors(oracle_mod):
         oracle_mod.dequant_per_token(np.zeros((2, 3), np.uint8), np.ones(2, np.float32), y_dtype="int4", cols=5)
     with pytest.raises(oracle_mod.OracleError):
         oracle_mod.dequant_per_token(np.zeros((2, 1), np.uint32), np.ones(2, np.float32), y_dtype="int32", cols=4)
+
+
+# ---------------------------------------------------------------- PER_GROUP dequantization (AntiQuantize)
+
+def _load_group_golden():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "antiquant_per_group.txt")
+    recs = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k_dim, g, codes, scale, offset, want = (f.strip() for f in line.split("|"))
+        rows = lambda t, conv=float: np.array([[conv(v) for v in r.split()] for r in t.split(";")])
+        recs.append(dict(k_dim=int(k_dim), g=int(g), codes=rows(codes, int).astype(np.int8),
+                         scale=rows(scale).astype(np.float32), offset=rows(offset).astype(np.float32),
+                         want=rows(want)))
+    return recs
+
+
+GROUP_RECORDS = _load_group_golden()
+
+
+@pytest.mark.parametrize("rec", GROUP_RECORDS, ids=[f"group{i + 1}" for i in range(len(GROUP_RECORDS))])
+def test_per_group_worked_examples(oracle_mod, rec):
+    out = oracle_mod.dequant_per_group(rec["codes"], rec["scale"], rec["offset"], group_size=rec["g"],
+                                       k_dim=rec["k_dim"], out_dtype="f32")
+    np.testing.assert_array_equal(out.astype(np.float64), rec["want"])
+
+
+def _group_case(rows, cols, g, k_dim, seed, sdt=np.float32):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(-128, 128, size=(rows, cols)).astype(np.int8)
+    shape = (rows, -(-cols // g)) if k_dim == 1 else (-(-rows // g), cols)
+    scale = rng.uniform(1e-3, 0.1, size=shape).astype(sdt)
+    offset = rng.normal(0, 10, size=shape).astype(sdt)
+    return codes, scale, offset
+
+
+@pytest.mark.parametrize("out_dtype", ["f32", "f16", "bf16"])
+def test_per_group_row_groups_are_per_token_on_the_reshaped_rows(oracle_mod, out_dtype):
+    """kDim 1 with g | cols: each row splits into cols/g independent groups, which
+    is the PER_TOKEN dequantizer on the [rows*cols/g, g] view."""
+    rows, cols, g = 6, 256, 64
+    codes, scale, offset = _group_case(rows, cols, g, 1, seed=1)
+    got = oracle_mod.dequant_per_group(codes, scale, offset, group_size=g, k_dim=1, out_dtype=out_dtype)
+    want = oracle_mod.dequant_per_token(codes.reshape(-1, g), scale.reshape(-1), offset.reshape(-1),
+                                        out_dtype=out_dtype).reshape(rows, cols)
+    np.testing.assert_array_equal(got.view(np.uint16) if out_dtype != "f32" else got,
+                                  want.view(np.uint16) if out_dtype != "f32" else want)
+
+
+def test_per_group_one_group_per_row_is_per_token(oracle_mod):
+    codes, scale, offset = _group_case(5, 100, 128, 1, seed=2)
+    got = oracle_mod.dequant_per_group(codes, scale, offset, group_size=128, k_dim=1)
+    np.testing.assert_array_equal(got, oracle_mod.dequant_per_token(codes, scale[:, 0], offset[:, 0]))
+
+
+@pytest.mark.parametrize("rows,g", [(96, 32), (70, 32), (40, 64)])
+def test_per_group_column_groups_are_row_groups_of_the_transpose(oracle_mod, rows, g):
+    """kDim 0 on [m, n] equals kDim 1 on the transpose [n, m] with the transposed
+    table; with g >= m it is per-channel (one scale per column)."""
+    cols = 48
+    codes, scale, offset = _group_case(rows, cols, g, 0, seed=rows)
+    got = oracle_mod.dequant_per_group(codes, scale, offset, group_size=g, k_dim=0, out_dtype="bf16")
+    want = oracle_mod.dequant_per_group(np.ascontiguousarray(codes.T), np.ascontiguousarray(scale.T),
+                                        np.ascontiguousarray(offset.T), group_size=g, k_dim=1, out_dtype="bf16").T
+    np.testing.assert_array_equal(got, want)
+    if g >= rows:
+        per_channel = oracle_mod.dequant_per_token(np.ascontiguousarray(codes.T), scale[0], offset[0],
+                                                   out_dtype="bf16").T
+        np.testing.assert_array_equal(got, per_channel)
+
+
+def test_per_group_argument_errors(oracle_mod):
+    codes, scale, offset = _group_case(4, 64, 32, 1, seed=3)
+    for kw in (dict(group_size=16), dict(group_size=0), dict(group_size=48), dict(k_dim=2)):
+        args = dict(group_size=32, k_dim=1)
+        args.update(kw)
+        with pytest.raises(oracle_mod.OracleError):
+            oracle_mod.dequant_per_group(codes, scale, offset, **args)
