@@ -54,8 +54,8 @@ def algorithmic_bytes(wl) -> int:
     """HBM bytes one call must move: x read, codes + per-row floats written, side tables read."""
     t = wl.tensors
     rows, cols = wl.rows, wl.cols
-    if wl.kind == "dequant_per_token":
-        # codes + per-row scale (and offset) read, [rows, cols] outputs written
+    if wl.kind.startswith("dequant"):
+        # codes + scale (and offset) tables read, [rows, cols] outputs written
         total = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
         return int(total + rows * cols * {"f32": 4, "f16": 2, "bf16": 2}[wl.out_dtype])
     x = t["x"]
@@ -77,10 +77,13 @@ def algorithmic_bytes(wl) -> int:
 
 def workload_config(wl) -> dict:
     """The config keys that describe a workload's operation and types."""
-    if wl.kind == "dequant_per_token":
-        return {"operation": "dequant_per_token", "rows": wl.rows, "cols": wl.cols, "y_dtype": wl.y_dtype,
-                "scale_dtype": str(wl.tensors["scale"].dtype).replace("torch.", ""), "out_dtype": wl.out_dtype,
-                "offset": wl.tensors.get("offset") is not None}
+    if wl.kind.startswith("dequant"):
+        c = {"operation": wl.kind, "rows": wl.rows, "cols": wl.cols, "y_dtype": wl.y_dtype,
+             "scale_dtype": str(wl.tensors["scale"].dtype).replace("torch.", ""), "out_dtype": wl.out_dtype,
+             "offset": wl.tensors.get("offset") is not None}
+        if wl.kind == "dequant_per_group":
+            c.update(group_size=wl.group_size, k_dim=wl.k_dim)
+        return c
     return {"operation": wl.kind, "x_dtype": "bf16" if "bf16" in wl.name else "f16", "rows": wl.rows,
             "cols": wl.cols, "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric", "y_dtype": wl.y_dtype}
 
@@ -246,7 +249,7 @@ class Launcher:
         xs = wl.primary.to(device)
         for i in range(sets):
             x = xs if i == 0 else xs.clone()
-            if wl.kind == "dequant_per_token":
+            if wl.kind.startswith("dequant"):
                 out = torch.empty((wl.rows, wl.cols), dtype={"f32": torch.float32, "f16": torch.float16,
                                                               "bf16": torch.bfloat16}[wl.out_dtype], device=device)
                 self.sets.append(dict(x=x, out=out))
@@ -263,7 +266,7 @@ class Launcher:
                 qs = torch.empty(tuple(t["x"].shape[:2]), dtype=torch.float32, device=device)
                 self.sets.append(dict(x=x, out=out, qs=qs))
         self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k not in ("x", "y")}
-        if wl.kind == "dequant_per_token":
+        if wl.kind.startswith("dequant"):
             self.ws_bytes, self.ws = 0, None
         elif wl.kind == "dynamic_quant":
             gi = self.side.get("group_index")
@@ -297,6 +300,11 @@ class Launcher:
                 args = (p(s["x"]), ycode[wl.y_dtype], wl.rows, wl.cols, p(sc), p(off), code[sc.dtype],
                         p(s["out"]), code[s["out"].dtype], self.sptr)
                 self.calls.append((dq.dq_dequant_per_token, args))
+            elif wl.kind == "dequant_per_group":
+                sc, off = self.side["scale"], self.side.get("offset")
+                args = (p(s["x"]), ycode[wl.y_dtype], wl.rows, wl.cols, p(sc), p(off), code[sc.dtype], wl.group_size,
+                        wl.k_dim, p(s["out"]), code[s["out"].dtype], self.sptr)
+                self.calls.append((dq.dq_dequant_per_group, args))
             elif wl.kind == "dynamic_quant":
                 sm = self.side.get("smooth")
                 gi = self.side.get("group_index")
@@ -421,7 +429,8 @@ def run_ours(args, world, rank, local):
                 else "fallback 6.65 TB/s",
                 "traffic": traffic,
                 "kernel": {"dynamic_quant": "dynamic_quant_tma_kernel",
-                           "dequant_per_token": "dequant_per_token_vec_kernel",
+                           "dequant_per_token": "dequant_vec_kernel (per-token layout)",
+                           "dequant_per_group": "dequant_vec_kernel (per-group layout)",
                            "ada_layernorm_quant": "ada_layernorm_quant_tma_kernel (time of the whole call: "
                                                   "affine-table kernel included)"}[wl.kind],
             },
@@ -454,10 +463,15 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
     sets = []
     for _ in range(nsets):
         d_in = {k: (v.to(device) if v is not None else None) for k, v in host_in.items()}  # outputs sized by a real call
+        odt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wl.out_dtype]
         if wl.kind == "dequant_per_token":
             o = dq.dequant_per_token(d_in["y"], d_in["scale"], d_in.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
-                                     out_dtype={"f32": torch.float32, "f16": torch.float16,
-                                                "bf16": torch.bfloat16}[wl.out_dtype], stream=s_call.cuda_stream)
+                                     out_dtype=odt, stream=s_call.cuda_stream)
+            outs = (o,)
+        elif wl.kind == "dequant_per_group":
+            o = dq.dequant_per_group(d_in["y"], d_in["scale"], d_in.get("offset"), group_size=wl.group_size,
+                                     k_dim=wl.k_dim, y_dtype=wl.y_dtype, cols=wl.cols, out_dtype=odt,
+                                     stream=s_call.cuda_stream)
             outs = (o,)
         elif wl.kind == "dynamic_quant":
             y, sc, off, ws = dq.dynamic_quant(d_in["x"], d_in.get("smooth"), d_in.get("group_index"), mode=wl.mode,
@@ -471,7 +485,7 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
                                                                      dq._dtype_code(d_in["ada_scale"]))
             ws = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=device) if ws_bytes else None
             outs = (y, sc, ws)
-        keep = {"dynamic_quant": 3, "ada_layernorm_quant": 2, "dequant_per_token": 1}[wl.kind]
+        keep = {"dynamic_quant": 3, "ada_layernorm_quant": 2, "dequant_per_token": 1, "dequant_per_group": 1}[wl.kind]
         results = [o for o in outs[:keep] if o is not None]
         h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in results]
         ev = {n: torch.cuda.Event() for n in ("in", "call", "out")}
@@ -494,6 +508,9 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
         if wl.kind == "dequant_per_token":
             dq.dequant_per_token(d["y"], d["scale"], d.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
                                  out=st["outs"][0], stream=s_call.cuda_stream)
+        elif wl.kind == "dequant_per_group":
+            dq.dequant_per_group(d["y"], d["scale"], d.get("offset"), group_size=wl.group_size, k_dim=wl.k_dim,
+                                 y_dtype=wl.y_dtype, cols=wl.cols, out=st["outs"][0], stream=s_call.cuda_stream)
         elif wl.kind == "dynamic_quant":
             dq.dynamic_quant(d["x"], d.get("smooth"), d.get("group_index"), mode=wl.mode, y_dtype=wl.y_dtype,
                              out=st["outs"], stream=s_call.cuda_stream)
@@ -539,6 +556,16 @@ def _oracle_rows(wl, r0, r1):
     import oracle
 
     t = wl.tensors
+    if wl.kind == "dequant_per_group":
+        off = t.get("offset")
+        if wl.k_dim == 1:
+            tr = slice(r0, r1)
+        else:  # column groups: start the sample on a group boundary
+            r0 -= r0 % wl.group_size
+            tr = slice(r0 // wl.group_size, -(-r1 // wl.group_size))
+        return oracle.dequant_per_group(t["y"][r0:r1].numpy(), t["scale"][tr], None if off is None else off[tr],
+                                        group_size=wl.group_size, k_dim=wl.k_dim, y_dtype=wl.y_dtype, cols=wl.cols,
+                                        out_dtype=wl.out_dtype)
     if wl.kind == "dequant_per_token":
         off = t.get("offset")
         return oracle.dequant_per_token(t["y"][r0:r1].numpy(), t["scale"][r0:r1],

@@ -1,7 +1,7 @@
 /*
  * dq.h — C ABI of the B200 (sm_100a) per-token dynamic quantization library.
  *
- * Three operations, launched asynchronously on the caller's stream:
+ * Four operations, launched asynchronously on the caller's stream:
  *
  *   dq_dynamic_quant        aclnnDynamicQuantV2, "Formula" and "Description":
  *                           per-row (per-token) symmetric or asymmetric
@@ -14,6 +14,9 @@
  *                           then symmetric INT8 dynamic quantization.
  *   dq_dequant_per_token    AntiQuantize, PER_TOKEN policy: codes back to
  *                           floats with one scale (and offset) per row.
+ *   dq_dequant_per_group    AntiQuantize, PER_GROUP policy: one scale (and
+ *                           offset) per group of elements along a row or
+ *                           down a column.
  *
  * plus the workspace queries of the two-phase calling convention both pages
  * describe ("...GetWorkspaceSize" first, then the run): dq_get_workspace_size
@@ -240,6 +243,26 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype,
  * DQ_ERR_CUDA. */
 dq_status dq_dequant_per_token(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols,
                                const void* scale, const void* offset, dq_dtype scale_dtype,
+                               void* out, dq_dtype out_dtype, cudaStream_t stream);
+
+/* Per-group dequantization (AntiQuantize, PER_GROUP policy): along the k
+ * axis every group_size elements share one scale and one offset.
+ *   k_dim = 1 (k runs along a row): scale/offset tables [rows, ceil(cols/g)];
+ *             element (i, j) uses entry (i, j / g).
+ *   k_dim = 0 (k runs down a column): tables [ceil(rows/g), cols]; element
+ *             (i, j) uses entry (i / g, j).
+ * group_size > 0 and a multiple of 32 (the page's constraint). The value is
+ * computed as in dq_dequant_per_token with the element's scale and offset;
+ * the page's formula images were lost, so that is a reading (the inverse of
+ * the quantizer). The page's int8 ("b8") source scenario is covered, with
+ * the int4 / INT32 containers accepted as well; its fp4 / fp8 / hifloat8
+ * scenarios are not (their formats are not defined on the pages).
+ * Arguments, alignment and errors as dq_dequant_per_token, plus
+ * DQ_ERR_BAD_ARGUMENT for a bad group_size or k_dim. With k_dim = 0, tables
+ * that are 16-byte aligned take the vectorised path. */
+dq_status dq_dequant_per_group(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols,
+                               const void* scale, const void* offset, dq_dtype scale_dtype,
+                               int64_t group_size, int32_t k_dim,
                                void* out, dq_dtype out_dtype, cudaStream_t stream);
 
 /* Largest batch * hidden that dq_ada_layernorm_quant_noalloc accepts (its

@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant_get_workspace_size",
-              "dq_ada_layernorm_quant", "dq_dequant_per_token", "dq_status_string"):
+              "dq_ada_layernorm_quant", "dq_dequant_per_token", "dq_dequant_per_group", "dq_status_string"):
         assert n in names
 
 
@@ -198,6 +198,24 @@ def test_dequant_per_token_validation(dq_lib):
     ]
     for kw, want in cases:
         assert _deq(d, **kw) == want, kw
+
+
+def test_dequant_per_group_validation(dq_lib):
+    d = dq_lib
+
+    def grp(**kw):
+        args = dict(y=FAKE, y_dtype=d.DQ_INT8, rows=64, cols=64, scale=FAKE, offset=None, scale_dtype=d.DQ_F32,
+                    group_size=32, k_dim=1, out=FAKE, out_dtype=d.DQ_BF16, stream=None)
+        args.update(kw)
+        return d.dq_dequant_per_group(**args)
+
+    assert grp(rows=0, y=None, out=None) == d.DQ_OK
+    for kw in (dict(group_size=0), dict(group_size=16), dict(group_size=48), dict(group_size=-32), dict(k_dim=2),
+               dict(k_dim=-1)):
+        assert grp(**kw) == d.DQ_ERR_BAD_ARGUMENT, kw
+    assert grp(y=None) == d.DQ_ERR_NULL_POINTER
+    assert grp(cols=0) == d.DQ_ERR_BAD_SHAPE
+    assert grp(scale=FAKE + 2) == d.DQ_ERR_MISALIGNED
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -1,4 +1,4 @@
-"""GPU parity of per-token dequantization (AntiQuantize, PER_TOKEN policy).
+"""GPU parity of dequantization (AntiQuantize, PER_TOKEN and PER_GROUP policies).
 
 dq_dequant_per_token through the C ABI against the CPU oracle, bit for bit:
 out = (code - offset) * scale in binary32, rounded once to the output type.
@@ -144,4 +144,84 @@ def test_dequant_workload_full_size(dq):
     got = got.cpu().view(torch.int16).numpy().view(np.uint16)
     rows = np.random.default_rng(0).choice(t["y"].shape[0], size=64, replace=False)
     want = oracle.dequant_per_token(t["y"][rows].numpy(), t["scale"][rows], out_dtype="bf16")
+    np.testing.assert_array_equal(got[rows], want)
+
+
+# ---------------------------------------------------------------- PER_GROUP
+
+def _group_tables(rows, cols, g, k_dim, dtype, seed, offset):
+    gen = torch.Generator().manual_seed(seed)
+    shape = (rows, -(-cols // g)) if k_dim == 1 else (-(-rows // g), cols)
+    scale = (torch.rand(shape, generator=gen) * 0.05 + 1e-3).to(dtype)
+    off = (torch.randn(shape, generator=gen) * 10).to(dtype) if offset else None
+    return scale, off
+
+
+def _group_gpu(dq, y, cols, y_dtype, scale, off, g, k_dim, out_dtype, misalign_table=False):
+    dev = torch.device("cuda:0")
+    sg = scale.to(dev)
+    if misalign_table:  # a table that is element-aligned but not 16-byte aligned
+        buf = torch.empty(scale.numel() + 1, dtype=scale.dtype, device=dev)
+        sg = buf[1:].view(scale.shape)
+        sg.copy_(scale.to(dev))
+    o = dq.dequant_per_group(y.to(dev), sg, None if off is None else off.to(dev), group_size=g, k_dim=k_dim,
+                             y_dtype=y_dtype, cols=cols, out_dtype=_TORCH_DT[out_dtype])
+    torch.cuda.synchronize()
+    o = o.cpu()
+    return o.view(torch.int16).numpy().view(np.uint16) if out_dtype != "f32" else o.numpy().view(np.uint32)
+
+
+def _group_oracle(y, cols, y_dtype, scale, off, g, k_dim, out_dtype):
+    out = oracle.dequant_per_group(y.numpy() if y_dtype != "int32" else y.numpy().view(np.uint32), scale, off,
+                                   group_size=g, k_dim=k_dim, y_dtype=y_dtype, cols=cols, out_dtype=out_dtype)
+    return out.view(np.uint16) if out_dtype in ("f16", "bf16") else out.view(np.uint32)
+
+
+GROUP_SHAPES = [(8, 256, 32), (33, 4096, 128), (70, 96, 64), (5, 1000, 32), (100, 512, 96)]
+
+
+@pytest.mark.parametrize("shape", GROUP_SHAPES, ids=[f"{r}x{c}g{g}" for r, c, g in GROUP_SHAPES])
+@pytest.mark.parametrize("k_dim", [1, 0])
+@pytest.mark.parametrize("y_dtype", ["int8", "int4"])
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("offset", [False, True])
+def test_dequant_per_group_matches_oracle(dq, shape, k_dim, y_dtype, out_dtype, offset):
+    rows, cols, g = shape
+    y = _codes(rows, cols, y_dtype, seed=rows + cols + g)
+    scale, off = _group_tables(rows, cols, g, k_dim, torch.float32, seed=g + k_dim, offset=offset)
+    want = _group_oracle(y, cols, y_dtype, scale, off, g, k_dim, out_dtype)
+    got = _group_gpu(dq, y, cols, y_dtype, scale, off, g, k_dim, out_dtype)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("sdt", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("k_dim", [1, 0])
+def test_dequant_per_group_half_tables(dq, sdt, k_dim):
+    y = _codes(40, 512, "int8", seed=13)
+    scale, off = _group_tables(40, 512, 32, k_dim, sdt, seed=14, offset=True)
+    want = _group_oracle(y, 512, "int8", scale, off, 32, k_dim, "f16")
+    got = _group_gpu(dq, y, 512, "int8", scale, off, 32, k_dim, "f16")
+    np.testing.assert_array_equal(got, want)
+
+
+def test_dequant_per_group_unaligned_column_table(dq):
+    y = _codes(64, 256, "int8", seed=15)
+    scale, _ = _group_tables(64, 256, 32, 0, torch.float32, seed=16, offset=False)
+    want = _group_oracle(y, 256, "int8", scale, None, 32, 0, "bf16")
+    got = _group_gpu(dq, y, 256, "int8", scale, None, 32, 0, "bf16", misalign_table=True)
+    np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.slow
+def test_dequant_per_group_workload_full_size(dq):
+    wl = workloads.make("dequant_per_group_int8_bf16_8192x4096_g128")
+    t = wl.tensors
+    dev = torch.device("cuda:0")
+    got = dq.dequant_per_group(t["y"].to(dev), t["scale"].to(dev), t["offset"].to(dev), group_size=wl.group_size,
+                               k_dim=wl.k_dim, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    got = got.cpu().view(torch.int16).numpy().view(np.uint16)
+    rows = np.random.default_rng(1).choice(t["y"].shape[0], size=64, replace=False)
+    want = oracle.dequant_per_group(t["y"][rows].numpy(), t["scale"][rows], t["offset"][rows],
+                                    group_size=wl.group_size, k_dim=wl.k_dim, out_dtype="bf16")
     np.testing.assert_array_equal(got[rows], want)

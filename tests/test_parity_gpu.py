@@ -299,7 +299,7 @@ def test_empty_input_is_a_noop(dq):
 
 # ---------------------------------------------------------------- full-size workloads
 
-DQ_WORKLOADS = [w for w in workloads.WORKLOADS if not w.startswith(("ada_", "dequant_"))]
+DQ_WORKLOADS = [w for w in workloads.WORKLOADS if not w.startswith(("ada_", "dequant"))]
 
 
 @pytest.mark.slow

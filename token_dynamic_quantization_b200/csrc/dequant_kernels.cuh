@@ -1,9 +1,11 @@
-// Per-token dequantization (AntiQuantize, PER_TOKEN policy), sm_100a.
+// Dequantization (AntiQuantize, PER_TOKEN and PER_GROUP policies), sm_100a.
 //
-// One scale and one optional offset per row of an [m, n] code matrix. The
-// page's formula images were lost; the operation is the inverse of the
-// aclnnDynamicQuantV2 quantizer (codes = round(x / scale + offset)):
-//   out[r,c] = (code[r,c] - offset[r]) * scale[r]
+// One scale and one optional offset per row of an [m, n] code matrix
+// (PER_TOKEN), or per group of groupSize elements along a row or down a
+// column (PER_GROUP). The page's formula images were lost; the operation is
+// the inverse of the aclnnDynamicQuantV2 quantizer (codes = round(x / scale +
+// offset)):
+//   out[i,j] = (code[i,j] - offset[e]) * scale[e]   (e: the element's table entry)
 // in binary32, one rounding per operation, then rounded to nearest even into
 // the output type.
 //
@@ -30,13 +32,20 @@ namespace dq {
 struct DequantArgs {
   const void* y;       // codes
   int64_t rows, cols;
-  const void* scale;   // [rows] of scale_dtype
-  const void* offset;  // [rows] of scale_dtype or nullptr
+  const void* scale;   // scale table of scale_dtype (layout below)
+  const void* offset;  // table of the same shape and dtype, or nullptr
   int scale_dtype;     // kF32 / kF16 / kBF16
   void* out;           // [rows, cols] of the output type
+  int64_t group_size;  // group layouts only
+  int64_t table_cols;  // row length of the scale table
 };
 
 enum : int { kOutF32 = 0, kOutF16 = 1, kOutBF16 = 2 };
+
+// Scale-table layouts (AntiQuantize policies): PER_TOKEN [rows]; PER_GROUP
+// with k along a row (kDim 1) [rows, ceil(cols/g)], entry (i, j / g); PER_GROUP
+// with k down a column (kDim 0) [ceil(rows/g), cols], entry (i / g, j).
+enum : int { kPerToken = 0, kGroupAlongRow = 1, kGroupDownColumn = 2 };
 
 // Output element storage and pair narrowing (round to nearest even).
 template <int OUT>
@@ -114,6 +123,48 @@ __device__ __forceinline__ void apply_row_constants(float (&v)[N], float scale, 
   }
 }
 
+// (v - offset[e]) * scale[e] with per-element tables.
+template <int N, bool kOff>
+__device__ __forceinline__ void apply_element_constants(float (&v)[N], const float (&scale)[N], const float (&off)[N]) {
+#pragma unroll
+  for (int p = 0; p < N / 2; ++p) {
+    float2 t = make_float2(v[2 * p], v[2 * p + 1]);
+    if (kOff) t = __fadd2_rn(t, make_float2(-off[2 * p], -off[2 * p + 1]));
+    t = __fmul2_rn(t, make_float2(scale[2 * p], scale[2 * p + 1]));
+    v[2 * p] = t.x;
+    v[2 * p + 1] = t.y;
+  }
+}
+
+// N consecutive table values from element `first` (16-byte aligned), widened.
+template <int N>
+__device__ __forceinline__ void load_table(const void* table, int dtype, int64_t first, float (&t)[N]) {
+  if (dtype == kF32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(table) + first);
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 f = __ldg(p + q);
+      t[4 * q] = f.x;
+      t[4 * q + 1] = f.y;
+      t[4 * q + 2] = f.z;
+      t[4 * q + 3] = f.w;
+    }
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(table) + first);
+#pragma unroll
+    for (int q = 0; q < N / 8; ++q) {
+      float h[8];
+      if (dtype == kF16) {
+        InTraits<__half>::widen8(__ldg(p + q), h);
+      } else {
+        InTraits<__nv_bfloat16>::widen8(__ldg(p + q), h);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) t[8 * q + e] = h[e];
+    }
+  }
+}
+
 template <int OUT, int N>
 __device__ __forceinline__ void store_vector(void* out_row, int vi, const float (&v)[N]) {
   if constexpr (OUT == kOutF32) {
@@ -142,8 +193,8 @@ constexpr int kDequantUnroll = 4;  // 16-byte code vectors in flight per lane
 // x kDequantUnroll vectors (2048 int8 or 4096 int4 codes). Items are many
 // and small, and the grid covers them all (a grid-stride loop only beyond
 // the grid limit), so the block scheduler balances the tail.
-template <int OUT, bool kFour, bool kOff>
-__global__ void __launch_bounds__(kDequantBlock) dequant_per_token_vec_kernel(const DequantArgs a) {
+template <int OUT, bool kFour, bool kOff, int LAYOUT>
+__global__ void __launch_bounds__(kDequantBlock) dequant_vec_kernel(const DequantArgs a) {
   constexpr int N = kFour ? 32 : 16;  // codes per 16-byte vector
   constexpr int kWarps = kDequantBlock / 32;
   pdl_launch_dependents();
@@ -158,8 +209,11 @@ __global__ void __launch_bounds__(kDequantBlock) dequant_per_token_vec_kernel(co
        item += static_cast<int64_t>(gridDim.x) * kWarps) {
     const int64_t r = item / chunks;
     const int v0 = static_cast<int>(item - r * chunks) * (32 * kDequantUnroll) + lane;
-    const float scale = load_param(a.scale, a.scale_dtype, r);
-    const float offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
+    float scale = 0.0f, offset = 0.0f;
+    if (LAYOUT == kPerToken) {
+      scale = load_param(a.scale, a.scale_dtype, r);
+      offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
+    }
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.y) + r * row_code_bytes);
     void* dst = static_cast<uint8_t*>(a.out) + r * row_out_bytes;
     uint4 w[kDequantUnroll];
@@ -174,7 +228,20 @@ __global__ void __launch_bounds__(kDequantBlock) dequant_per_token_vec_kernel(co
       if (vi < nvec) {
         float v[N];
         codes_of<kFour>(w[u], v);
-        apply_row_constants<N, kOff>(v, scale, offset);
+        if (LAYOUT == kPerToken) {
+          apply_row_constants<N, kOff>(v, scale, offset);
+        } else if (LAYOUT == kGroupAlongRow) {
+          // a vector lies inside one group (the group size is a multiple of 32)
+          const int64_t entry = r * a.table_cols + static_cast<int64_t>(vi) * N / a.group_size;
+          apply_row_constants<N, kOff>(v, load_param(a.scale, a.scale_dtype, entry),
+                                       kOff ? load_param(a.offset, a.scale_dtype, entry) : 0.0f);
+        } else {
+          const int64_t first = (r / a.group_size) * a.table_cols + static_cast<int64_t>(vi) * N;
+          float sc[N], of[N];
+          load_table<N>(a.scale, a.scale_dtype, first, sc);
+          if (kOff) load_table<N>(a.offset, a.scale_dtype, first, of);
+          apply_element_constants<N, kOff>(v, sc, of);
+        }
         store_vector<OUT, N>(dst, vi, v);
       }
     }
@@ -182,14 +249,17 @@ __global__ void __launch_bounds__(kDequantBlock) dequant_per_token_vec_kernel(co
 }
 
 // Any shape and alignment: one element per thread step, grid-strided rows.
-template <int OUT, bool kFour, bool kOff>
-__global__ void __launch_bounds__(kDequantBlock) dequant_per_token_generic_kernel(const DequantArgs a) {
+template <int OUT, bool kFour, bool kOff, int LAYOUT>
+__global__ void __launch_bounds__(kDequantBlock) dequant_generic_kernel(const DequantArgs a) {
   pdl_launch_dependents();
   pdl_wait_primary();
   for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
-    const float scale = load_param(a.scale, a.scale_dtype, r);
-    const float offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
     for (int64_t c = threadIdx.x; c < a.cols; c += kDequantBlock) {
+      const int64_t entry = LAYOUT == kPerToken        ? r
+                            : LAYOUT == kGroupAlongRow ? r * a.table_cols + c / a.group_size
+                                                       : (r / a.group_size) * a.table_cols + c;
+      const float scale = load_param(a.scale, a.scale_dtype, entry);
+      const float offset = kOff ? load_param(a.offset, a.scale_dtype, entry) : 0.0f;
       const int64_t i = r * a.cols + c;
       int code;
       if (kFour) {

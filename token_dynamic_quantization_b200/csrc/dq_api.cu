@@ -391,14 +391,12 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
 
 // ---------------------------------------------------------------- dequantization dispatch
 
-template <int OUT, bool kFour, bool kOff>
+template <int OUT, bool kFour, bool kOff, int LAYOUT>
 dq_status launch_dequant(const dq::DequantArgs& a, bool vec, cudaStream_t stream) {
-  const int device = current_device();
-  const int sms = sm_count(device);
   if (vec) {
     // one warp per row chunk, a grid that covers every chunk (capped: the
     // kernel loops beyond the cap)
-    void (*kfn)(const dq::DequantArgs) = dq::dequant_per_token_vec_kernel<OUT, kFour, kOff>;
+    void (*kfn)(const dq::DequantArgs) = dq::dequant_vec_kernel<OUT, kFour, kOff, LAYOUT>;
     const int64_t nvec = a.cols / (kFour ? 32 : 16);
     const int64_t chunks = (nvec + 32 * dq::kDequantUnroll - 1) / (32 * dq::kDequantUnroll);
     const int64_t warps_per_block = dq::kDequantBlock / 32;
@@ -406,11 +404,56 @@ dq_status launch_dequant(const dq::DequantArgs& a, bool vec, cudaStream_t stream
     if (grid > (int64_t(1) << 30)) grid = int64_t(1) << 30;
     return launch_programmatic(kfn, a, static_cast<int>(grid), dq::kDequantBlock, 0, stream);
   }
-  void (*gfn)(const dq::DequantArgs) = dq::dequant_per_token_generic_kernel<OUT, kFour, kOff>;
+  const int device = current_device();
+  const int sms = sm_count(device);
+  void (*gfn)(const dq::DequantArgs) = dq::dequant_generic_kernel<OUT, kFour, kOff, LAYOUT>;
   const int64_t resident =
       static_cast<int64_t>(sms) * blocks_per_sm(reinterpret_cast<const void*>(gfn), dq::kDequantBlock, 0, device);
   const int64_t g = a.rows < resident ? a.rows : resident;
   return launch_programmatic(gfn, a, static_cast<int>(g < 1 ? 1 : g), dq::kDequantBlock, 0, stream);
+}
+
+// Shared validation and dispatch of the two dequantization entry points.
+template <int LAYOUT>
+dq_status dequantize(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols, const void* scale,
+                     const void* offset, dq_dtype scale_dtype, int64_t group_size, int64_t table_cols, void* out,
+                     dq_dtype out_dtype, bool table_vec_ok, cudaStream_t stream) {
+  if (rows < 0 || cols < 1 || cols > (int64_t(1) << 31) || rows > (int64_t(1) << 40)) return DQ_ERR_BAD_SHAPE;
+  if (!is_code_type(y_dtype) || !is_param_float(scale_dtype) || !is_param_float(out_dtype)) return DQ_ERR_BAD_DTYPE;
+  if (y_dtype == DQ_INT4X2 && cols % 2 != 0) return DQ_ERR_BAD_SHAPE;
+  if (y_dtype == DQ_INT32 && cols % 8 != 0) return DQ_ERR_BAD_SHAPE;
+  if (rows == 0) return DQ_OK;
+  if (y == nullptr || scale == nullptr || out == nullptr) return DQ_ERR_NULL_POINTER;
+  const size_t ss = float_size(scale_dtype), os = float_size(out_dtype);
+  if (!aligned(scale, ss) || (offset && !aligned(offset, ss)) || !aligned(out, os) ||
+      (y_dtype == DQ_INT32 && !aligned(y, 4)))
+    return DQ_ERR_MISALIGNED;
+  dq::DequantArgs a{};
+  a.y = y;
+  a.rows = rows;
+  a.cols = cols;
+  a.scale = scale;
+  a.offset = offset;
+  a.scale_dtype = static_cast<int>(scale_dtype);
+  a.out = out;
+  a.group_size = group_size;
+  a.table_cols = table_cols;
+  const bool four = y_dtype != DQ_INT8;
+  const int out_kind = out_dtype == DQ_F32 ? dq::kOutF32 : (out_dtype == DQ_F16 ? dq::kOutF16 : dq::kOutBF16);
+  const bool has_offset = offset != nullptr;
+  const int64_t per_vec = four ? 32 : 16;
+  const bool vec = cols % per_vec == 0 && aligned(y, 16) && aligned(out, 16) && table_vec_ok;
+  switch (out_kind * 4 + (four ? 2 : 0) + (has_offset ? 1 : 0)) {
+#define DQ_DEQ_CASE(O, F, H)              \
+  case O * 4 + (F ? 2 : 0) + (H ? 1 : 0): \
+    return launch_dequant<O, F, H, LAYOUT>(a, vec, stream);
+    DQ_DEQ_CASE(0, false, false) DQ_DEQ_CASE(0, false, true) DQ_DEQ_CASE(0, true, false) DQ_DEQ_CASE(0, true, true)
+    DQ_DEQ_CASE(1, false, false) DQ_DEQ_CASE(1, false, true) DQ_DEQ_CASE(1, true, false) DQ_DEQ_CASE(1, true, true)
+    DQ_DEQ_CASE(2, false, false) DQ_DEQ_CASE(2, false, true) DQ_DEQ_CASE(2, true, false) DQ_DEQ_CASE(2, true, true)
+#undef DQ_DEQ_CASE
+    default:
+      return DQ_ERR_BAD_DTYPE;
+  }
 }
 
 dq_status check_ada(int64_t batch, int64_t seq, int64_t hidden, dq_dtype x_dtype, dq_dtype param_dtype) {
@@ -558,40 +601,23 @@ dq_status dq_ada_layernorm_quant(const void* x, dq_dtype x_dtype, int64_t batch,
 dq_status dq_dequant_per_token(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols, const void* scale,
                                const void* offset, dq_dtype scale_dtype, void* out, dq_dtype out_dtype,
                                cudaStream_t stream) {
-  if (rows < 0 || cols < 1 || cols > (int64_t(1) << 31) || rows > (int64_t(1) << 40)) return DQ_ERR_BAD_SHAPE;
-  if (!is_code_type(y_dtype) || !is_param_float(scale_dtype) || !is_param_float(out_dtype)) return DQ_ERR_BAD_DTYPE;
-  if (y_dtype == DQ_INT4X2 && cols % 2 != 0) return DQ_ERR_BAD_SHAPE;
-  if (y_dtype == DQ_INT32 && cols % 8 != 0) return DQ_ERR_BAD_SHAPE;
-  if (rows == 0) return DQ_OK;
-  if (y == nullptr || scale == nullptr || out == nullptr) return DQ_ERR_NULL_POINTER;
-  const size_t ss = float_size(scale_dtype), os = float_size(out_dtype);
-  if (!aligned(scale, ss) || (offset && !aligned(offset, ss)) || !aligned(out, os) ||
-      (y_dtype == DQ_INT32 && !aligned(y, 4)))
-    return DQ_ERR_MISALIGNED;
-  dq::DequantArgs a{};
-  a.y = y;
-  a.rows = rows;
-  a.cols = cols;
-  a.scale = scale;
-  a.offset = offset;
-  a.scale_dtype = static_cast<int>(scale_dtype);
-  a.out = out;
-  const bool four = y_dtype != DQ_INT8;
-  const int out_kind = out_dtype == DQ_F32 ? dq::kOutF32 : (out_dtype == DQ_F16 ? dq::kOutF16 : dq::kOutBF16);
-  const bool has_offset = offset != nullptr;
-  const int64_t per_vec = four ? 32 : 16;
-  const bool vec = cols % per_vec == 0 && aligned(y, 16) && aligned(out, 16);
-  switch (out_kind * 4 + (four ? 2 : 0) + (has_offset ? 1 : 0)) {
-#define DQ_DEQ_CASE(O, F, H)                                         \
-  case O * 4 + (F ? 2 : 0) + (H ? 1 : 0):                            \
-    return launch_dequant<O, F, H>(a, vec, stream);
-    DQ_DEQ_CASE(0, false, false) DQ_DEQ_CASE(0, false, true) DQ_DEQ_CASE(0, true, false) DQ_DEQ_CASE(0, true, true)
-    DQ_DEQ_CASE(1, false, false) DQ_DEQ_CASE(1, false, true) DQ_DEQ_CASE(1, true, false) DQ_DEQ_CASE(1, true, true)
-    DQ_DEQ_CASE(2, false, false) DQ_DEQ_CASE(2, false, true) DQ_DEQ_CASE(2, true, false) DQ_DEQ_CASE(2, true, true)
-#undef DQ_DEQ_CASE
-    default:
-      return DQ_ERR_BAD_DTYPE;
+  return dequantize<dq::kPerToken>(y, y_dtype, rows, cols, scale, offset, scale_dtype, 0, 1, out, out_dtype, true,
+                                   stream);
+}
+
+dq_status dq_dequant_per_group(const void* y, dq_dtype y_dtype, int64_t rows, int64_t cols, const void* scale,
+                               const void* offset, dq_dtype scale_dtype, int64_t group_size, int32_t k_dim,
+                               void* out, dq_dtype out_dtype, cudaStream_t stream) {
+  if (group_size <= 0 || group_size % 32 != 0 || (k_dim != 0 && k_dim != 1)) return DQ_ERR_BAD_ARGUMENT;
+  if (k_dim == 1) {
+    const int64_t groups = (cols + group_size - 1) / group_size;
+    return dequantize<dq::kGroupAlongRow>(y, y_dtype, rows, cols, scale, offset, scale_dtype, group_size, groups,
+                                          out, out_dtype, true, stream);
   }
+  // per-column tables are read as 16-byte vectors on the vectorised path
+  const bool table_vec_ok = aligned(scale, 16) && (offset == nullptr || aligned(offset, 16));
+  return dequantize<dq::kGroupDownColumn>(y, y_dtype, rows, cols, scale, offset, scale_dtype, group_size, cols, out,
+                                          out_dtype, table_vec_ok, stream);
 }
 
 }  // extern "C"

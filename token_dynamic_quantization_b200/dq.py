@@ -61,6 +61,8 @@ _lib.dq_ada_layernorm_quant.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _v
 _lib.dq_ada_layernorm_quant.restype = _ci
 _lib.dq_dequant_per_token.argtypes = [_vp, _ci, _i64, _i64, _vp, _vp, _ci, _vp, _ci, _vp]
 _lib.dq_dequant_per_token.restype = _ci
+_lib.dq_dequant_per_group.argtypes = [_vp, _ci, _i64, _i64, _vp, _vp, _ci, _i64, _i32, _vp, _ci, _vp]
+_lib.dq_dequant_per_group.restype = _ci
 _lib.dq_ada_layernorm_quant_noalloc.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp,
                                                 _vp, _vp]
 _lib.dq_ada_layernorm_quant_noalloc.restype = _ci
@@ -115,6 +117,13 @@ def dq_ada_layernorm_quant(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift,
 def dq_dequant_per_token(y, y_dtype, rows, cols, scale, offset, scale_dtype, out, out_dtype, stream) -> int:
     """Raw call: pointers are ints (0/None for NULL). Returns the dq_status."""
     return _lib.dq_dequant_per_token(y, y_dtype, rows, cols, scale, offset, scale_dtype, out, out_dtype, stream)
+
+
+def dq_dequant_per_group(y, y_dtype, rows, cols, scale, offset, scale_dtype, group_size, k_dim, out, out_dtype,
+                         stream) -> int:
+    """Raw call: pointers are ints (0/None for NULL). Returns the dq_status."""
+    return _lib.dq_dequant_per_group(y, y_dtype, rows, cols, scale, offset, scale_dtype, group_size, k_dim, out,
+                                     out_dtype, stream)
 
 
 def dq_ada_layernorm_quant_noalloc(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias, smooth,
@@ -261,6 +270,33 @@ def dequant_per_token(y, scale, offset=None, y_dtype: str = "int8", cols: int | 
         stream = torch.cuda.current_stream(y.device).cuda_stream
     st = dq_dequant_per_token(_dev_ptr(y, "y"), yc, rows, cols, _dev_ptr(scale, "scale"), _dev_ptr(offset, "offset"),
                               sdt, _dev_ptr(out, "out"), _dtype_code(out), stream)
+    if check and st != DQ_OK:
+        raise DQError(st)
+    return out
+
+
+def dequant_per_group(y, scale, offset=None, group_size: int = 32, k_dim: int = 1, y_dtype: str = "int8",
+                      cols: int | None = None, out_dtype=None, out=None, stream=None, check: bool = True):
+    """Per-group dequantization of CUDA codes ``y`` (AntiQuantize, PER_GROUP).
+
+    ``scale`` / ``offset``: CUDA tables [rows, ceil(cols/g)] (``k_dim`` 1) or
+    [ceil(rows/g), cols] (``k_dim`` 0) of one float dtype. Returns the
+    [rows, cols] output tensor (``out_dtype`` defaults to the scale's dtype).
+    """
+    torch = _torch()
+    yc = _YTYPES[y_dtype]
+    rows = int(y.shape[0]) if y.dim() else 0
+    if cols is None:
+        cols = int(y.shape[-1]) * {DQ_INT8: 1, DQ_INT4X2: 2, DQ_INT32: 8}[yc]
+    sdt = _dtype_code(scale)
+    if offset is not None and _dtype_code(offset) != sdt:
+        raise TypeError("offset must have the dtype of scale")
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype or scale.dtype, device=y.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(y.device).cuda_stream
+    st = dq_dequant_per_group(_dev_ptr(y, "y"), yc, rows, cols, _dev_ptr(scale, "scale"), _dev_ptr(offset, "offset"),
+                              sdt, int(group_size), int(k_dim), _dev_ptr(out, "out"), _dtype_code(out), stream)
     if check and st != DQ_OK:
         raise DQError(st)
     return out

@@ -30,6 +30,11 @@ LayerNorm path):
   policy; the inverse of the 8192 x 4096 quantization workload): codes int8
   [8192, 4096] uniform in [-127, 127] (seed 8), per-row scale fp32 [8192]
   ~ U(0.001, 0.05) (seed 9), no offset, bfloat16 output.
+* ``dequant_per_group_int8_bf16_8192x4096_g128`` (AntiQuantize page,
+  PER_GROUP policy, kDim 1): codes int8 [8192, 4096] uniform in [-127, 127]
+  (seed 8), groups of 128 along each row with fp32 scale [8192, 32]
+  ~ U(0.001, 0.05) (seed 9) and offset [8192, 32] ~ N(0, 8) (seed 10),
+  bfloat16 output.
 """
 
 from __future__ import annotations
@@ -84,17 +89,19 @@ class Workload:
     """One synthetic workload: named tensors on the CPU plus the call's options."""
 
     name: str
-    kind: str                    # "dynamic_quant" | "ada_layernorm_quant" | "dequant_per_token"
+    kind: str                    # "dynamic_quant" | "ada_layernorm_quant" | "dequant_per_token" | "dequant_per_group"
     tensors: dict = field(default_factory=dict)
     mode: str = "symmetric"      # dynamic_quant only
     y_dtype: str = "int8"        # code container (dynamic_quant output, dequant_per_token input)
     epsilon: float = 1e-6        # ada_layernorm_quant only
-    out_dtype: str = "bf16"      # dequant_per_token only
+    out_dtype: str = "bf16"      # dequantization only
+    group_size: int = 0          # dequant_per_group only
+    k_dim: int = 1               # dequant_per_group only
 
     @property
     def primary(self):
         """The per-row input: x, or the codes of a dequantization."""
-        return self.tensors["y"] if self.kind == "dequant_per_token" else self.tensors["x"]
+        return self.tensors["y"] if self.kind.startswith("dequant") else self.tensors["x"]
 
     @property
     def rows(self) -> int:
@@ -103,7 +110,7 @@ class Workload:
 
     @property
     def cols(self) -> int:
-        if self.kind == "dequant_per_token":
+        if self.kind.startswith("dequant"):
             return int(self.tensors["y"].shape[-1]) * {"int8": 1, "int4": 2, "int32": 8}[self.y_dtype]
         return int(self.tensors["x"].shape[-1])
 
@@ -115,6 +122,7 @@ WORKLOADS = (
     "asym_int4_f16_16384x8192",
     "ada_layernorm_quant_bf16_4x4096x3072",
     "dequant_per_token_int8_bf16_8192x4096",
+    "dequant_per_group_int8_bf16_8192x4096_g128",
 )
 
 
@@ -160,4 +168,12 @@ def make(name: str, rows: int | None = None) -> Workload:
         y = torch.randint(-127, 128, (r, 4096), generator=g, dtype=torch.int32).to(torch.int8)
         scale = uniform((r,), torch.float32, 9, 0.001, 0.05)
         return Workload(name, "dequant_per_token", {"y": y, "scale": scale}, y_dtype="int8", out_dtype="bf16")
+    if name == "dequant_per_group_int8_bf16_8192x4096_g128":
+        r = rows or 8192
+        g = _gen(8)
+        y = torch.randint(-127, 128, (r, 4096), generator=g, dtype=torch.int32).to(torch.int8)
+        scale = uniform((r, 32), torch.float32, 9, 0.001, 0.05)
+        offset = normal((r, 32), torch.float32, 10, std=8.0)
+        return Workload(name, "dequant_per_group", {"y": y, "scale": scale, "offset": offset}, y_dtype="int8",
+                        out_dtype="bf16", group_size=128, k_dim=1)
     raise KeyError(f"unknown workload {name!r}; known: {', '.join(WORKLOADS)}")
