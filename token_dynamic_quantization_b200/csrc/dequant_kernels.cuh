@@ -209,11 +209,6 @@ __global__ void __launch_bounds__(kDequantBlock) dequant_vec_kernel(const Dequan
        item += static_cast<int64_t>(gridDim.x) * kWarps) {
     const int64_t r = item / chunks;
     const int v0 = static_cast<int>(item - r * chunks) * (32 * kDequantUnroll) + lane;
-    float scale = 0.0f, offset = 0.0f;
-    if (LAYOUT == kPerToken) {
-      scale = load_param(a.scale, a.scale_dtype, r);
-      offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
-    }
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.y) + r * row_code_bytes);
     void* dst = static_cast<uint8_t*>(a.out) + r * row_out_bytes;
     uint4 w[kDequantUnroll];
@@ -221,6 +216,13 @@ __global__ void __launch_bounds__(kDequantBlock) dequant_vec_kernel(const Dequan
     for (int u = 0; u < kDequantUnroll; ++u) {
       const int vi = v0 + 32 * u;
       w[u] = vi < nvec ? __ldcs(src + vi) : make_uint4(0, 0, 0, 0);
+    }
+    // the row's constants after the code loads are in flight (measured:
+    // loading them first delays the stream)
+    float scale = 0.0f, offset = 0.0f;
+    if (LAYOUT == kPerToken) {
+      scale = load_param(a.scale, a.scale_dtype, r);
+      offset = kOff ? load_param(a.offset, a.scale_dtype, r) : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < kDequantUnroll; ++u) {
