@@ -11,8 +11,7 @@
 //
 // The work is 1 (int8) or 0.5 (int4) byte in and 2 or 4 bytes out per element,
 // so the kernel is HBM-bound. A warp takes one chunk of a row at a time; each
-// lane streams 16-byte vectors of codes (16 int8 or 32 int4 codes), four loads
-// in flight.
+// lane streams 16-byte vectors of codes (16 int8 or 32 int4 codes).
 // A code becomes a float without the conversion unit: XOR with the sign bit
 // makes it an unsigned byte u = code + 128 (u = code + 8 for nibbles), a byte
 // permute places u in the low byte of the pattern of 1.5 * 2^23, and one
@@ -186,17 +185,30 @@ __device__ __forceinline__ void store_vector(void* out_row, int vi, const float 
 }
 
 constexpr int kDequantBlock = 256;
-constexpr int kDequantUnroll = 4;  // 16-byte code vectors in flight per lane
+// 16-byte code vectors per lane and work item, per scale layout (measured:
+// per-token rows stream best with one vector per lane and item, grouped
+// tables with two, which amortize the table lookups).
+#ifndef DQ_DEQUANT_UNROLL_TOKEN
+#define DQ_DEQUANT_UNROLL_TOKEN 1
+#endif
+#ifndef DQ_DEQUANT_UNROLL_GROUP
+#define DQ_DEQUANT_UNROLL_GROUP 2
+#endif
+template <int LAYOUT>
+__host__ __device__ constexpr int dequant_unroll() {
+  return LAYOUT == kPerToken ? DQ_DEQUANT_UNROLL_TOKEN : DQ_DEQUANT_UNROLL_GROUP;
+}
 
 // Rows whose code bytes are a whole number of 16-byte vectors, 16-byte
 // aligned codes and output rows. A work item is one chunk of a row: 32 lanes
-// x kDequantUnroll vectors (2048 int8 or 4096 int4 codes). Items are many
+// x dequant_unroll vectors (512 or 1024 int8 codes). Items are many
 // and small, and the grid covers them all (a grid-stride loop only beyond
 // the grid limit), so the block scheduler balances the tail.
 template <int OUT, bool kFour, bool kOff, int LAYOUT>
 __global__ void __launch_bounds__(kDequantBlock) dequant_vec_kernel(const DequantArgs a) {
   constexpr int N = kFour ? 32 : 16;  // codes per 16-byte vector
   constexpr int kWarps = kDequantBlock / 32;
+  constexpr int kDequantUnroll = dequant_unroll<LAYOUT>();
   pdl_launch_dependents();
   pdl_wait_primary();  // launched as a programmatic dependent: inputs are visible from here on
   const int lane = threadIdx.x & 31;

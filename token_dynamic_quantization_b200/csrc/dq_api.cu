@@ -398,7 +398,8 @@ dq_status launch_dequant(const dq::DequantArgs& a, bool vec, cudaStream_t stream
     // kernel loops beyond the cap)
     void (*kfn)(const dq::DequantArgs) = dq::dequant_vec_kernel<OUT, kFour, kOff, LAYOUT>;
     const int64_t nvec = a.cols / (kFour ? 32 : 16);
-    const int64_t chunks = (nvec + 32 * dq::kDequantUnroll - 1) / (32 * dq::kDequantUnroll);
+    constexpr int kUnroll = dq::dequant_unroll<LAYOUT>();
+    const int64_t chunks = (nvec + 32 * kUnroll - 1) / (32 * kUnroll);
     const int64_t warps_per_block = dq::kDequantBlock / 32;
     int64_t grid = (a.rows * chunks + warps_per_block - 1) / warps_per_block;
     if (grid > (int64_t(1) << 30)) grid = int64_t(1) << 30;
