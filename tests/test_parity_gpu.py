@@ -81,6 +81,7 @@ def rows_mix(rows, cols, dtype, seed):
 
 
 SHAPES = [(1, 8), (3, 16), (5, 24), (37, 1000), (64, 1024), (130, 4096), (17, 7168), (5, 8192), (9, 16384),
+          (11, 3072), (7, 1792), (6, 3584), (4, 5376),
           (3, 16392), (2, 32768), (7, 40), (6, 2), (11, 520), (300, 64)]
 
 

@@ -173,7 +173,7 @@ dq_status launch_programmatic(void (*kernel)(const Args), const Args& a, int gri
 GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
   GroupShape best{0, 0};
   double best_eff = -1.0;
-  static const int kVpts[3] = {2, 4, 8};
+  static const int kVpts[5] = {2, 4, 6, 7, 8};
   for (int vpt : kVpts) {
     const int64_t warps = (nvec + 32 * vpt - 1) / (32 * vpt);
     if (warps > 16) continue;
@@ -220,6 +220,8 @@ dq_status launch_dq_vpt(dq::RowQuantArgs a, int vpt, int device, int sms, cudaSt
   switch (vpt) {
     case 2: return launch_dq_ragged<InT, MODE, OUT, SMK, 2>(a, device, sms, stream);
     case 4: return launch_dq_ragged<InT, MODE, OUT, SMK, 4>(a, device, sms, stream);
+    case 6: return launch_dq_ragged<InT, MODE, OUT, SMK, 6>(a, device, sms, stream);
+    case 7: return launch_dq_ragged<InT, MODE, OUT, SMK, 7>(a, device, sms, stream);
     default: return launch_dq_ragged<InT, MODE, OUT, SMK, 8>(a, device, sms, stream);
   }
 }
