@@ -4,8 +4,9 @@ A plain, single-threaded C++ implementation (``dq_oracle.cpp``) of the
 formulas on the aclnnDynamicQuantV2 page ("Formula": symmetric and
 asymmetric quantization, with and without smooth scales; MoE smooth-scale
 selection from "Description") and the aclnnAdaLayerNormQuant page
-("Formula", steps 1-5), plus the PER_TOKEN and PER_GROUP dequantizers of the
-AntiQuantize page, wrapped here with ctypes + numpy.
+("Formula", steps 1-5), the PER_TOKEN and PER_GROUP dequantizers of the
+AntiQuantize page and the per-token x per-channel scaled W8A8 product of the
+aclnnQuantBatchMatmulInplaceAdd page, wrapped here with ctypes + numpy.
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
 leg may import this package. It shares nothing with the CUDA library: no
@@ -80,6 +81,8 @@ def _load():
             lib.oracle_dequant_per_token.restype = ci
             lib.oracle_dequant_per_group.argtypes = [vp, ci, i64, i64, vp, vp, ci, i64, ci, ci, vp]
             lib.oracle_dequant_per_group.restype = ci
+            lib.oracle_w8a8_gemm.argtypes = [vp, vp, i64, i64, i64, vp, vp, ci, ci, vp]
+            lib.oracle_w8a8_gemm.restype = ci
             lib.oracle_float_to_half_bits.argtypes = [f32]
             lib.oracle_float_to_half_bits.restype = ctypes.c_uint16
             lib.oracle_float_to_bfloat16_bits.argtypes = [f32]
@@ -258,6 +261,31 @@ def dequant_per_group(codes, scale, offset=None, group_size: int = 32, k_dim: in
     _check(lib.oracle_dequant_per_group(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, int(group_size),
                                         int(k_dim), oc_out, _ptr(out)))
     return out.view(np.float16) if oc_out == F16 else out
+
+
+def w8a8_gemm(a, b, a_scale, b_scale, out_dtype: str = "f32", accumulate_into=None):
+    """out[m, n] = float(sum_k a[m,k] b[n,k]) * (a_scale[m] * b_scale[n])
+    (+ accumulate_into[m, n]), binary32, rounded once per operation in that
+    order, then narrowed to ``out_dtype``. a: int8 [M, K]; b: int8 [N, K]."""
+    lib = _load()
+    ab = np.ascontiguousarray(a, dtype=np.int8)
+    bb = np.ascontiguousarray(b, dtype=np.int8)
+    m, k = ab.shape
+    n = bb.shape[0]
+    if bb.shape[1] != k:
+        raise ValueError("oracle.w8a8_gemm: K mismatch")
+    sa = np.ascontiguousarray(a_scale, dtype=np.float32)
+    sb = np.ascontiguousarray(b_scale, dtype=np.float32)
+    oc = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
+    if accumulate_into is not None:
+        if oc != F32:
+            raise ValueError("accumulation needs float32 output")
+        out = np.array(accumulate_into, dtype=np.float32, copy=True)
+    else:
+        out = np.zeros((m, n), dtype=np.float32 if oc == F32 else np.uint16)
+    _check(lib.oracle_w8a8_gemm(_ptr(ab), _ptr(bb), m, n, k, _ptr(sa), _ptr(sb), oc,
+                                1 if accumulate_into is not None else 0, _ptr(out)))
+    return out.view(np.float16) if oc == F16 else out
 
 
 def float_to_half_bits(v: float) -> int:

@@ -56,6 +56,12 @@
 //     offset of a [rows, ceil(cols/g)] or [ceil(rows/g), cols] table (the
 //     page's shapes); the value is the PER_TOKEN reading with that element's
 //     scale and offset (the page's formula images were lost here too);
+//   * aclnnQuantBatchMatmulInplaceAdd, "计算公式" (T-T form): the quantized
+//     product sum_k x1[m,k] x2[k,n] times (scale1 * scale2), plus y; read
+//     with scale1 per row (per token, as the quantizer produces it) and
+//     scale2 per output column (per channel), the product of the two scales
+//     taken first as printed, then the multiply, then the optional add, each
+//     rounded once in binary32 (the integer sum is exact);
 //   * AdaLayerNormQuant: the mean and the biased variance (divide by H) are
 //     accumulated in double over the fp32-widened row and rounded to float
 //     once; epsilon is added inside the square root; x - E(x) is divided by
@@ -458,6 +464,34 @@ int oracle_dequant_per_group(const void* y, int y_dtype, int64_t rows, int64_t c
         static_cast<uint16_t*>(out)[e] = narrow_to_half(v);
       } else {
         static_cast<uint16_t*>(out)[e] = narrow_to_bfloat16(v);
+      }
+    }
+  }
+  return ORACLE_OK;
+}
+
+int oracle_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
+                     const float* a_scale, const float* b_scale, int out_dtype, int accumulate, void* out) {
+  if (m < 0 || n < 0 || k < 1) return ORACLE_ERR_SHAPE;
+  if (k > (int64_t(1) << 17)) return ORACLE_ERR_SHAPE;  // |acc| < 2^31 for any int8 codes
+  if (!is_float_dtype(out_dtype)) return ORACLE_ERR_DTYPE;
+  if (accumulate && out_dtype != ORACLE_F32) return ORACLE_ERR_ARGUMENT;
+  if (m > 0 && n > 0 && (a == nullptr || b == nullptr || a_scale == nullptr || b_scale == nullptr || out == nullptr))
+    return ORACLE_ERR_ARGUMENT;
+  for (int64_t i = 0; i < m; ++i) {
+    for (int64_t j = 0; j < n; ++j) {
+      int64_t acc = 0;
+      for (int64_t kk = 0; kk < k; ++kk) acc += static_cast<int64_t>(a[i * k + kk]) * static_cast<int64_t>(b[j * k + kk]);
+      const float scales = a_scale[i] * b_scale[j];
+      float t = static_cast<float>(static_cast<int32_t>(acc)) * scales;
+      const int64_t e = i * n + j;
+      if (out_dtype == ORACLE_F32) {
+        float* o = static_cast<float*>(out);
+        o[e] = accumulate ? t + o[e] : t;
+      } else if (out_dtype == ORACLE_F16) {
+        static_cast<uint16_t*>(out)[e] = narrow_to_half(t);
+      } else {
+        static_cast<uint16_t*>(out)[e] = narrow_to_bfloat16(t);
       }
     }
   }

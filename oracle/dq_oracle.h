@@ -75,6 +75,21 @@ int oracle_dequant_per_group(const void* y, int y_dtype, int64_t rows, int64_t c
                              const void* scale, const void* offset, int scale_dtype,
                              int64_t group_size, int k_dim, int out_dtype, void* out);
 
+/* W8A8 GEMM with per-token x per-channel scales (the quantized matrix
+ * product that consumes the codes; aclnnQuantBatchMatmulInplaceAdd,
+ * "计算公式", T-T form, with scale1 per row of x1 and scale2 per column of
+ * the product):
+ *   acc[m,n] = sum_k a[m,k] * b[n,k]            (exact integer)
+ *   t        = float(acc[m,n]) * (a_scale[m] * b_scale[n])   (binary32: the
+ *              int32 -> float conversion, the scale product and the multiply
+ *              are each rounded once, in the formula's order)
+ *   out[m,n] = accumulate ? t + out[m,n] : t     (then narrowed to out_dtype)
+ * a: int8 [M, K]; b: int8 [N, K] (each output column's weights contiguous);
+ * a_scale [M], b_scale [N] float; out [M, N] of out_dtype (accumulate only
+ * with ORACLE_F32). */
+int oracle_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
+                     const float* a_scale, const float* b_scale, int out_dtype, int accumulate, void* out);
+
 /* binary32 -> binary16 / bfloat16 bit patterns, round to nearest even (the
  * narrowing the dequantizer ends with; exported for its pins). */
 uint16_t oracle_float_to_half_bits(float f);

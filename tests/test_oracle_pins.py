@@ -680,3 +680,73 @@ def test_per_group_argument_errors(oracle_mod):
         args.update(kw)
         with pytest.raises(oracle_mod.OracleError):
             oracle_mod.dequant_per_group(codes, scale, offset, **args)
+
+
+# ---------------------------------------------------------------- W8A8 product (aclnnQuantBatchMatmulInplaceAdd)
+
+def _int8(rng, shape):
+    return rng.integers(-128, 128, size=shape).astype(np.int8)
+
+
+def test_w8a8_unit_scales_are_the_integer_product(oracle_mod):
+    """With scales 1 the value is the exact integer sum (below 2^24 it is
+    exact in binary32), checked against numpy's int64 matmul."""
+    rng = np.random.default_rng(21)
+    a, b = _int8(rng, (40, 512)), _int8(rng, (24, 512))
+    got = oracle_mod.w8a8_gemm(a, b, np.ones(40), np.ones(24))
+    want = a.astype(np.int64) @ b.astype(np.int64).T
+    assert np.abs(want).max() < 2 ** 24
+    np.testing.assert_array_equal(got.astype(np.int64), want)
+
+
+def test_w8a8_power_of_two_scales_are_exact(oracle_mod):
+    rng = np.random.default_rng(22)
+    a, b = _int8(rng, (16, 256)), _int8(rng, (12, 256))
+    ka, kb = rng.integers(-10, 10, 16), rng.integers(-10, 10, 12)
+    got = oracle_mod.w8a8_gemm(a, b, np.ldexp(1.0, ka), np.ldexp(1.0, kb))
+    want = (a.astype(np.int64) @ b.astype(np.int64).T) * np.ldexp(1.0, ka[:, None] + kb[None, :])
+    np.testing.assert_array_equal(got.astype(np.float64), want)
+
+
+def test_w8a8_operand_roles_transpose(oracle_mod):
+    """Swapping the operands (and their scales) transposes the product: catches
+    an index mix-up between a[m,k] and b[n,k]."""
+    rng = np.random.default_rng(23)
+    a, b = _int8(rng, (9, 96)), _int8(rng, (13, 96))
+    sa, sb = rng.uniform(0.01, 2, 9).astype(np.float32), rng.uniform(0.01, 2, 13).astype(np.float32)
+    x = oracle_mod.w8a8_gemm(a, b, sa, sb)
+    y = oracle_mod.w8a8_gemm(b, a, sb, sa)
+    np.testing.assert_array_equal(x, y.T)
+
+
+def test_w8a8_scale_product_is_taken_first(oracle_mod):
+    """The formula multiplies the sum by (scale1 * scale2): rounded products in
+    that order. Cases where (acc * s1) * s2 would round differently pin it."""
+    rng = np.random.default_rng(24)
+    found = 0
+    for _ in range(200):
+        a = _int8(rng, (1, 64))
+        b = _int8(rng, (1, 64))
+        s1 = np.float32(rng.uniform(0.001, 1))
+        s2 = np.float32(rng.uniform(0.001, 1))
+        acc = np.float32(int((a.astype(np.int64) @ b.astype(np.int64).T)[0, 0]))
+        page = np.float32(acc * np.float32(s1 * s2))
+        other = np.float32(np.float32(acc * s1) * s2)
+        if page == other:
+            continue
+        found += 1
+        got = oracle_mod.w8a8_gemm(a, b, np.array([s1]), np.array([s2]))[0, 0]
+        assert got == page and got != other
+    assert found >= 10
+
+
+def test_w8a8_accumulate_and_narrow(oracle_mod):
+    rng = np.random.default_rng(25)
+    a, b = _int8(rng, (8, 128)), _int8(rng, (8, 128))
+    sa, sb = rng.uniform(0.01, 0.1, 8).astype(np.float32), rng.uniform(0.01, 0.1, 8).astype(np.float32)
+    base = oracle_mod.w8a8_gemm(a, b, sa, sb)  # |values| well inside the binary16 range
+    y = rng.standard_normal((8, 8)).astype(np.float32)
+    np.testing.assert_array_equal(oracle_mod.w8a8_gemm(a, b, sa, sb, accumulate_into=y), (base + y).astype(np.float32))
+    np.testing.assert_array_equal(oracle_mod.w8a8_gemm(a, b, sa, sb, out_dtype="f16"), base.astype(np.float16))
+    bf = oracle_mod.w8a8_gemm(a, b, sa, sb, out_dtype="bf16")
+    np.testing.assert_array_equal(bf, torch.from_numpy(base).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
