@@ -1,7 +1,7 @@
 /*
  * dq.h — C ABI of the B200 (sm_100a) per-token dynamic quantization library.
  *
- * Four operations, launched asynchronously on the caller's stream:
+ * Five operations, launched asynchronously on the caller's stream:
  *
  *   dq_dynamic_quant        aclnnDynamicQuantV2, "Formula" and "Description":
  *                           per-row (per-token) symmetric or asymmetric
@@ -17,6 +17,9 @@
  *   dq_dequant_per_group    AntiQuantize, PER_GROUP policy: one scale (and
  *                           offset) per group of elements along a row or
  *                           down a column.
+ *   dq_w8a8_gemm            aclnnQuantBatchMatmulInplaceAdd: the consumer of
+ *                           the codes, a W8A8 product with per-token x
+ *                           per-channel scales on the tensor cores.
  *
  * plus the workspace queries of the two-phase calling convention both pages
  * describe ("...GetWorkspaceSize" first, then the run): dq_get_workspace_size
@@ -264,6 +267,29 @@ dq_status dq_dequant_per_group(const void* y, dq_dtype y_dtype, int64_t rows, in
                                const void* scale, const void* offset, dq_dtype scale_dtype,
                                int64_t group_size, int32_t k_dim,
                                void* out, dq_dtype out_dtype, cudaStream_t stream);
+
+/* W8A8 product with per-token x per-channel scales, on the tensor cores
+ * (aclnnQuantBatchMatmulInplaceAdd, "计算公式", T-T form: the quantized
+ * product times (scale1 * scale2), plus y), with scale1 per row of a (per
+ * token, as dq_dynamic_quant produces it) and scale2 per output column:
+ *   acc[m,n] = sum_k a[m,k] * b[n,k]                     (exact int32)
+ *   out[m,n] = float(acc) * (a_scale[m] * b_scale[n])  (+ out[m,n] when
+ *              accumulate), each binary32 operation rounded once in that
+ *              order, then narrowed to out_dtype (round to nearest even).
+ * Arguments
+ *   a        device int8 [m, k] (the quantized activations, rows contiguous).
+ *   b        device int8 [n, k] (each output column's weights contiguous).
+ *   a_scale  device float [m]; b_scale device float [n].
+ *   out      device [m, n] of out_dtype (DQ_F32, DQ_F16, DQ_BF16);
+ *            accumulate = 1 adds into it (DQ_F32 only), 0 overwrites.
+ * k <= 2^17 (int32 sums cannot overflow). m, n, k multiples of 128 with
+ * 16-byte aligned a and b run on tcgen05 tensor cores (128 x 128 tiles);
+ * other shapes run a CUDA-core kernel with the same results.
+ * Errors: DQ_ERR_BAD_SHAPE, DQ_ERR_BAD_DTYPE, DQ_ERR_BAD_ARGUMENT,
+ * DQ_ERR_NULL_POINTER, DQ_ERR_MISALIGNED, DQ_ERR_CUDA. */
+dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
+                       const float* a_scale, const float* b_scale, void* out, dq_dtype out_dtype,
+                       int32_t accumulate, cudaStream_t stream);
 
 /* Largest batch * hidden that dq_ada_layernorm_quant_noalloc accepts (its
  * fixed table holds this many 8-byte entries: 1 MiB per device). */

@@ -1,0 +1,334 @@
+// W8A8 product with per-token x per-channel scales on the sm_100a tensor
+// cores (tcgen05), the consumer of the quantizer's codes.
+//
+// aclnnQuantBatchMatmulInplaceAdd, "计算公式" (T-T form): the quantized product
+// sum_k x1[m,k] * x2[k,n] is multiplied by (scale1 * scale2) and added to y.
+// Here scale1 is per row of x1 (per token, as dq_dynamic_quant produces it)
+// and scale2 per output column (per channel of the weights):
+//   acc[m,n] = sum_k a[m,k] * b[n,k]                      (exact, int32)
+//   out[m,n] = float(acc) * (a_scale[m] * b_scale[n])  (+ out[m,n])
+// each binary32 operation rounded once in that order, then narrowed.
+//
+// Tensor-core path (M, N, K multiples of 128; 16-byte aligned operands): one
+// CTA per 128 x 128 output tile, 6 warps.
+//   warp 0      TMA producer: 128-row x 128-byte K tiles of A and B (K-major,
+//               128-byte swizzle) into a 4-stage shared-memory ring.
+//   warp 1      allocates 128 TMEM columns (the int32 accumulator, row m in
+//               lane m); one lane issues tcgen05.mma.kind::i8 (M=128, N=128,
+//               K=32, four per stage) and releases each stage with
+//               tcgen05.commit, then commits the accumulator.
+//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, 32 columns at
+//               a time, scales, optional accumulation, narrowing, stores.
+// Every mbarrier wait is bounded; the MMA lane always issues the final
+// commit, so teardown never frees TMEM under MMAs in flight.
+// Other shapes or alignments: a CUDA-core kernel with the same arithmetic.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "dq.h"
+#include "tma_pipeline.cuh"
+
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kBK = 128;  // tile; kBK bytes = one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr uint32_t kTileBytes = kBM * kBK;  // 16 KB for A and for B (kBM == kBN)
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 128;
+constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + 256;  // alignment slack + ring + barriers
+
+struct W8A8Args {
+  const int8_t* a;
+  const int8_t* b;
+  const float* a_scale;
+  const float* b_scale;
+  void* out;
+  int64_t m, n, k;
+  int out_kind;    // 0 f32, 1 f16, 2 bf16
+  int accumulate;  // out (f32) += product
+};
+
+__device__ __forceinline__ void store_out(const W8A8Args& a, int64_t e, float t) {
+  if (a.out_kind == 0) {
+    float* o = static_cast<float*>(a.out);
+    o[e] = a.accumulate ? __fadd_rn(t, o[e]) : t;
+  } else if (a.out_kind == 1) {
+    static_cast<__half*>(a.out)[e] = __float2half_rn(t);
+  } else {
+    static_cast<__nv_bfloat16*>(a.out)[e] = __float2bfloat16_rn(t);
+  }
+}
+
+// ---------------------------------------------------------------- tcgen05 helpers
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major tile in the 128-byte swizzle
+// layout: rows of 128 bytes, groups of 8 rows 1024 bytes apart (stride byte
+// offset 1024; the leading byte offset is 1 for swizzled K-major tiles),
+// descriptor version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc_k_sw128(const void* tile) {
+  const uint64_t start = (dq::smem_addr(tile) >> 4) & 0x3FFFu;
+  return start | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Instruction descriptor of kind::i8: int32 accumulator (format 2), signed A
+// and B (format 1), both K-major, N / 8 and M / 16.
+constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(dq::smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dq::smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(dq::smem_addr(bar))
+      : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tc_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- kernels
+
+__global__ void __launch_bounds__(kThreads, 1)
+w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const W8A8Args a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + kStages * kTileBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kStages * kTileBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_ready = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
+  const int ktiles = static_cast<int>(a.k / kBK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      dq::mbar_init(full + s, 1);
+      dq::mbar_init(empty + s, 1);
+    }
+    dq::mbar_init(acc_ready, 1);
+    dq::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dq::smem_addr(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // launched as a programmatic dependent: the codes may come from the
+  // previous kernel, so no global memory is read before this
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == 0) {
+    if (lane == 0) {  // producer
+      for (int kt = 0; kt < ktiles; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
+        if (!dq::mbar_wait_parity(empty + s, ph ^ 1u)) break;
+        dq::mbar_arrive_expect_tx(full + s, 2 * kTileBytes);
+        tma_load_2d(sa + s * kTileBytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
+        tma_load_2d(sb + s * kTileBytes, &map_b, kt * kBK, static_cast<int>(n0), full + s);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      for (int kt = 0; kt < ktiles; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
+        if (!dq::mbar_wait_parity(full + s, ph)) break;
+        tc_fence_after();
+        const uint64_t ad = smem_desc_k_sw128(sa + s * kTileBytes);
+        const uint64_t bd = smem_desc_k_sw128(sb + s * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 32; ++kk) {
+          // +32 bytes along K = +2 in the descriptor's 16-byte address units
+          tc_mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, (kt | kk) != 0 ? 1u : 0u);
+        }
+        tc_commit(empty + s);  // the stage is free once these MMAs have read it
+      }
+      tc_commit(acc_ready);  // every MMA issued above is complete when this arrives
+    }
+  } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
+    const bool ready = dq::mbar_wait_parity(acc_ready, 0);
+    tc_fence_after();
+    const int quarter = warp & 3;
+    const int64_t row = m0 + 32 * quarter + lane;
+    const float sa_row = a.a_scale[row];
+#pragma unroll 1
+    for (int c = 0; c < kBN / 32; ++c) {
+      uint32_t r[32];
+      tc_ld_32cols(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * c), r);
+      if (!ready) continue;
+      const int64_t col0 = n0 + 32 * c;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float scales = __fmul_rn(sa_row, a.b_scale[col0 + j]);
+        const float t = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
+        store_out(a, row * a.n + col0 + j, t);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// Any shape: one output per thread, integer dot product on CUDA cores.
+__global__ void __launch_bounds__(256) w8a8_gemm_generic_kernel(const W8A8Args a) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int64_t total = a.m * a.n;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / a.n, j = e - (e / a.n) * a.n;
+    const int8_t* ar = a.a + i * a.k;
+    const int8_t* br = a.b + j * a.k;
+    int acc = 0;
+    for (int64_t kk = 0; kk < a.k; ++kk) acc += static_cast<int>(ar[kk]) * static_cast<int>(br[kk]);
+    const float scales = __fmul_rn(a.a_scale[i], a.b_scale[j]);
+    store_out(a, e, __fmul_rn(__int2float_rn(acc), scales));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// [rows, k] int8, k contiguous: 128-byte x 128-row boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};  // bytes between rows
+  const cuuint32_t box[2] = {kBK, kBM};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned_to(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; }
+
+template <typename Kernel, typename... Args>
+dq_status launch_pdl(Kernel kernel, dim3 grid, int block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+    cudaGetLastError();
+    return DQ_ERR_CUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
+                                  const float* a_scale, const float* b_scale, void* out, dq_dtype out_dtype,
+                                  int32_t accumulate, cudaStream_t stream) {
+  if (m < 0 || n < 0 || k < 1 || k > (int64_t(1) << 17) || m > (int64_t(1) << 31) || n > (int64_t(1) << 31))
+    return DQ_ERR_BAD_SHAPE;
+  if (out_dtype != DQ_F32 && out_dtype != DQ_F16 && out_dtype != DQ_BF16) return DQ_ERR_BAD_DTYPE;
+  if (accumulate != 0 && accumulate != 1) return DQ_ERR_BAD_ARGUMENT;
+  if (accumulate && out_dtype != DQ_F32) return DQ_ERR_BAD_ARGUMENT;
+  if (m == 0 || n == 0) return DQ_OK;
+  if (a == nullptr || b == nullptr || a_scale == nullptr || b_scale == nullptr || out == nullptr)
+    return DQ_ERR_NULL_POINTER;
+  const size_t os = out_dtype == DQ_F32 ? 4 : 2;
+  if (!aligned_to(a_scale, 4) || !aligned_to(b_scale, 4) || !aligned_to(out, os)) return DQ_ERR_MISALIGNED;
+  W8A8Args args{a, b, a_scale, b_scale, out, m, n, k, out_dtype == DQ_F32 ? 0 : (out_dtype == DQ_F16 ? 1 : 2),
+                accumulate};
+  const bool tiles = m % kBM == 0 && n % kBN == 0 && k % kBK == 0 && m / kBM <= 65535 &&
+                     aligned_to(a, 16) && aligned_to(b, 16);
+  if (tiles) {
+    CUtensorMap ma, mb;
+    if (make_map(&ma, a, m, k) && make_map(&mb, b, n, k)) {
+      static std::once_flag smem_once;
+      static bool smem_ok = false;
+      std::call_once(smem_once, [] {
+        smem_ok = cudaFuncSetAttribute(w8a8_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes)) == cudaSuccess;
+        if (!smem_ok) cudaGetLastError();
+      });
+      if (smem_ok) {
+        return launch_pdl(w8a8_gemm_tc_kernel, dim3(static_cast<unsigned>(n / kBN), static_cast<unsigned>(m / kBM)),
+                          kThreads, kSmemBytes, stream, ma, mb, args);
+      }
+    }
+  }
+  const int64_t total = m * n;
+  int64_t grid = (total + 255) / 256;
+  if (grid > 148 * 64) grid = 148 * 64;
+  return launch_pdl(w8a8_gemm_generic_kernel, dim3(static_cast<unsigned>(grid)), 256, 0, stream, args);
+}

@@ -63,6 +63,8 @@ _lib.dq_dequant_per_token.argtypes = [_vp, _ci, _i64, _i64, _vp, _vp, _ci, _vp, 
 _lib.dq_dequant_per_token.restype = _ci
 _lib.dq_dequant_per_group.argtypes = [_vp, _ci, _i64, _i64, _vp, _vp, _ci, _i64, _i32, _vp, _ci, _vp]
 _lib.dq_dequant_per_group.restype = _ci
+_lib.dq_w8a8_gemm.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _vp, _vp, _ci, _i32, _vp]
+_lib.dq_w8a8_gemm.restype = _ci
 _lib.dq_ada_layernorm_quant_noalloc.argtypes = [_vp, _ci, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _ci, _f32, _vp,
                                                 _vp, _vp]
 _lib.dq_ada_layernorm_quant_noalloc.restype = _ci
@@ -124,6 +126,11 @@ def dq_dequant_per_group(y, y_dtype, rows, cols, scale, offset, scale_dtype, gro
     """Raw call: pointers are ints (0/None for NULL). Returns the dq_status."""
     return _lib.dq_dequant_per_group(y, y_dtype, rows, cols, scale, offset, scale_dtype, group_size, k_dim, out,
                                      out_dtype, stream)
+
+
+def dq_w8a8_gemm(a, b, m, n, k, a_scale, b_scale, out, out_dtype, accumulate, stream) -> int:
+    """Raw call: pointers are ints (0/None for NULL). Returns the dq_status."""
+    return _lib.dq_w8a8_gemm(a, b, m, n, k, a_scale, b_scale, out, out_dtype, accumulate, stream)
 
 
 def dq_ada_layernorm_quant_noalloc(x, x_dtype, batch, seq, hidden, ada_scale, ada_shift, weight, bias, smooth,
@@ -297,6 +304,28 @@ def dequant_per_group(y, scale, offset=None, group_size: int = 32, k_dim: int = 
         stream = torch.cuda.current_stream(y.device).cuda_stream
     st = dq_dequant_per_group(_dev_ptr(y, "y"), yc, rows, cols, _dev_ptr(scale, "scale"), _dev_ptr(offset, "offset"),
                               sdt, int(group_size), int(k_dim), _dev_ptr(out, "out"), _dtype_code(out), stream)
+    if check and st != DQ_OK:
+        raise DQError(st)
+    return out
+
+
+def w8a8_gemm(a, b, a_scale, b_scale, out_dtype=None, out=None, accumulate: bool = False, stream=None,
+              check: bool = True):
+    """out = float(a @ b.T) * (a_scale[:, None] * b_scale[None, :]) (+ out).
+
+    ``a``: CUDA int8 [M, K]; ``b``: CUDA int8 [N, K]; scales float32 [M], [N].
+    Returns the [M, N] output (``out_dtype`` default float32).
+    """
+    torch = _torch()
+    m, k = (int(v) for v in a.shape)
+    n = int(b.shape[0])
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype or torch.float32, device=a.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(a.device).cuda_stream
+    st = dq_w8a8_gemm(_dev_ptr(a, "a"), _dev_ptr(b, "b"), m, n, k, _dev_ptr(a_scale, "a_scale"),
+                      _dev_ptr(b_scale, "b_scale"), _dev_ptr(out, "out"), _dtype_code(out), 1 if accumulate else 0,
+                      stream)
     if check and st != DQ_OK:
         raise DQError(st)
     return out
