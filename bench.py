@@ -50,10 +50,25 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ---------------------------------------------------------------- helpers
 
+METRIC_W8A8 = "W8A8 product TFLOP/s (int8 tensor ops, per-token x per-channel scales) and % of the tensor roofline"
+
+
+def work(wl):
+    """(units per step, divisor to the reported unit, unit, metric): HBM bytes for
+    the bandwidth-bound operations, tensor ops (2 M N K) for the W8A8 product."""
+    if wl.kind == "w8a8_gemm":
+        m, k = (int(v) for v in wl.tensors["a"].shape)
+        n = int(wl.tensors["b"].shape[0])
+        return 2 * m * n * k, 1e12, "TFLOP/s", METRIC_W8A8
+    return algorithmic_bytes(wl), 1e9, "GB/s", METRIC
+
+
 def algorithmic_bytes(wl) -> int:
     """HBM bytes one call must move: x read, codes + per-row floats written, side tables read."""
     t = wl.tensors
     rows, cols = wl.rows, wl.cols
+    if wl.kind == "w8a8_gemm":
+        return int(sum(v.numel() * v.element_size() for v in t.values()) + rows * int(t["b"].shape[0]) * 2)
     if wl.kind.startswith("dequant"):
         # codes + scale (and offset) tables read, [rows, cols] outputs written
         total = sum(v.numel() * v.element_size() for v in t.values() if v is not None)
@@ -77,6 +92,9 @@ def algorithmic_bytes(wl) -> int:
 
 def workload_config(wl) -> dict:
     """The config keys that describe a workload's operation and types."""
+    if wl.kind == "w8a8_gemm":
+        return {"operation": "w8a8_gemm", "m": int(wl.tensors["a"].shape[0]), "n": int(wl.tensors["b"].shape[0]),
+                "k": int(wl.tensors["a"].shape[1]), "out_dtype": wl.out_dtype, "scales": "per-token x per-channel"}
     if wl.kind.startswith("dequant"):
         c = {"operation": wl.kind, "rows": wl.rows, "cols": wl.cols, "y_dtype": wl.y_dtype,
              "scale_dtype": str(wl.tensors["scale"].dtype).replace("torch.", ""), "out_dtype": wl.out_dtype,
@@ -94,14 +112,19 @@ def launches_per_call(wl) -> int:
     return 2 if wl.kind == "ada_layernorm_quant" else 1
 
 
-def measured_peaks():
+def measured_peaks(tensor: bool = False):
+    """(peak, kind): the measured HBM copy bandwidth (GB/s), or for the int8
+    tensor product the measured bf16 burst GEMM rate x 2 (the nominal int8 :
+    bf16 ratio, 4.5 : 2.25 PFLOP/s dense)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
             d = json.load(f)
+        if tensor:
+            return 2.0 * float(d["bf16_tflops"]), "measured"
         return float(d["hbm_gbs"]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return (2.0 * 1590.0 if tensor else FALLBACK_HBM_GBS), "fallback"
 
 
 def source_hash() -> str:
@@ -249,7 +272,10 @@ class Launcher:
         xs = wl.primary.to(device)
         for i in range(sets):
             x = xs if i == 0 else xs.clone()
-            if wl.kind.startswith("dequant"):
+            if wl.kind == "w8a8_gemm":
+                out = torch.empty((wl.rows, int(t["b"].shape[0])), dtype=torch.bfloat16, device=device)
+                self.sets.append(dict(x=x, out=out))
+            elif wl.kind.startswith("dequant"):
                 out = torch.empty((wl.rows, wl.cols), dtype={"f32": torch.float32, "f16": torch.float16,
                                                               "bf16": torch.bfloat16}[wl.out_dtype], device=device)
                 self.sets.append(dict(x=x, out=out))
@@ -265,8 +291,8 @@ class Launcher:
                 out = torch.empty(tuple(t["x"].shape), dtype=torch.int8, device=device)
                 qs = torch.empty(tuple(t["x"].shape[:2]), dtype=torch.float32, device=device)
                 self.sets.append(dict(x=x, out=out, qs=qs))
-        self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k not in ("x", "y")}
-        if wl.kind.startswith("dequant"):
+        self.side = {k: (v.to(device) if v is not None else None) for k, v in t.items() if k not in ("x", "y", "a")}
+        if wl.kind.startswith("dequant") or wl.kind == "w8a8_gemm":
             self.ws_bytes, self.ws = 0, None
         elif wl.kind == "dynamic_quant":
             gi = self.side.get("group_index")
@@ -295,7 +321,12 @@ class Launcher:
         self.calls = []
         ycode = {"int8": dq.DQ_INT8, "int4": dq.DQ_INT4X2, "int32": dq.DQ_INT32}
         for s in self.sets:
-            if wl.kind == "dequant_per_token":
+            if wl.kind == "w8a8_gemm":
+                d = self.side
+                args = (p(s["x"]), p(d["b"]), wl.rows, int(d["b"].shape[0]), int(s["x"].shape[1]), p(d["a_scale"]),
+                        p(d["b_scale"]), p(s["out"]), code[s["out"].dtype], 0, self.sptr)
+                self.calls.append((dq.dq_w8a8_gemm, args))
+            elif wl.kind == "dequant_per_token":
                 sc, off = self.side["scale"], self.side.get("offset")
                 args = (p(s["x"]), ycode[wl.y_dtype], wl.rows, wl.cols, p(sc), p(off), code[sc.dtype],
                         p(s["out"]), code[s["out"].dtype], self.sptr)
@@ -382,8 +413,8 @@ def run_ours(args, world, rank, local):
         del graph
 
     ms_per_step = ms / args.steps
-    gbs_per_gpu = nbytes / (ms_per_step * 1e-3) / 1e9
-    value = gbs_per_gpu * world  # every rank moved nbytes per step in ms_per_step (max over ranks)
+    units, divisor, unit, metric = work(wl)
+    value = units * world / (ms_per_step * 1e-3) / divisor  # every rank did `units` per step (max over ranks)
     rows_per_s = wl.rows * world / (ms_per_step * 1e-3)
 
     # end to end through the public API with host buffers: H2D of the step's
@@ -392,15 +423,16 @@ def run_ours(args, world, rank, local):
     if not args.no_e2e:
         e2e = run_e2e(dq, wl, device, nbytes, world, min(args.steps, 20))
 
-    peak, peak_kind = measured_peaks()
-    achieved = nbytes / (ms_local / args.steps * 1e-3) / 1e9
+    tensor = wl.kind == "w8a8_gemm"
+    peak, peak_kind = measured_peaks(tensor)
+    achieved = units / (ms_local / args.steps * 1e-3) / divisor
     result = None
     if rank == 0:
         traffic = profiled_traffic(args.workload)
         result = {
-            "metric": METRIC,
+            "metric": metric,
             "value": round(value, 2),
-            "unit": "GB/s",
+            "unit": unit,
             "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup,
@@ -408,7 +440,7 @@ def run_ours(args, world, rank, local):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32",
+            "dtype": "s8 x s8 -> s32, f32 scales" if tensor else "f32",
             "data": "synthetic",
             "config": {
                 "workload": args.workload,
@@ -420,15 +452,16 @@ def run_ours(args, world, rank, local):
                 "launch": "cuda graph of K launches" if args.graph else "eager C-ABI launches",
             },
             "roofline": {
-                "bound": "hbm",
+                "bound": "tensor" if tensor else "hbm",
                 "achieved": round(achieved, 2),
                 "peak": peak,
-                "unit": "GB/s",
+                "unit": unit,
                 "frac": round(achieved / peak, 4),
-                "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, copy kernel)" if peak_kind == "measured"
-                else "fallback 6.65 TB/s",
+                "peak_kind": ("measured bf16 burst GEMM (MEASURED_PEAKS.json bf16_tflops) x 2, the nominal int8 ratio"
+                              if tensor else "measured (MEASURED_PEAKS.json hbm_gbs, copy kernel)")
+                if peak_kind == "measured" else "fallback",
                 "traffic": traffic,
-                "kernel": {"dynamic_quant": "dynamic_quant_tma_kernel",
+                "kernel": {"dynamic_quant": "dynamic_quant_tma_kernel", "w8a8_gemm": "w8a8_gemm_tc_kernel",
                            "dequant_per_token": "dequant_vec_kernel (per-token layout)",
                            "dequant_per_group": "dequant_vec_kernel (per-group layout)",
                            "ada_layernorm_quant": "ada_layernorm_quant_tma_kernel (time of the whole call: "
@@ -464,7 +497,11 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
     for _ in range(nsets):
         d_in = {k: (v.to(device) if v is not None else None) for k, v in host_in.items()}  # outputs sized by a real call
         odt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}[wl.out_dtype]
-        if wl.kind == "dequant_per_token":
+        if wl.kind == "w8a8_gemm":
+            o = dq.w8a8_gemm(d_in["a"], d_in["b"], d_in["a_scale"], d_in["b_scale"], out_dtype=odt,
+                             stream=s_call.cuda_stream)
+            outs = (o,)
+        elif wl.kind == "dequant_per_token":
             o = dq.dequant_per_token(d_in["y"], d_in["scale"], d_in.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
                                      out_dtype=odt, stream=s_call.cuda_stream)
             outs = (o,)
@@ -485,7 +522,8 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
                                                                      dq._dtype_code(d_in["ada_scale"]))
             ws = torch.empty((ws_bytes + 15) // 16 * 4, dtype=torch.float32, device=device) if ws_bytes else None
             outs = (y, sc, ws)
-        keep = {"dynamic_quant": 3, "ada_layernorm_quant": 2, "dequant_per_token": 1, "dequant_per_group": 1}[wl.kind]
+        keep = {"dynamic_quant": 3, "ada_layernorm_quant": 2, "dequant_per_token": 1, "dequant_per_group": 1,
+                "w8a8_gemm": 1}[wl.kind]
         results = [o for o in outs[:keep] if o is not None]
         h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in results]
         ev = {n: torch.cuda.Event() for n in ("in", "call", "out")}
@@ -505,7 +543,9 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
             ev["in"].record(s_in)
         s_call.wait_event(ev["in"])
         d = st["in"]
-        if wl.kind == "dequant_per_token":
+        if wl.kind == "w8a8_gemm":
+            dq.w8a8_gemm(d["a"], d["b"], d["a_scale"], d["b_scale"], out=st["outs"][0], stream=s_call.cuda_stream)
+        elif wl.kind == "dequant_per_token":
             dq.dequant_per_token(d["y"], d["scale"], d.get("offset"), y_dtype=wl.y_dtype, cols=wl.cols,
                                  out=st["outs"][0], stream=s_call.cuda_stream)
         elif wl.kind == "dequant_per_group":
@@ -544,7 +584,8 @@ def run_e2e(dq, wl, device, nbytes, world, steps):
     ms = max_over_ranks(start.elapsed_time(end), world, device) / steps
     h2d = sum(v.numel() * v.element_size() for v in host_in.values() if v is not None)
     d2h = sum(o.numel() * o.element_size() for o in sets[0]["results"])
-    return {"value": round(nbytes * world / (ms * 1e-3) / 1e9, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+    units, divisor, unit, _ = work(wl)
+    return {"value": round(units * world / (ms * 1e-3) / divisor, 3), "unit": unit, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4), "steps": steps,
             "note": "every step: pinned host inputs -> device, C-ABI call, results -> pinned host; "
                     "pipelined over 3 buffer sets on separate copy / compute streams"}
@@ -556,6 +597,9 @@ def _oracle_rows(wl, r0, r1):
     import oracle
 
     t = wl.tensors
+    if wl.kind == "w8a8_gemm":
+        return oracle.w8a8_gemm(t["a"][r0:r1].numpy(), t["b"].numpy(), t["a_scale"][r0:r1].numpy(),
+                                t["b_scale"].numpy(), out_dtype=wl.out_dtype)
     if wl.kind == "dequant_per_group":
         off = t.get("offset")
         if wl.k_dim == 1:
@@ -594,7 +638,8 @@ def _oracle_rows(wl, r0, r1):
 def cpu_baseline(wl, nbytes, target_s: float = 10.0):
     """The oracle as it stands, single-threaded, on a bounded sample of rows."""
     rows = wl.rows
-    bytes_per_row = nbytes / rows
+    units, divisor, unit, _ = work(wl)
+    bytes_per_row = units / rows  # work units (bytes, or tensor ops) per row
     # calibrate on a small slice, then size the sample to ~target_s of CPU work
     n0 = min(rows, 64)
     t0 = time.perf_counter()
@@ -609,10 +654,10 @@ def cpu_baseline(wl, nbytes, target_s: float = 10.0):
         elapsed += time.perf_counter() - t0
         done += n
         passes += 1
-    gbs = done * bytes_per_row / elapsed / 1e9
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    gbs = done * bytes_per_row / elapsed / divisor
+    return {"value": round(gbs, 6), "unit": unit, "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {rows} rows x {passes} pass(es) ({elapsed:.1f} s), "
-                      "single-threaded C++ oracle, GB/s of the same algorithmic bytes",
+                      f"single-threaded C++ oracle, {unit} of the same algorithmic work",
             "host_cpus": os.cpu_count()}
 
 
@@ -622,9 +667,9 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     wl = workloads.make(args.workload, rows=args.rows)
-    nbytes = algorithmic_bytes(wl)
+    units, divisor, unit, metric = work(wl)
     rows = wl.rows
-    bytes_per_row = nbytes / rows
+    bytes_per_row = units / rows  # work units (bytes, or tensor ops) per row
     # size each step so that warmup + steps take about args.cpu_seconds in total
     n0 = min(rows, 64)
     t0 = time.perf_counter()
@@ -639,13 +684,13 @@ def run_reference(args, world, rank):
         _oracle_rows(wl, 0, n)
     elapsed = time.perf_counter() - t0
     ms_per_step = elapsed / args.steps * 1e3
-    gbs = n * bytes_per_row * args.steps / elapsed / 1e9
+    gbs = n * bytes_per_row * args.steps / elapsed / divisor
     sample = f"first {n} of {rows} rows per step, single-threaded C++ oracle"
     return {
         "impl": "reference",
-        "metric": METRIC,
-        "value": round(gbs, 4),
-        "unit": "GB/s",
+        "metric": metric,
+        "value": round(gbs, 6),
+        "unit": unit,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -657,8 +702,8 @@ def run_reference(args, world, rank):
         "data": "synthetic",
         "config": {"workload": args.workload, **workload_config(wl), "rows_per_step": n,
                    "rows_per_s": round(n * args.steps / elapsed, 1)},
-        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
-        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": round(gbs, 6), "unit": unit, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "reference arm = the CPU oracle (the pages ship no runnable implementation)",
     }
 

@@ -12,13 +12,16 @@
 // Tensor-core path (M, N, K multiples of 128; 16-byte aligned operands): one
 // CTA per 128 x 128 output tile, 6 warps.
 //   warp 0      TMA producer: 128-row x 128-byte K tiles of A and B (K-major,
-//               128-byte swizzle) into a 4-stage shared-memory ring.
+//               128-byte swizzle) into a 3-stage shared-memory ring.
 //   warp 1      allocates 128 TMEM columns (the int32 accumulator, row m in
 //               lane m); one lane issues tcgen05.mma.kind::i8 (M=128, N=128,
 //               K=32, four per stage) and releases each stage with
 //               tcgen05.commit, then commits the accumulator.
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, 32 columns at
-//               a time, scales, optional accumulation, narrowing, stores.
+//   warps 2-5   epilogue: the tile's column scales staged in shared memory,
+//               tcgen05.ld of their 32-lane quarter, 32 columns at a time,
+//               scales, optional accumulation, narrowing, 16-byte stores.
+// Three ring stages keep a CTA at 97 KB of shared memory, so two CTAs share
+// an SM and one's epilogue overlaps the other's main loop.
 // Every mbarrier wait is bounded; the MMA lane always issues the final
 // commit, so teardown never frees TMEM under MMAs in flight.
 // Other shapes or alignments: a CUDA-core kernel with the same arithmetic.
@@ -37,11 +40,11 @@
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kBK = 128;  // tile; kBK bytes = one 128-byte swizzle row
-constexpr int kStages = 4;
+constexpr int kStages = 3;  // 96 KB of ring: two CTAs share an SM, one's epilogue overlapping the other's MMAs
 constexpr uint32_t kTileBytes = kBM * kBK;  // 16 KB for A and for B (kBM == kBN)
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 128;
-constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + 256;  // alignment slack + ring + barriers
+constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + 256 + kBN * 4;  // slack, ring, barriers, scales
 
 struct W8A8Args {
   const int8_t* a;
@@ -52,6 +55,7 @@ struct W8A8Args {
   int64_t m, n, k;
   int out_kind;    // 0 f32, 1 f16, 2 bf16
   int accumulate;  // out (f32) += product
+  int vec_out;     // out is 16-byte aligned: whole-row-chunk vector stores
 };
 
 __device__ __forceinline__ void store_out(const W8A8Args& a, int64_t e, float t) {
@@ -131,6 +135,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   uint64_t* empty = full + kStages;
   uint64_t* acc_ready = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 1);
+  float* col_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // the tile's b_scale
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -192,6 +197,9 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       tc_commit(acc_ready);  // every MMA issued above is complete when this arrives
     }
   } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
+    // the tile's column scales, staged once (128 threads, one each)
+    col_scale[threadIdx.x - 64] = a.b_scale[n0 + threadIdx.x - 64];
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     const bool ready = dq::mbar_wait_parity(acc_ready, 0);
     tc_fence_after();
     const int quarter = warp & 3;
@@ -202,12 +210,47 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       uint32_t r[32];
       tc_ld_32cols(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * c), r);
       if (!ready) continue;
-      const int64_t col0 = n0 + 32 * c;
+      float t[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float scales = __fmul_rn(sa_row, a.b_scale[col0 + j]);
-        const float t = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
-        store_out(a, row * a.n + col0 + j, t);
+        const float scales = __fmul_rn(sa_row, col_scale[32 * c + j]);
+        t[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
+      }
+      const int64_t e0 = row * a.n + n0 + 32 * c;  // 32 consecutive outputs of this row
+      if (a.vec_out) {
+        if (a.out_kind == 0) {
+          float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + e0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 v = make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
+            if (a.accumulate) {
+              const float4 y = o[q];
+              v = make_float4(__fadd_rn(v.x, y.x), __fadd_rn(v.y, y.y), __fadd_rn(v.z, y.z), __fadd_rn(v.w, y.w));
+            }
+            o[q] = v;
+          }
+        } else {
+          uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + e0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float x0 = t[8 * q + 2 * h], x1 = t[8 * q + 2 * h + 1];
+              if (a.out_kind == 1) {
+                const __half2 p2 = __floats2half2_rn(x0, x1);
+                w[h] = *reinterpret_cast<const uint32_t*>(&p2);
+              } else {
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(x0, x1);
+                w[h] = *reinterpret_cast<const uint32_t*>(&p2);
+              }
+            }
+            o[q] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) store_out(a, e0 + j, t[j]);
       }
     }
   }
@@ -308,7 +351,7 @@ extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, i
   const size_t os = out_dtype == DQ_F32 ? 4 : 2;
   if (!aligned_to(a_scale, 4) || !aligned_to(b_scale, 4) || !aligned_to(out, os)) return DQ_ERR_MISALIGNED;
   W8A8Args args{a, b, a_scale, b_scale, out, m, n, k, out_dtype == DQ_F32 ? 0 : (out_dtype == DQ_F16 ? 1 : 2),
-                accumulate};
+                accumulate, aligned_to(out, 16) ? 1 : 0};
   const bool tiles = m % kBM == 0 && n % kBN == 0 && k % kBK == 0 && m / kBM <= 65535 &&
                      aligned_to(a, 16) && aligned_to(b, 16);
   if (tiles) {

@@ -35,6 +35,11 @@ LayerNorm path):
   (seed 8), groups of 128 along each row with fp32 scale [8192, 32]
   ~ U(0.001, 0.05) (seed 9) and offset [8192, 32] ~ N(0, 8) (seed 10),
   bfloat16 output.
+* ``w8a8_gemm_int8_bf16_4096x4096x4096`` (aclnnQuantBatchMatmulInplaceAdd,
+  the consumer of the codes): a int8 [4096, 4096] and b int8 [4096, 4096]
+  uniform in [-127, 127] (seeds 11, 12), per-token scale fp32 [4096]
+  ~ U(0.001, 0.02) (seed 13), per-channel scale fp32 [4096] ~ U(0.001, 0.02)
+  (seed 14), bfloat16 output.
 """
 
 from __future__ import annotations
@@ -89,7 +94,7 @@ class Workload:
     """One synthetic workload: named tensors on the CPU plus the call's options."""
 
     name: str
-    kind: str                    # "dynamic_quant" | "ada_layernorm_quant" | "dequant_per_token" | "dequant_per_group"
+    kind: str                    # "dynamic_quant" | "ada_layernorm_quant" | "dequant_per_token" | "dequant_per_group" | "w8a8_gemm"
     tensors: dict = field(default_factory=dict)
     mode: str = "symmetric"      # dynamic_quant only
     y_dtype: str = "int8"        # code container (dynamic_quant output, dequant_per_token input)
@@ -101,6 +106,8 @@ class Workload:
     @property
     def primary(self):
         """The per-row input: x, or the codes of a dequantization."""
+        if self.kind == "w8a8_gemm":
+            return self.tensors["a"]
         return self.tensors["y"] if self.kind.startswith("dequant") else self.tensors["x"]
 
     @property
@@ -110,6 +117,8 @@ class Workload:
 
     @property
     def cols(self) -> int:
+        if self.kind == "w8a8_gemm":
+            return int(self.tensors["a"].shape[-1])
         if self.kind.startswith("dequant"):
             return int(self.tensors["y"].shape[-1]) * {"int8": 1, "int4": 2, "int32": 8}[self.y_dtype]
         return int(self.tensors["x"].shape[-1])
@@ -123,6 +132,7 @@ WORKLOADS = (
     "ada_layernorm_quant_bf16_4x4096x3072",
     "dequant_per_token_int8_bf16_8192x4096",
     "dequant_per_group_int8_bf16_8192x4096_g128",
+    "w8a8_gemm_int8_bf16_4096x4096x4096",
 )
 
 
@@ -176,4 +186,11 @@ def make(name: str, rows: int | None = None) -> Workload:
         offset = normal((r, 32), torch.float32, 10, std=8.0)
         return Workload(name, "dequant_per_group", {"y": y, "scale": scale, "offset": offset}, y_dtype="int8",
                         out_dtype="bf16", group_size=128, k_dim=1)
+    if name == "w8a8_gemm_int8_bf16_4096x4096x4096":
+        m = rows or 4096
+        a = torch.randint(-127, 128, (m, 4096), generator=_gen(11), dtype=torch.int32).to(torch.int8)
+        b = torch.randint(-127, 128, (4096, 4096), generator=_gen(12), dtype=torch.int32).to(torch.int8)
+        return Workload(name, "w8a8_gemm", {"a": a, "b": b, "a_scale": uniform((m,), torch.float32, 13, 0.001, 0.02),
+                                            "b_scale": uniform((4096,), torch.float32, 14, 0.001, 0.02)},
+                        out_dtype="bf16")
     raise KeyError(f"unknown workload {name!r}; known: {', '.join(WORKLOADS)}")
