@@ -127,20 +127,30 @@ def measured_peaks(tensor: bool = False):
         return (2.0 * 1590.0 if tensor else FALLBACK_HBM_GBS), "fallback"
 
 
-def source_hash() -> str:
+# The sources each operation's kernels are built from (a profile's traffic
+# figure stays valid while these are unchanged).
+KERNEL_SOURCES = {
+    "dynamic_quant": ("dynamic_quant_kernels.cuh", "dq_device.cuh", "tma_pipeline.cuh", "dq_api.cu"),
+    "ada_layernorm_quant": ("ada_layernorm_quant_kernels.cuh", "dq_device.cuh", "tma_pipeline.cuh", "dq_api.cu"),
+    "dequant_per_token": ("dequant_kernels.cuh", "dq_device.cuh", "dq_api.cu"),
+    "dequant_per_group": ("dequant_kernels.cuh", "dq_device.cuh", "dq_api.cu"),
+    "w8a8_gemm": ("w8a8_gemm.cu", "tma_pipeline.cuh"),
+}
+
+
+def source_hash(kind: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "token_dynamic_quantization_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kind: str):
     """dram read+write bytes per launch from the committed ncu summary, if it
-    was taken on the current kernel sources (else None)."""
+    was taken on the current sources of the workload's kernels (else None)."""
     path = os.path.join(ROOT, "profiles", f"ncu_{workload}.md")
     try:
         text = open(path).read()
@@ -148,7 +158,7 @@ def profiled_traffic(workload: str):
         return None
     m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != source_hash(kind):
         return None
     return int(m_bytes.group(1))
 
@@ -428,7 +438,7 @@ def run_ours(args, world, rank, local):
     achieved = units / (ms_local / args.steps * 1e-3) / divisor
     result = None
     if rank == 0:
-        traffic = profiled_traffic(args.workload)
+        traffic = profiled_traffic(args.workload, wl.kind)
         result = {
             "metric": metric,
             "value": round(value, 2),

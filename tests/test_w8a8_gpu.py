@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import oracle
+from token_dynamic_quantization_b200 import workloads
 
 pytestmark = pytest.mark.gpu
 
@@ -106,3 +107,30 @@ def test_quantize_then_multiply(dq):
     yo, so, _ = oracle.dynamic_quant(x)
     want = oracle.w8a8_gemm(yo, w.numpy(), so, ws.numpy(), out_dtype="bf16")
     np.testing.assert_array_equal(_bits(got.cpu()), want.view(np.uint16))
+
+
+def test_empty_product(dq):
+    dev = torch.device("cuda:0")
+    a = torch.empty(0, 256, dtype=torch.int8, device=dev)
+    b = torch.randint(-128, 128, (128, 256), dtype=torch.int32).to(torch.int8).to(dev)
+    o = dq.w8a8_gemm(a, b, torch.empty(0, device=dev), torch.ones(128, device=dev), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert tuple(o.shape) == (0, 128)
+
+
+@pytest.mark.slow
+def test_w8a8_workload_full_size(dq):
+    """The benchmark's 4096^3 product, bf16 out, on sampled rows: one at random
+    in each 128-row tile band, plus the first and last rows of the matrix."""
+    wl = workloads.make("w8a8_gemm_int8_bf16_4096x4096x4096")
+    t = wl.tensors
+    dev = torch.device("cuda:0")
+    got = dq.w8a8_gemm(t["a"].to(dev), t["b"].to(dev), t["a_scale"].to(dev), t["b_scale"].to(dev),
+                       out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    got = _bits(got.cpu())
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 128) + rng.integers(0, 128, 32), [0, 4095]]))
+    want = oracle.w8a8_gemm(t["a"][rows].numpy(), t["b"].numpy(), t["a_scale"][rows].numpy(),
+                            t["b_scale"].numpy(), out_dtype="bf16")
+    np.testing.assert_array_equal(got[rows], want.view(np.uint16))
