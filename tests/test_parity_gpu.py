@@ -300,7 +300,7 @@ def test_empty_input_is_a_noop(dq):
 
 # ---------------------------------------------------------------- full-size workloads
 
-DQ_WORKLOADS = [w for w in workloads.WORKLOADS if not w.startswith(("ada_", "dequant"))]
+DQ_WORKLOADS = [w for w in workloads.WORKLOADS if not w.startswith(("ada_", "dequant", "w8a8"))]
 
 
 @pytest.mark.slow
@@ -395,6 +395,19 @@ def test_ada_large_mean_rows(dq, h, dtype):
     """Rows with mean far above their spread (1000 +- 3): E(x) must be accurate
     to well below the spread, or most codes move."""
     x, sc, sh, w, bias, sm = _ada_inputs(3, 13, h, dtype, torch.bfloat16, seed=h + 5, x_mean=1000.0, x_std=3.0)
+    want = oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6)
+    got = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
+    assert_ada_close(got, want)
+
+
+@pytest.mark.parametrize("h", [3072, 1000])
+def test_ada_rows_with_outlying_first_elements(dq, h):
+    """Rows whose first 8 elements sit far from the row mean: the one-reduction
+    moments about those elements would cancel, so these rows take the centred
+    second pass."""
+    x, sc, sh, w, bias, sm = _ada_inputs(2, 9, h, torch.bfloat16, torch.bfloat16, seed=h + 9)
+    x[:, ::2, :8] = 40.0
+    x[:, 1::4, :8] = -25.0
     want = oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6)
     got = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
     assert_ada_close(got, want)

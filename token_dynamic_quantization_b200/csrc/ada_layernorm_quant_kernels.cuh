@@ -19,17 +19,21 @@
 //      the row kernel only after that work has completed.
 //
 // Arithmetic:
-//   * E(x), Var(x): the row is resident, so a two-pass mean / centred
-//     variance costs no extra traffic (no Welford needed). Per-thread partial
-//     sums are fp32, the cross-thread sums double; the variance is corrected
-//     to the double mean, sum (v - m_d)^2 = sum (v - m_f)^2 - H (m_d - m_f)^2,
-//     so both statistics match a double evaluation rounded to fp32 except for
-//     the last bit in rare rows.
-//   * n = (x - E(x)) * rstd with rstd = RN(1 / RN(sqrt(Var + eps))), then
-//     y = n * A + B. Against a sequential evaluation that rounds every printed
-//     operation separately and divides by the square root, this moves y by a
-//     few ulps: quant_scale stays within a relative 1e-6 and about one code in
-//     10^6 moves by one (measured on the 4 x 4096 x 3072 workload).
+//   * E(x), Var(x) from one row reduction: each thread sums d = x - K and d^2
+//     over its share, with K the mean of the row's first 8 elements (the same
+//     value in every thread; d is exact when x and K are within a factor 2,
+//     as on rows whose mean is far above their spread). Partial sums are fp32,
+//     the sums across warps double; E(x) = K + E(d), Var = E(d^2) - E(d)^2.
+//     While E(d)^2 <= 3/4 E(d^2) that difference loses at most a factor 4 of
+//     relative accuracy. Rows past the bound (first elements far from the
+//     mean) take a centred second pass about RN(E(x)). E(x) is rounded to
+//     fp32 once, as the formula's mean is.
+//   * n = (x - E(x)) * rstd with rstd = RN(1 / RN(sqrt(Var + eps))), as
+//     fma(d, rstd, -(E(x) - K) * rstd), then y = n * A + B. Against a
+//     sequential evaluation that rounds every printed operation separately
+//     and divides by the square root, this moves y by a few ulps:
+//     quant_scale stays within a relative 1e-6 and about one code in 10^6
+//     moves by one.
 //   * steps 4-5 are the DynamicQuant quantizer (exact IEEE semantics).
 #pragma once
 
@@ -118,6 +122,9 @@ __device__ __noinline__ void ada_quantize_row_exact(const uint4* srow, const flo
 #define DQ_ADA_MAX_BLOCK 512
 #endif
 constexpr int kAdaMaxBlock = DQ_ADA_MAX_BLOCK;
+#ifndef DQ_ADA_ONEPASS
+#define DQ_ADA_ONEPASS 1  // both moments from one row reduction (see pass 1)
+#endif
 #ifndef DQ_ADA_MAX_REGS
 #define DQ_ADA_MAX_REGS 128  // the row share stays in registers across four passes
 #endif
@@ -130,7 +137,7 @@ template <typename InT, int VPT, bool kRagged>
 __global__ void __maxnreg__(DQ_ADA_MAX_REGS)
 ada_layernorm_quant_tma_kernel(const AdaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ double red_d[2][2][kAdaMaxBlock / 32];  // [parity][sum|sq][warp]
+  __shared__ double red_d[2][3][kAdaMaxBlock / 32];  // [parity][sum|sq|centred sq][warp]
   __shared__ float red_f[2][kAdaMaxBlock / 32];       // [parity][warp] absmax
 
   const int tpr = a.tpr;
@@ -208,6 +215,132 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const bool arrived = mbar_wait_parity(bars + c_stage, phase);
     const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(c_stage) * stride);
 
+#if DQ_ADA_ONEPASS
+    // ---- pass 1: load, widen, shift by K, both moments of d = x - K
+    // K is the mean of the row's first 8 elements, the same value in every
+    // thread. E(d) and E(d^2) come out of one reduction; Var = E(d^2) - E(d)^2
+    // loses at most a factor 4 of relative accuracy while E(d)^2 <= 3/4 E(d^2),
+    // and rows past that bound take a centred second pass.
+    constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
+    float K;
+    {
+      float f[8];
+      InTraits<InT>::widen8(srow[0], f);
+      K = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(f[0], f[1]), __fadd_rn(f[2], f[3])),
+                              __fadd_rn(__fadd_rn(f[4], f[5]), __fadd_rn(f[6], f[7]))),
+                    0.125f);
+    }
+    float v[VPT][8];
+    float2 acc[NACC], acq[NACC];
+#pragma unroll
+    for (int j = 0; j < NACC; ++j) acc[j] = acq[j] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const bool active = in_row(k);
+      InTraits<InT>::widen8(active ? srow[vbase + 32 * k] : make_uint4(0, 0, 0, 0), v[k]);
+      float2 d[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        d[p] = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-K));
+        if (kRagged && !active) d[p] = make_float2(0.0f, 0.0f);
+        v[k][2 * p] = d[p].x;
+        v[k][2 * p + 1] = d[p].y;
+        acq[(k + p) % NACC] = __ffma2_rn(d[p], d[p], acq[(k + p) % NACC]);
+      }
+      acc[k % NACC] = __fadd2_rn(acc[k % NACC], __fadd2_rn(__fadd2_rn(d[0], d[1]), __fadd2_rn(d[2], d[3])));
+    }
+#pragma unroll
+    for (int j = 1; j < NACC; ++j) {
+      acc[0] = __fadd2_rn(acc[0], acc[j]);
+      acq[0] = __fadd2_rn(acq[0], acq[j]);
+    }
+    // butterflies: every lane ends with the same bits (each step adds the
+    // same two operands on both lanes of a pair)
+    float s1 = __fadd_rn(acc[0].x, acc[0].y), s2 = __fadd_rn(acq[0].x, acq[0].y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+      s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
+    }
+    double sum = s1, sq = s2;
+    bool failed;
+    if (nwarps_g > 1) {
+      if (lane == 0) {
+        red_d[parity][0][warp] = sum;
+        red_d[parity][1][warp] = sq;
+      }
+      failed = group_barrier_or(1 + g, tpr, !arrived);
+      sum = 0.0;
+      sq = 0.0;
+      for (int w = 0; w < nwarps_g; ++w) {
+        sum += red_d[parity][0][warp_g0 + w];
+        sq += red_d[parity][1][warp_g0 + w];
+      }
+    } else {
+      failed = __any_sync(0xffffffffu, !arrived);
+      __syncwarp();
+    }
+    if (failed) {
+      for (int64_t rr = r + lane_g; rr < r_end; rr += tpr) a.quant_scale[rr] = __int_as_float(0x7fc00000);
+      if (leader) {
+        int st = c_stage;
+        uint32_t ph = phase;
+        for (int64_t j = r - r_begin + 1; j < issued; ++j) {
+          st = st + 1 == S ? 0 : st + 1;
+          if (st == 0) ph ^= 1u;
+          mbar_wait_parity(bars + st, ph);
+        }
+      }
+      return;
+    }
+    // refill the stage of the previous row (S - 1 copies stay in flight; the
+    // current row's stage is kept for the out-of-line exact path)
+    if (leader && issued < n) {
+      fence_proxy_async_smem();
+      issue_next();
+    }
+    c_stage = c_stage + 1 == S ? 0 : c_stage + 1;
+    if (c_stage == 0) phase ^= 1u;
+    const double m1 = sum * a.inv_hidden;  // E(d)
+    const double m2 = sq * a.inv_hidden;   // E(d^2)
+    const double mean_d = static_cast<double>(K) + m1;
+    const float mean_f = __double2float_rn(mean_d);
+    const float c_f = __fsub_rn(mean_f, K);  // mean_f - K (exact when K and mean_f are within a factor 2)
+    double var_d;
+    if (m1 * m1 <= 0.75 * m2) {
+      var_d = m2 - m1 * m1;
+    } else {
+      // ---- centred second pass (rows whose first elements sit far from the mean)
+#pragma unroll
+      for (int j = 0; j < NACC; ++j) acq[j] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        const bool active = in_row(k);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          float2 e = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-c_f));
+          if (kRagged && !active) e = make_float2(0.0f, 0.0f);
+          acq[(k + p) % NACC] = __ffma2_rn(e, e, acq[(k + p) % NACC]);
+        }
+      }
+#pragma unroll
+      for (int j = 1; j < NACC; ++j) acq[0] = __fadd2_rn(acq[0], acq[j]);
+      double sc = warp_sum(static_cast<double>(acq[0].x) + static_cast<double>(acq[0].y));
+      if (nwarps_g > 1) {
+        if (lane == 0) red_d[parity][2][warp] = sc;
+        group_barrier(1 + g, tpr);
+        sc = 0.0;
+        for (int w = 0; w < nwarps_g; ++w) sc += red_d[parity][2][warp_g0 + w];
+      }
+      const double dm = m1 - static_cast<double>(c_f);
+      var_d = sc * a.inv_hidden - dm * dm;
+    }
+    var_d = var_d > 0.0 ? var_d : 0.0;
+    const float var_f = __double2float_rn(var_d);
+    const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
+    // n = (x - mean_f) * rstd = fma(d, rstd, -(mean_f - K) * rstd)
+    const float nb = -__fmul_rn(c_f, rstd);
+#else
     // ---- pass 1: load, widen, E(x)
     constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
     float v[VPT][8];
@@ -290,6 +423,7 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const float var_f = __double2float_rn(var_d);
     const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
 
+#endif
     // ---- pass 3: y = n * A + B, absmax
     float amx[NACC];
 #pragma unroll
@@ -303,7 +437,11 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
         const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
+#if DQ_ADA_ONEPASS
+          const float2 nn = __ffma2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd), f2(nb));
+#else
           const float2 nn = __fmul2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd));
+#endif
           const float2 y =
               __ffma2_rn(nn, make_float2(Av[2 * p], Av[2 * p + 1]), make_float2(Bv[2 * p], Bv[2 * p + 1]));
           v[k][2 * p] = y.x;
