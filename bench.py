@@ -139,12 +139,18 @@ KERNEL_SOURCES = {
 
 
 def source_hash(kind: str) -> str:
+    """Hash of the code in those sources: comments and blank lines are left
+    out, so a comment edit does not void a capture."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "token_dynamic_quantization_b200", "csrc")
     for name in KERNEL_SOURCES[kind]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(name.encode())
+        h.update(code.encode())
     return h.hexdigest()[:16]
 
 

@@ -282,9 +282,10 @@ dq_status dq_dequant_per_group(const void* y, dq_dtype y_dtype, int64_t rows, in
  *   a_scale  device float [m]; b_scale device float [n].
  *   out      device [m, n] of out_dtype (DQ_F32, DQ_F16, DQ_BF16);
  *            accumulate = 1 adds into it (DQ_F32 only), 0 overwrites.
- * k <= 2^17 (int32 sums cannot overflow). m, n, k multiples of 128 with
- * 16-byte aligned a and b run on tcgen05 tensor cores (128 x 128 tiles);
- * other shapes run a CUDA-core kernel with the same results.
+ * k <= 2^17 (int32 sums cannot overflow). With k a multiple of 16 and
+ * 16-byte aligned a and b, any m and n run on tcgen05 tensor cores
+ * (128 x 256 or 128 x 128 tiles, ragged edges zero-filled and masked); other
+ * shapes run a CUDA-core kernel with the same results.
  * Errors: DQ_ERR_BAD_SHAPE, DQ_ERR_BAD_DTYPE, DQ_ERR_BAD_ARGUMENT,
  * DQ_ERR_NULL_POINTER, DQ_ERR_MISALIGNED, DQ_ERR_CUDA. */
 dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,

@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("dq_get_workspace_size", "dq_dynamic_quant", "dq_ada_layernorm_quant_get_workspace_size",
-              "dq_ada_layernorm_quant", "dq_dequant_per_token", "dq_dequant_per_group", "dq_status_string"):
+              "dq_ada_layernorm_quant", "dq_dequant_per_token", "dq_dequant_per_group", "dq_w8a8_gemm",
+              "dq_ada_layernorm_quant_noalloc", "dq_status_string"):
         assert n in names
 
 
@@ -227,3 +228,44 @@ def test_binding_fails_loudly_without_library(tmp_path):
     res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
     assert res.returncode != 0
     assert "ImportError" in res.stderr and "no CPU fallback" in res.stderr
+
+
+def test_w8a8_gemm_validation(dq_lib):
+    """Every invalid W8A8 call is rejected on the host before any launch."""
+    d = dq_lib
+
+    def mm(**kw):
+        args = dict(a=FAKE, b=FAKE, m=256, n=256, k=256, a_scale=FAKE, b_scale=FAKE, out=FAKE,
+                    out_dtype=d.DQ_BF16, accumulate=0, stream=None)
+        args.update(kw)
+        return d.dq_w8a8_gemm(**args)
+
+    assert mm(m=0, a=None, out=None) == d.DQ_OK  # empty: nothing launched
+    assert mm(n=0, b=None, out=None) == d.DQ_OK
+    cases = [
+        (dict(k=0), d.DQ_ERR_BAD_SHAPE),
+        (dict(k=(1 << 17) + 16), d.DQ_ERR_BAD_SHAPE),  # int32 sums could overflow
+        (dict(m=-1), d.DQ_ERR_BAD_SHAPE),
+        (dict(out_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
+        (dict(accumulate=2), d.DQ_ERR_BAD_ARGUMENT),
+        (dict(accumulate=1), d.DQ_ERR_BAD_ARGUMENT),  # the in-place add needs an f32 out
+        (dict(a=None), d.DQ_ERR_NULL_POINTER),
+        (dict(b_scale=None), d.DQ_ERR_NULL_POINTER),
+        (dict(a_scale=FAKE + 2), d.DQ_ERR_MISALIGNED),
+        (dict(out=FAKE + 1), d.DQ_ERR_MISALIGNED),
+        (dict(out_dtype=d.DQ_F32, out=FAKE + 2), d.DQ_ERR_MISALIGNED),
+    ]
+    for kw, want in cases:
+        assert mm(**kw) == want, kw
+
+
+def test_w8a8_helper_checks_shapes_on_the_host(dq_lib):
+    import torch
+
+    a = torch.zeros(4, 32, dtype=torch.int8)
+    with pytest.raises(ValueError):
+        dq_lib.w8a8_gemm(a, torch.zeros(8, 16, dtype=torch.int8), torch.ones(4), torch.ones(8))
+    with pytest.raises(TypeError):
+        dq_lib.w8a8_gemm(a, torch.zeros(8, 32, dtype=torch.int8), torch.ones(3), torch.ones(8))
+    with pytest.raises(TypeError):
+        dq_lib.w8a8_gemm(a.float(), torch.zeros(8, 32, dtype=torch.int8), torch.ones(4), torch.ones(8))

@@ -3,8 +3,8 @@
 dq_w8a8_gemm through the C ABI against the CPU oracle, bit for bit: the
 integer sum is exact on both sides, and the scale product, the multiply, the
 optional accumulation and the narrowing are single binary32 roundings in the
-same order. Shapes that are multiples of 128 run on the tcgen05 tensor cores;
-others on the CUDA-core kernel.
+same order. Shapes with K a multiple of 16 run on the tcgen05 tensor cores
+(ragged M and N included); others on the CUDA-core kernel.
 """
 
 import numpy as np
@@ -44,7 +44,7 @@ def _bits(t):
     return t.view(torch.int16).numpy().view(np.uint16) if t.dtype != torch.float32 else t.numpy().view(np.uint32)
 
 
-TC_SHAPES = [(128, 128, 128), (256, 384, 512), (128, 256, 1024), (384, 128, 2048)]
+TC_SHAPES = [(128, 128, 128), (256, 384, 512), (128, 256, 1024), (384, 128, 2048), (256, 768, 384), (128, 512, 4096)]
 
 
 @pytest.mark.parametrize("shape", TC_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in TC_SHAPES])
@@ -85,7 +85,32 @@ def test_extreme_codes_large_k(dq):
     np.testing.assert_array_equal(got.numpy().view(np.uint32), want.view(np.uint32))
 
 
-@pytest.mark.parametrize("shape", [(5, 7, 33), (130, 128, 128), (128, 128, 96), (64, 200, 256)])
+RAGGED_TC_SHAPES = [(130, 128, 128), (128, 128, 96), (64, 200, 256), (1, 256, 16), (200, 300, 272),
+                    (77, 520, 1040), (129, 385, 4112), (300, 640, 128)]
+
+
+@pytest.mark.parametrize("shape", RAGGED_TC_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in RAGGED_TC_SHAPES])
+@pytest.mark.parametrize("out_dtype,name", [(torch.float32, "f32"), (torch.bfloat16, "bf16")])
+def test_ragged_tensor_core_path_matches_oracle(dq, shape, out_dtype, name):
+    """m, n, k not multiples of the tile (k a multiple of 16): zero-filled
+    loads and masked stores on the tensor-core path, bit for bit."""
+    m, n, k = shape
+    a, b, sa, sb = _case(m, n, k, seed=m + n + k)
+    want = oracle.w8a8_gemm(a.numpy(), b.numpy(), sa.numpy(), sb.numpy(), out_dtype=name)
+    got = _run(dq, a, b, sa, sb, out_dtype=out_dtype)
+    np.testing.assert_array_equal(_bits(got), want.view(np.uint32 if name == "f32" else np.uint16))
+
+
+def test_ragged_accumulate(dq):
+    a, b, sa, sb = _case(150, 330, 208, seed=12)
+    base = torch.randn(150, 330, generator=torch.Generator().manual_seed(13))
+    want = oracle.w8a8_gemm(a.numpy(), b.numpy(), sa.numpy(), sb.numpy(), out_dtype="f32",
+                            accumulate_into=base.numpy().copy())
+    got = _run(dq, a, b, sa, sb, accumulate_into=base.clone())
+    np.testing.assert_array_equal(_bits(got), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", [(5, 7, 33), (3, 40, 40), (64, 130, 200)])
 def test_cuda_core_path_matches_oracle(dq, shape):
     m, n, k = shape
     a, b, sa, sb = _case(m, n, k, seed=m * n + k)

@@ -320,13 +320,13 @@ dq_status launch_ada_ragged(dq::AdaArgs a, int device, int sms, cudaStream_t str
 
 // AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8}, fewest wasted lanes,
 // then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
-// three row reductions; the row share stays in registers). DQ_ADA_STAGES row
+// two row reductions; the row share stays in registers). DQ_ADA_STAGES row
 // buffers per group, one of them holding the row being processed.
 #ifndef DQ_ADA_TARGET_VPT
-#define DQ_ADA_TARGET_VPT 4
+#define DQ_ADA_TARGET_VPT 6  // hidden 3072: 2 warps x 6 vectors per row (2811 GB/s) over 3 x 4 (2652)
 #endif
 #ifndef DQ_ADA_CTA_BYTES
-#define DQ_ADA_CTA_BYTES 98304
+#define DQ_ADA_CTA_BYTES 147456  // 8 row groups of 64 threads at hidden 3072: 16 warps per SM
 #endif
 #ifndef DQ_ADA_STAGES
 #define DQ_ADA_STAGES 3

@@ -9,22 +9,27 @@
 //   out[m,n] = float(acc) * (a_scale[m] * b_scale[n])  (+ out[m,n])
 // each binary32 operation rounded once in that order, then narrowed.
 //
-// Tensor-core path (M, N, K multiples of 128; 16-byte aligned operands): one
-// CTA per 128 x 128 output tile, 6 warps.
-//   warp 0      TMA producer: 128-row x 128-byte K tiles of A and B (K-major,
-//               128-byte swizzle) into a 3-stage shared-memory ring.
-//   warp 1      allocates 128 TMEM columns (the int32 accumulator, row m in
-//               lane m); one lane issues tcgen05.mma.kind::i8 (M=128, N=128,
+// Tensor-core path (K a multiple of 16, 16-byte aligned operands; any M, N):
+// one CTA per 128 x BN output tile, 6 warps, BN = 256 unless a 128-wide last
+// tile wastes less. Tiles past M, N or K are zero-filled by the loads and
+// masked in the epilogue.
+//   warp 0      TMA producer: 128-byte K slices of 128 rows of A and BN rows
+//               of B (K-major, 128-byte swizzle) into a shared-memory ring.
+//   warp 1      allocates BN TMEM columns (the int32 accumulator, row m in
+//               lane m); one lane issues tcgen05.mma.kind::i8 (M=128, N=BN,
 //               K=32, four per stage) and releases each stage with
 //               tcgen05.commit, then commits the accumulator.
 //   warps 2-5   epilogue: the tile's column scales staged in shared memory,
 //               tcgen05.ld of their 32-lane quarter, 32 columns at a time,
 //               scales, optional accumulation, narrowing, 16-byte stores.
-// Three ring stages keep a CTA at 97 KB of shared memory, so two CTAs share
-// an SM and one's epilogue overlaps the other's main loop.
+// The ring holds 96 KB (2 stages of 48 KB at BN = 256, 3 of 32 KB at 128),
+// so two CTAs share an SM (and its 512 TMEM columns) and one's epilogue
+// overlaps the other's main loop. The 256-wide tile reads 48 KB of operands
+// per 2^22 multiply-adds instead of 64 KB: on 4096^3, 58.6 us against 65.4.
 // Every mbarrier wait is bounded; the MMA lane always issues the final
 // commit, so teardown never frees TMEM under MMAs in flight.
-// Other shapes or alignments: a CUDA-core kernel with the same arithmetic.
+// K not a multiple of 16, or unaligned operands: a CUDA-core kernel with the
+// same arithmetic.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -39,12 +44,33 @@
 
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kBK = 128;  // tile; kBK bytes = one 128-byte swizzle row
-constexpr int kStages = 3;  // 96 KB of ring: two CTAs share an SM, one's epilogue overlapping the other's MMAs
-constexpr uint32_t kTileBytes = kBM * kBK;  // 16 KB for A and for B (kBM == kBN)
+// Output tile kBM x BN (BN = 128 or 256 columns), K in steps of kBK bytes =
+// one 128-byte swizzle row.
+constexpr int kBM = 128, kBK = 128;
+#ifndef DQ_W8A8_BN
+#define DQ_W8A8_BN 256  // widest tile the dispatcher may use (4096^3: 58.6 us at 256, 65.4 at 128)
+#endif
+#ifndef DQ_W8A8_STAGES_128
+#define DQ_W8A8_STAGES_128 3  // 96 KB of ring: two CTAs share an SM, one's epilogue overlapping the other's MMAs
+#endif
+#ifndef DQ_W8A8_STAGES_256
+#define DQ_W8A8_STAGES_256 2  // 96 KB of ring for 128 x 256 tiles: again two CTAs per SM
+#endif
+constexpr uint32_t kTileABytes = kBM * kBK;  // 16 KB
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 128;
-constexpr size_t kSmemBytes = 1024 + 2 * kStages * kTileBytes + 256 + kBN * 4;  // slack, ring, barriers, scales
+
+template <int BN, int STAGES>
+struct TileConfig {
+  static constexpr uint32_t kTileBBytes = BN * kBK;
+  static constexpr uint32_t kStageBytes = kTileABytes + kTileBBytes;
+  static constexpr uint32_t kTmemCols = BN;  // one int32 accumulator column per output column
+  // slack for 1024-byte alignment, ring, barriers, column scales
+  static constexpr size_t kSmemBytes = 1024 + STAGES * kStageBytes + 256 + BN * 4;
+  // kind::i8: int32 accumulator (format 2), signed A and B (format 1), both
+  // K-major, N / 8 and M / 16.
+  static constexpr uint32_t kIdesc =
+      (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+};
 
 struct W8A8Args {
   const int8_t* a;
@@ -83,16 +109,13 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(const void* tile) {
   return start | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-// Instruction descriptor of kind::i8: int32 accumulator (format 2), signed A
-// and B (format 1), both K-major, N / 8 and M / 16.
-constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
-
-__device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
-      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -124,14 +147,19 @@ __device__ __forceinline__ void tc_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) 
 
 // ---------------------------------------------------------------- kernels
 
+template <int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const W8A8Args a) {
+  using Cfg = TileConfig<BN, STAGES>;
+  constexpr int kStages = STAGES;
+  constexpr int kBN = BN;
+  constexpr uint32_t kTmemCols = Cfg::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sa = smem;
-  uint8_t* sb = smem + kStages * kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kStages * kTileBytes);
+  uint8_t* sa = smem;                             // kStages x 16 KB (A tiles)
+  uint8_t* sb = smem + kStages * kTileABytes;     // kStages x BN * 128 bytes (B tiles)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kStages * Cfg::kTileBBytes);
   uint64_t* empty = full + kStages;
   uint64_t* acc_ready = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 1);
@@ -141,7 +169,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   const int lane = threadIdx.x & 31;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
-  const int ktiles = static_cast<int>(a.k / kBK);
+  const int ktiles = static_cast<int>((a.k + kBK - 1) / kBK);  // the last slice is zero-filled past k
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -173,9 +201,9 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         const int s = kt % kStages;
         const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
         if (!dq::mbar_wait_parity(empty + s, ph ^ 1u)) break;
-        dq::mbar_arrive_expect_tx(full + s, 2 * kTileBytes);
-        tma_load_2d(sa + s * kTileBytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
-        tma_load_2d(sb + s * kTileBytes, &map_b, kt * kBK, static_cast<int>(n0), full + s);
+        dq::mbar_arrive_expect_tx(full + s, Cfg::kStageBytes);
+        tma_load_2d(sa + s * kTileABytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
+        tma_load_2d(sb + s * Cfg::kTileBBytes, &map_b, kt * kBK, static_cast<int>(n0), full + s);
       }
     }
   } else if (warp == 1) {
@@ -185,39 +213,43 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
         if (!dq::mbar_wait_parity(full + s, ph)) break;
         tc_fence_after();
-        const uint64_t ad = smem_desc_k_sw128(sa + s * kTileBytes);
-        const uint64_t bd = smem_desc_k_sw128(sb + s * kTileBytes);
+        const uint64_t ad = smem_desc_k_sw128(sa + s * kTileABytes);
+        const uint64_t bd = smem_desc_k_sw128(sb + s * Cfg::kTileBBytes);
 #pragma unroll
         for (int kk = 0; kk < kBK / 32; ++kk) {
           // +32 bytes along K = +2 in the descriptor's 16-byte address units
-          tc_mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, (kt | kk) != 0 ? 1u : 0u);
+          tc_mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, Cfg::kIdesc, (kt | kk) != 0 ? 1u : 0u);
         }
         tc_commit(empty + s);  // the stage is free once these MMAs have read it
       }
       tc_commit(acc_ready);  // every MMA issued above is complete when this arrives
     }
   } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
-    // the tile's column scales, staged once (128 threads, one each)
-    col_scale[threadIdx.x - 64] = a.b_scale[n0 + threadIdx.x - 64];
+    // the tile's column scales, staged once by the 128 epilogue threads
+#pragma unroll
+    for (int j = threadIdx.x - 64; j < kBN; j += 128) col_scale[j] = n0 + j < a.n ? a.b_scale[n0 + j] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");
     const bool ready = dq::mbar_wait_parity(acc_ready, 0);
     tc_fence_after();
     const int quarter = warp & 3;
     const int64_t row = m0 + 32 * quarter + lane;
-    const float sa_row = a.a_scale[row];
+    const bool row_ok = row < a.m;  // rows past m (zero-filled operands) are not stored
+    const float sa_row = row_ok ? a.a_scale[row] : 0.0f;
 #pragma unroll 1
     for (int c = 0; c < kBN / 32; ++c) {
+      const int64_t c0 = n0 + 32 * c;
+      if (c0 >= a.n) break;  // the same for every lane: the collective loads below stay warp-uniform
       uint32_t r[32];
       tc_ld_32cols(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * c), r);
-      if (!ready) continue;
+      if (!ready || !row_ok) continue;
       float t[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float scales = __fmul_rn(sa_row, col_scale[32 * c + j]);
         t[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
       }
-      const int64_t e0 = row * a.n + n0 + 32 * c;  // 32 consecutive outputs of this row
-      if (a.vec_out) {
+      const int64_t e0 = row * a.n + c0;  // 32 consecutive outputs of this row
+      if (a.vec_out && c0 + 32 <= a.n) {
         if (a.out_kind == 0) {
           float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + e0);
 #pragma unroll
@@ -250,7 +282,9 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) store_out(a, e0 + j, t[j]);
+        for (int j = 0; j < 32; ++j) {
+          if (c0 + j < a.n) store_out(a, e0 + j, t[j]);
+        }
       }
     }
   }
@@ -301,13 +335,13 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// [rows, k] int8, k contiguous: 128-byte x 128-row boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k) {
+// [rows, k] int8, k contiguous: 128-byte x box_rows boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k, uint32_t box_rows) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};  // bytes between rows
-  const cuuint32_t box[2] = {kBK, kBM};
+  const cuuint32_t box[2] = {kBK, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -335,6 +369,40 @@ dq_status launch_pdl(Kernel kernel, dim3 grid, int block, size_t smem, cudaStrea
   return cudaGetLastError() == cudaSuccess ? DQ_OK : DQ_ERR_CUDA;
 }
 
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return d;
+}
+
+constexpr dq_status kNotLaunchable = static_cast<dq_status>(-1);  // use the next path
+
+constexpr int kMaxDevices = 64;
+
+// Tensor-core launch of one tile configuration; kNotLaunchable when the
+// tensor maps or the shared-memory opt-in are unavailable.
+template <int BN, int STAGES>
+dq_status launch_tc(const W8A8Args& args, int device, cudaStream_t stream) {
+  using Cfg = TileConfig<BN, STAGES>;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, args.a, args.m, args.k, kBM) || !make_map(&mb, args.b, args.n, args.k, BN)) return kNotLaunchable;
+  // the opt-in above 48 KB of dynamic shared memory, once per device
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  if (device < 0 || device >= kMaxDevices) return kNotLaunchable;
+  std::call_once(once[device], [device] {
+    ok[device] = cudaFuncSetAttribute(w8a8_gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(Cfg::kSmemBytes)) == cudaSuccess;
+    if (!ok[device]) cudaGetLastError();
+  });
+  if (!ok[device]) return kNotLaunchable;
+  return launch_pdl(w8a8_gemm_tc_kernel<BN, STAGES>, dim3(static_cast<unsigned>((args.n + BN - 1) / BN),
+                    static_cast<unsigned>((args.m + kBM - 1) / kBM)), kThreads, Cfg::kSmemBytes, stream, ma, mb, args);
+}
+
 }  // namespace
 
 extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
@@ -350,25 +418,22 @@ extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, i
     return DQ_ERR_NULL_POINTER;
   const size_t os = out_dtype == DQ_F32 ? 4 : 2;
   if (!aligned_to(a_scale, 4) || !aligned_to(b_scale, 4) || !aligned_to(out, os)) return DQ_ERR_MISALIGNED;
+  // 16-byte stores need every row of out to start on a 16-byte boundary
+  const bool vec = aligned_to(out, 16) && (n * static_cast<int64_t>(os)) % 16 == 0;
   W8A8Args args{a, b, a_scale, b_scale, out, m, n, k, out_dtype == DQ_F32 ? 0 : (out_dtype == DQ_F16 ? 1 : 2),
-                accumulate, aligned_to(out, 16) ? 1 : 0};
-  const bool tiles = m % kBM == 0 && n % kBN == 0 && k % kBK == 0 && m / kBM <= 65535 &&
-                     aligned_to(a, 16) && aligned_to(b, 16);
+                accumulate, vec ? 1 : 0};
+  // tensor maps need 16-byte row pitches (k % 16 == 0) and bases; ragged m,
+  // n and k are zero-filled by the loads and masked in the epilogue
+  const bool tiles = k % 16 == 0 && (m + kBM - 1) / kBM <= 65535 && aligned_to(a, 16) && aligned_to(b, 16);
   if (tiles) {
-    CUtensorMap ma, mb;
-    if (make_map(&ma, a, m, k) && make_map(&mb, b, n, k)) {
-      static std::once_flag smem_once;
-      static bool smem_ok = false;
-      std::call_once(smem_once, [] {
-        smem_ok = cudaFuncSetAttribute(w8a8_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes)) == cudaSuccess;
-        if (!smem_ok) cudaGetLastError();
-      });
-      if (smem_ok) {
-        return launch_pdl(w8a8_gemm_tc_kernel, dim3(static_cast<unsigned>(n / kBN), static_cast<unsigned>(m / kBM)),
-                          kThreads, kSmemBytes, stream, ma, mb, args);
-      }
+    const int device = current_device();
+    // 256-wide tiles unless a 128-wide last tile would waste less
+    if (DQ_W8A8_BN >= 256 && (n % 256 == 0 || n % 256 > 128)) {
+      const dq_status st = launch_tc<256, DQ_W8A8_STAGES_256>(args, device, stream);
+      if (st != kNotLaunchable) return st;
     }
+    const dq_status st = launch_tc<128, DQ_W8A8_STAGES_128>(args, device, stream);
+    if (st != kNotLaunchable) return st;
   }
   const int64_t total = m * n;
   int64_t grid = (total + 255) / 256;

@@ -317,10 +317,19 @@ def w8a8_gemm(a, b, a_scale, b_scale, out_dtype=None, out=None, accumulate: bool
     Returns the [M, N] output (``out_dtype`` default float32).
     """
     torch = _torch()
+    if a.dim() != 2 or b.dim() != 2 or a.dtype != torch.int8 or b.dtype != torch.int8:
+        raise TypeError("a and b must be 2-D int8 tensors")
     m, k = (int(v) for v in a.shape)
     n = int(b.shape[0])
+    if int(b.shape[1]) != k:
+        raise ValueError(f"b must be [N, K] with the K of a ({k}), got {tuple(b.shape)}")
+    for name, t, length in (("a_scale", a_scale, m), ("b_scale", b_scale, n)):
+        if t.dtype != torch.float32 or t.numel() != length:
+            raise TypeError(f"{name} must be float32 with {length} elements")
     if out is None:
         out = torch.empty((m, n), dtype=out_dtype or torch.float32, device=a.device)
+    elif tuple(out.shape) != (m, n):
+        raise ValueError(f"out must be [{m}, {n}], got {tuple(out.shape)}")
     if stream is None:
         stream = torch.cuda.current_stream(a.device).cuda_stream
     st = dq_w8a8_gemm(_dev_ptr(a, "a"), _dev_ptr(b, "b"), m, n, k, _dev_ptr(a_scale, "a_scale"),
