@@ -714,7 +714,7 @@ def run_reference(args, world, rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "s8 x s8 -> s32, f32 scales" if wl.kind == "w8a8_gemm" else "f32",
         "data": "synthetic",
         "config": {"workload": args.workload, **workload_config(wl), "rows_per_step": n,
                    "rows_per_s": round(n * args.steps / elapsed, 1)},
