@@ -122,9 +122,6 @@ __device__ __noinline__ void ada_quantize_row_exact(const uint4* srow, const flo
 #define DQ_ADA_MAX_BLOCK 512
 #endif
 constexpr int kAdaMaxBlock = DQ_ADA_MAX_BLOCK;
-#ifndef DQ_ADA_ONEPASS
-#define DQ_ADA_ONEPASS 1  // both moments from one row reduction (see pass 1)
-#endif
 #ifndef DQ_ADA_MAX_REGS
 #define DQ_ADA_MAX_REGS 128  // the row share stays in registers across four passes
 #endif
@@ -215,7 +212,6 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const bool arrived = mbar_wait_parity(bars + c_stage, phase);
     const uint4* srow = reinterpret_cast<const uint4*>(ring + static_cast<size_t>(c_stage) * stride);
 
-#if DQ_ADA_ONEPASS
     // ---- pass 1: load, widen, shift by K, both moments of d = x - K
     // K is the mean of the row's first 8 elements, the same value in every
     // thread. E(d) and E(d^2) come out of one reduction; Var = E(d^2) - E(d)^2
@@ -340,90 +336,6 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
     const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
     // n = (x - mean_f) * rstd = fma(d, rstd, -(mean_f - K) * rstd)
     const float nb = -__fmul_rn(c_f, rstd);
-#else
-    // ---- pass 1: load, widen, E(x)
-    constexpr int NACC = VPT < 4 ? VPT : 4;  // independent accumulators: short dependency chains
-    float v[VPT][8];
-    float2 acc[NACC];
-#pragma unroll
-    for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      InTraits<InT>::widen8(in_row(k) ? srow[vbase + 32 * k] : make_uint4(0, 0, 0, 0), v[k]);  // zero when inactive
-      const float2 s01 = __fadd2_rn(make_float2(v[k][0], v[k][1]), make_float2(v[k][2], v[k][3]));
-      const float2 s23 = __fadd2_rn(make_float2(v[k][4], v[k][5]), make_float2(v[k][6], v[k][7]));
-      acc[k % NACC] = __fadd2_rn(acc[k % NACC], __fadd2_rn(s01, s23));
-    }
-#pragma unroll
-    for (int j = 1; j < NACC; ++j) acc[0] = __fadd2_rn(acc[0], acc[j]);
-    const float2 s1 = acc[0];
-    double sum = warp_sum(static_cast<double>(s1.x) + static_cast<double>(s1.y));
-    bool failed;
-    if (nwarps_g > 1) {
-      if (lane == 0) red_d[parity][0][warp] = sum;
-      failed = group_barrier_or(1 + g, tpr, !arrived);
-      sum = 0.0;
-      for (int w = 0; w < nwarps_g; ++w) sum += red_d[parity][0][warp_g0 + w];
-    } else {
-      failed = __any_sync(0xffffffffu, !arrived);
-      __syncwarp();
-    }
-    if (failed) {
-      for (int64_t rr = r + lane_g; rr < r_end; rr += tpr) a.quant_scale[rr] = __int_as_float(0x7fc00000);
-      if (leader) {
-        int st = c_stage;
-        uint32_t ph = phase;
-        for (int64_t j = r - r_begin + 1; j < issued; ++j) {
-          st = st + 1 == S ? 0 : st + 1;
-          if (st == 0) ph ^= 1u;
-          mbar_wait_parity(bars + st, ph);
-        }
-      }
-      return;
-    }
-    // refill the stage of the previous row (S - 1 copies stay in flight; the
-    // current row's stage is kept for the out-of-line exact path)
-    if (leader && issued < n) {
-      fence_proxy_async_smem();
-      issue_next();
-    }
-    c_stage = c_stage + 1 == S ? 0 : c_stage + 1;
-    if (c_stage == 0) phase ^= 1u;
-    const double mean_d = sum * a.inv_hidden;
-    const float mean_f = __double2float_rn(mean_d);
-
-    // ---- pass 2: Var(x), biased, about the double mean
-#pragma unroll
-    for (int j = 0; j < NACC; ++j) acc[j] = make_float2(0.0f, 0.0f);
-#pragma unroll
-    for (int k = 0; k < VPT; ++k) {
-      const bool active = in_row(k);
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float2 d = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-mean_f));
-        if (kRagged && !active) d = make_float2(0.0f, 0.0f);
-        v[k][2 * p] = d.x;
-        v[k][2 * p + 1] = d.y;
-        acc[(k + p) % NACC] = __ffma2_rn(d, d, acc[(k + p) % NACC]);
-      }
-    }
-#pragma unroll
-    for (int j = 1; j < NACC; ++j) acc[0] = __fadd2_rn(acc[0], acc[j]);
-    const float2 s2 = acc[0];
-    double sq = warp_sum(static_cast<double>(s2.x) + static_cast<double>(s2.y));
-    if (nwarps_g > 1) {
-      if (lane == 0) red_d[parity][1][warp] = sq;
-      group_barrier(1 + g, tpr);
-      sq = 0.0;
-      for (int w = 0; w < nwarps_g; ++w) sq += red_d[parity][1][warp_g0 + w];
-    }
-    const double dm = mean_d - static_cast<double>(mean_f);
-    double var_d = sq * a.inv_hidden - dm * dm;
-    var_d = var_d > 0.0 ? var_d : 0.0;
-    const float var_f = __double2float_rn(var_d);
-    const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(var_f, a.epsilon)));
-
-#endif
     // ---- pass 3: y = n * A + B, absmax
     float amx[NACC];
 #pragma unroll
@@ -437,11 +349,7 @@ ada_layernorm_quant_tma_kernel(const AdaArgs a) {
         const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-#if DQ_ADA_ONEPASS
           const float2 nn = __ffma2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd), f2(nb));
-#else
-          const float2 nn = __fmul2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd));
-#endif
           const float2 y =
               __ffma2_rn(nn, make_float2(Av[2 * p], Av[2 * p + 1]), make_float2(Bv[2 * p], Bv[2 * p + 1]));
           v[k][2 * p] = y.x;
