@@ -1,10 +1,12 @@
 """Multi-rank host logic on CPU (gloo, world size 2).
 
 The quantization path shards by rows with no data exchange (rows are
-independent; the MoE group index is rebased per shard). These tests run two
-gloo ranks that each quantize their shard with the CPU oracle and gather the
-results, and check the concatenation against one unsharded run; and they run
-the benchmark's reference arm under torchrun with two ranks.
+independent; the MoE group index is rebased per shard), and so does the W8A8
+product that consumes the codes (weights replicated). These tests run two
+gloo ranks that each quantize their shard with the CPU oracle, multiply it by
+the weights and gather the results, and check the concatenations against one
+unsharded run; and they run the benchmark's reference arm under torchrun with
+two ranks.
 """
 
 import json
@@ -57,11 +59,22 @@ def _worker(rank, world, port, out_path):
         ss = [torch.zeros_like(sp) for _ in range(world)]
         dist.all_gather(ys, yp)
         dist.all_gather(ss, sp)
+        # the consumer shards the same way: each rank multiplies its own codes
+        # (per-token scales) by the replicated int8 weights
+        w = workloads.uniform((40, cols), torch.float32, 8, -127.0, 127.0).round().to(torch.int8).numpy()
+        ws = workloads.uniform((40,), torch.float32, 9, 0.001, 0.02).numpy()
+        pp = torch.zeros(cap, 40, dtype=torch.float32)
+        pp[: end - start] = torch.from_numpy(oracle.w8a8_gemm(y, w, s, ws, out_dtype="f32"))
+        ps = [torch.zeros_like(pp) for _ in range(world)]
+        dist.all_gather(ps, pp)
         if rank == 0:
             y_all = torch.cat([ys[i][: sizes[i].item()] for i in range(world)]).numpy()
             s_all = torch.cat([ss[i][: sizes[i].item()] for i in range(world)]).numpy()
+            p_all = torch.cat([ps[i][: sizes[i].item()] for i in range(world)]).numpy()
             y_ref, s_ref, _ = oracle.dynamic_quant(x, smooth=smooth, group_index=gi)
-            ok = bool(np.array_equal(y_all, y_ref) and np.array_equal(s_all.view(np.uint32), s_ref.view(np.uint32)))
+            p_ref = oracle.w8a8_gemm(y_ref, w, s_ref, ws, out_dtype="f32")
+            ok = bool(np.array_equal(y_all, y_ref) and np.array_equal(s_all.view(np.uint32), s_ref.view(np.uint32))
+                      and np.array_equal(p_all.view(np.uint32), p_ref.view(np.uint32)))
             with open(out_path, "w") as f:
                 f.write("ok" if ok else "mismatch")
     finally:
