@@ -269,3 +269,43 @@ def test_w8a8_helper_checks_shapes_on_the_host(dq_lib):
         dq_lib.w8a8_gemm(a, torch.zeros(8, 32, dtype=torch.int8), torch.ones(3), torch.ones(8))
     with pytest.raises(TypeError):
         dq_lib.w8a8_gemm(a.float(), torch.zeros(8, 32, dtype=torch.int8), torch.ones(4), torch.ones(8))
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "dq.h"
+
+int main(void) {
+  size_t bytes = 123;
+  /* host-only calls: argument validation and the workspace query */
+  if (dq_get_workspace_size(32768, 7168, DQ_BF16, DQ_SYMMETRIC, DQ_INT8, 64, &bytes) != DQ_OK || bytes != 4) return 1;
+  if (dq_get_workspace_size(4, 7, DQ_F16, DQ_SYMMETRIC, DQ_INT4X2, 0, &bytes) != DQ_ERR_BAD_SHAPE) return 2;
+  if (dq_w8a8_gemm(NULL, NULL, 0, 16, 32, NULL, NULL, NULL, DQ_BF16, 0, 0) != DQ_OK) return 3;
+  if (dq_w8a8_gemm(NULL, NULL, 16, 16, 32, NULL, NULL, NULL, DQ_BF16, 0, 0) != DQ_ERR_NULL_POINTER) return 4;
+  printf("%s|%s\n", dq_status_string(DQ_OK), dq_status_string(DQ_ERR_MISALIGNED));
+  return 0;
+}
+"""
+
+
+def test_plain_c_program_uses_the_header_and_library(dq_lib, tmp_path):
+    """include/dq.h is plain C (no C++ types in the signatures): a C program
+    compiles against it with gcc, links libdq.so and runs its host-side calls
+    (no device needed)."""
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no gcc")
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(dq_lib.LIBRARY_PATH)
+    build = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc,
+                            str(src), "-L", lib_dir, "-l:libdq.so", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                           capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    ok, mis = run.stdout.strip().split("|")
+    assert ok == dq_lib.dq_status_string(dq_lib.DQ_OK)
+    assert mis == dq_lib.dq_status_string(dq_lib.DQ_ERR_MISALIGNED)
