@@ -86,7 +86,7 @@ def test_extreme_codes_large_k(dq):
 
 
 RAGGED_TC_SHAPES = [(130, 128, 128), (128, 128, 96), (64, 200, 256), (1, 256, 16), (200, 300, 272),
-                    (77, 520, 1040), (129, 385, 4112), (300, 640, 128)]
+                    (77, 520, 1040), (129, 385, 4112), (300, 640, 128), (5, 7, 48)]
 
 
 @pytest.mark.parametrize("shape", RAGGED_TC_SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in RAGGED_TC_SHAPES])
