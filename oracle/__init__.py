@@ -209,6 +209,11 @@ def ada_layernorm_quant(x, ada_scale, ada_shift, weight=None, bias=None, smooth=
     return out, qs
 
 
+def _need_entries(buf, n: int, what: str):
+    if buf is not None and np.asarray(buf).size != n:
+        raise ValueError(f"oracle: {what} must have {n} entries, got {np.asarray(buf).size}")
+
+
 def dequant_per_token(codes, scale, offset=None, y_dtype: str = "int8", cols: int | None = None,
                       out_dtype: str = "f32", scale_dtype: str | None = None):
     """Per-token dequantization (AntiQuantize, PER_TOKEN policy), read as the
@@ -232,6 +237,9 @@ def dequant_per_token(codes, scale, offset=None, y_dtype: str = "int8", cols: in
         ob, oc = _float_buffer(offset, scale_dtype)
         if oc != sc:
             raise TypeError("oracle: offset must have the dtype of scale")
+    _need_entries(sb, rows, "scale")
+    if ob is not None:
+        _need_entries(ob, rows, "offset")
     oc_out = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
     out = np.zeros((rows, cols), dtype=np.float32 if oc_out == F32 else np.uint16)
     _check(lib.oracle_dequant_per_token(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, oc_out, _ptr(out)))
@@ -256,6 +264,12 @@ def dequant_per_group(codes, scale, offset=None, group_size: int = 32, k_dim: in
         ob, oc = _float_buffer(offset, scale_dtype)
         if oc != sc:
             raise TypeError("oracle: offset must have the dtype of scale")
+    if int(group_size) > 0 and int(group_size) % 32 == 0 and int(k_dim) in (0, 1):  # else the oracle rejects it
+        g = int(group_size)
+        entries = rows * -(-cols // g) if int(k_dim) == 1 else -(-rows // g) * cols
+        _need_entries(sb, entries, "scale")
+        if ob is not None:
+            _need_entries(ob, entries, "offset")
     oc_out = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
     out = np.zeros((rows, cols), dtype=np.float32 if oc_out == F32 else np.uint16)
     _check(lib.oracle_dequant_per_group(_ptr(cb), yc, rows, cols, _ptr(sb), _ptr(ob), sc, int(group_size),
@@ -274,13 +288,17 @@ def w8a8_gemm(a, b, a_scale, b_scale, out_dtype: str = "f32", accumulate_into=No
     n = bb.shape[0]
     if bb.shape[1] != k:
         raise ValueError("oracle.w8a8_gemm: K mismatch")
-    sa = np.ascontiguousarray(a_scale, dtype=np.float32)
-    sb = np.ascontiguousarray(b_scale, dtype=np.float32)
+    sa = np.ascontiguousarray(a_scale, dtype=np.float32).reshape(-1)
+    sb = np.ascontiguousarray(b_scale, dtype=np.float32).reshape(-1)
+    if sa.size != m or sb.size != n:
+        raise ValueError(f"oracle.w8a8_gemm: scales must have {m} and {n} entries, got {sa.size} and {sb.size}")
     oc = {"f32": F32, "f16": F16, "bf16": BF16}[out_dtype]
     if accumulate_into is not None:
         if oc != F32:
             raise ValueError("accumulation needs float32 output")
         out = np.array(accumulate_into, dtype=np.float32, copy=True)
+        if out.shape != (m, n):
+            raise ValueError(f"oracle.w8a8_gemm: accumulate_into must be [{m}, {n}]")
     else:
         out = np.zeros((m, n), dtype=np.float32 if oc == F32 else np.uint16)
     _check(lib.oracle_w8a8_gemm(_ptr(ab), _ptr(bb), m, n, k, _ptr(sa), _ptr(sb), oc,

@@ -750,3 +750,32 @@ def test_w8a8_accumulate_and_narrow(oracle_mod):
     np.testing.assert_array_equal(oracle_mod.w8a8_gemm(a, b, sa, sb, out_dtype="f16"), base.astype(np.float16))
     bf = oracle_mod.w8a8_gemm(a, b, sa, sb, out_dtype="bf16")
     np.testing.assert_array_equal(bf, torch.from_numpy(base).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+# ---------------------------------------------------------------- W8A8 golden records
+
+def _load_w8a8_golden():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "quant_matmul_w8a8.txt")
+    recs = []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        a, b, sa, sb, y, out_dtype, want = (f.strip() for f in line.split("|"))
+        rows = lambda t, conv=float: [[conv(v) for v in r.split()] for r in t.split(";")]
+        recs.append(dict(a=np.array(rows(a, int), np.int8), b=np.array(rows(b, int), np.int8),
+                         sa=np.array(sa.split(), np.float32), sb=np.array(sb.split(), np.float32),
+                         y=None if y == "-" else np.array(rows(y), np.float32), out_dtype=out_dtype,
+                         want=np.array(rows(want), np.float64)))
+    return recs
+
+
+@pytest.mark.parametrize("rec", _load_w8a8_golden(), ids=lambda r: f"{r['a'].shape}x{r['b'].shape[0]}-{r['out_dtype']}")
+def test_w8a8_golden_records(oracle_mod, rec):
+    got = oracle_mod.w8a8_gemm(rec["a"], rec["b"], rec["sa"], rec["sb"], out_dtype=rec["out_dtype"],
+                               accumulate_into=None if rec["y"] is None else rec["y"].copy())
+    if rec["out_dtype"] == "f16":
+        got = got.view(np.float16).astype(np.float64)
+    else:
+        got = _as_float64(got, rec["out_dtype"])
+    np.testing.assert_array_equal(got, rec["want"])
