@@ -27,7 +27,10 @@
 // overlaps the other's main loop. The 256-wide tile reads 48 KB of operands
 // per 2^22 multiply-adds instead of 64 KB: on 4096^3, 58.6 us against 65.4.
 // Every mbarrier wait is bounded; the MMA lane always issues the final
-// commit, so teardown never frees TMEM under MMAs in flight.
+// commit, so teardown never frees TMEM under MMAs in flight. A tile whose
+// sum is incomplete (the epilogue's wait ran out, or the MMA lane gave up on
+// a stage and flagged it) is written as NaN, and the producer waits
+// (bounded) for its copies in flight before the CTA exits.
 // K not a multiple of 16, or unaligned operands: a CUDA-core kernel with the
 // same arithmetic.
 
@@ -83,6 +86,16 @@ struct W8A8Args {
   int accumulate;  // out (f32) += product
   int vec_out;     // out is 16-byte aligned: whole-row-chunk vector stores
 };
+
+// Quiet NaN in the output type: the mark of a tile whose accumulator never
+// became ready (a bounded wait ran out).
+__device__ __forceinline__ void store_nan(const W8A8Args& a, int64_t e) {
+  if (a.out_kind == 0) {
+    static_cast<float*>(a.out)[e] = __int_as_float(0x7fc00000);
+  } else {
+    static_cast<uint16_t*>(a.out)[e] = a.out_kind == 1 ? uint16_t(0x7e00) : uint16_t(0x7fc0);
+  }
+}
 
 __device__ __forceinline__ void store_out(const W8A8Args& a, int64_t e, float t) {
   if (a.out_kind == 0) {
@@ -163,6 +176,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   uint64_t* empty = full + kStages;
   uint64_t* acc_ready = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 1);
+  volatile uint32_t* mma_failed = tmem_slot + 1;  // set when the MMA lane gave up on a stage
   float* col_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // the tile's b_scale
 
   const int warp = threadIdx.x >> 5;
@@ -177,6 +191,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       dq::mbar_init(empty + s, 1);
     }
     dq::mbar_init(acc_ready, 1);
+    *mma_failed = 0u;
     dq::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -197,7 +212,8 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
 
   if (warp == 0) {
     if (lane == 0) {  // producer
-      for (int kt = 0; kt < ktiles; ++kt) {
+      int issued = 0;
+      for (int kt = 0; kt < ktiles; ++kt, ++issued) {
         const int s = kt % kStages;
         const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
         if (!dq::mbar_wait_parity(empty + s, ph ^ 1u)) break;
@@ -205,13 +221,24 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         tma_load_2d(sa + s * kTileABytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
         tma_load_2d(sb + s * Cfg::kTileBBytes, &map_b, kt * kBK, static_cast<int>(n0), full + s);
       }
+      // no copy may still be landing in this CTA's shared memory when it
+      // exits: wait (bounded) for the last copy of every stage. Normally they
+      // have long landed; after a timed-out wait elsewhere this drains them.
+      for (int kt = issued > kStages ? issued - kStages : 0; kt < issued; ++kt) {
+        dq::mbar_wait_parity(full + kt % kStages, static_cast<uint32_t>(kt / kStages) & 1u);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {  // MMA issuer
       for (int kt = 0; kt < ktiles; ++kt) {
         const int s = kt % kStages;
         const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
-        if (!dq::mbar_wait_parity(full + s, ph)) break;
+        if (!dq::mbar_wait_parity(full + s, ph)) {
+          // the sum will miss this stage: tell the epilogue before the commit
+          *mma_failed = 1u;
+          __threadfence_block();
+          break;
+        }
         tc_fence_after();
         const uint64_t ad = smem_desc_k_sw128(sa + s * kTileABytes);
         const uint64_t bd = smem_desc_k_sw128(sb + s * Cfg::kTileBBytes);
@@ -229,7 +256,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
 #pragma unroll
     for (int j = threadIdx.x - 64; j < kBN; j += 128) col_scale[j] = n0 + j < a.n ? a.b_scale[n0 + j] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool ready = dq::mbar_wait_parity(acc_ready, 0);
+    const bool ready = dq::mbar_wait_parity(acc_ready, 0) && *mma_failed == 0u;
     tc_fence_after();
     const int quarter = warp & 3;
     const int64_t row = m0 + 32 * quarter + lane;
@@ -241,7 +268,13 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
       if (c0 >= a.n) break;  // the same for every lane: the collective loads below stay warp-uniform
       uint32_t r[32];
       tc_ld_32cols(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(32 * c), r);
-      if (!ready || !row_ok) continue;
+      if (!row_ok) continue;
+      if (!ready) {  // the accumulator never became ready: NaN marks the tile
+        for (int j = 0; j < 32; ++j) {
+          if (c0 + j < a.n) store_nan(a, row * a.n + c0 + j);
+        }
+        continue;
+      }
       float t[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
