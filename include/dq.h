@@ -69,7 +69,7 @@ typedef enum dq_status {
   DQ_ERR_NULL_POINTER = 1,        /* a required pointer is NULL */
   DQ_ERR_BAD_SHAPE = 2,           /* negative/zero sizes, odd cols for INT4, ... */
   DQ_ERR_BAD_DTYPE = 3,           /* dtype not allowed in that argument */
-  DQ_ERR_UNSUPPORTED = 4,         /* valid request this build does not implement */
+  DQ_ERR_UNSUPPORTED = 4,         /* valid request this library does not implement */
   DQ_ERR_MISALIGNED = 5,          /* pointer below its element's natural alignment */
   DQ_ERR_WORKSPACE_TOO_SMALL = 6, /* workspace missing or smaller than queried */
   DQ_ERR_CUDA = 7,                /* the CUDA launch failed (cudaGetLastError) */

@@ -491,7 +491,7 @@ const char* dq_status_string(dq_status s) {
     case DQ_ERR_NULL_POINTER: return "DQ_ERR_NULL_POINTER: a required pointer is NULL";
     case DQ_ERR_BAD_SHAPE: return "DQ_ERR_BAD_SHAPE: invalid sizes for this call";
     case DQ_ERR_BAD_DTYPE: return "DQ_ERR_BAD_DTYPE: element type not allowed for this argument";
-    case DQ_ERR_UNSUPPORTED: return "DQ_ERR_UNSUPPORTED: request not implemented by this build";
+    case DQ_ERR_UNSUPPORTED: return "DQ_ERR_UNSUPPORTED: request not implemented by this library";
     case DQ_ERR_MISALIGNED: return "DQ_ERR_MISALIGNED: pointer below its element alignment";
     case DQ_ERR_WORKSPACE_TOO_SMALL: return "DQ_ERR_WORKSPACE_TOO_SMALL: workspace missing or too small";
     case DQ_ERR_CUDA: return "DQ_ERR_CUDA: the kernel launch failed";
