@@ -282,7 +282,8 @@ dq_status dq_dequant_per_group(const void* y, dq_dtype y_dtype, int64_t rows, in
  *   a_scale  device float [m]; b_scale device float [n].
  *   out      device [m, n] of out_dtype (DQ_F32, DQ_F16, DQ_BF16);
  *            accumulate = 1 adds into it (DQ_F32 only), 0 overwrites.
- * k <= 2^17 (int32 sums cannot overflow). With k a multiple of 16 and
+ * k < 2^17 (|sum| <= k * 128 * 128 < 2^31: int32 sums cannot overflow, even
+ * with every code at -128). With k a multiple of 16 and
  * 16-byte aligned a and b, any m and n run on tcgen05 tensor cores
  * (128 x 256 or 128 x 128 tiles, ragged edges zero-filled and masked); other
  * shapes run a CUDA-core kernel with the same results.
@@ -296,25 +297,29 @@ dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, i
  * fixed table holds this many 8-byte entries: 1 MiB per device). */
 #define DQ_ADA_NOALLOC_MAX_TABLE 131072
 
-/* dq_ada_layernorm_quant without a workspace argument: the same computation,
- * results and errors, with the scratch table kept in a fixed device array
- * inside the library. The pages have no counterpart to this entry point (their
- * two-phase calls always take a workspace); it exists for callers that cannot
- * allocate device memory: a plain C host program that links only this
- * library, or code that runs where allocating would re-enter the caller's own
- * allocator (for example an out-of-memory handler).
+/* dq_ada_layernorm_quant without a workspace argument: the same computation
+ * and results, with the scratch table kept in a fixed device array inside the
+ * library. The pages have no counterpart to this entry point (their two-phase
+ * calls always take a workspace); it exists for callers that cannot allocate
+ * device memory: a plain C host program that links only this library, or code
+ * that runs where allocating would re-enter the caller's own allocator (for
+ * example an out-of-memory handler).
  *   - Allocates nothing: no cudaMalloc/cudaFree, no library allocation.
- *   - batch * hidden <= DQ_ADA_NOALLOC_MAX_TABLE, else DQ_ERR_UNSUPPORTED and
- *     nothing is launched.
+ *   - Checks in dq_ada_layernorm_quant's order (shapes and dtypes, epsilon,
+ *     batch * seq == 0 returns DQ_OK, required pointers), then
+ *     batch * hidden <= DQ_ADA_NOALLOC_MAX_TABLE, else DQ_ERR_UNSUPPORTED
+ *     (where dq_ada_layernorm_quant checks its workspace); nothing is
+ *     launched on an error.
  *   - The first call on each device (with that device current) looks up the
- *     array's address with cudaGetSymbolAddress and caches it; make that first
- *     call before any stream capture. A failed lookup returns DQ_ERR_CUDA.
+ *     array's address with cudaGetSymbolAddress and caches it with the
+ *     identity of the device's context; the first call after a device reset
+ *     (cudaDeviceReset) looks it up again. Make such a call before any stream
+ *     capture. A failed lookup returns DQ_ERR_CUDA.
  *   - Nothing needs clearing beforehand: each call writes every table entry it
  *     reads.
  *   - The array is shared by all calls on a device: calls whose executions
  *     overlap (other streams, other host threads) race on it and must use
- *     dq_ada_layernorm_quant with separate workspaces instead.
- * batch * seq == 0 returns DQ_OK without any CUDA call. */
+ *     dq_ada_layernorm_quant with separate workspaces instead. */
 dq_status dq_ada_layernorm_quant_noalloc(const void* x, dq_dtype x_dtype,
                                          int64_t batch, int64_t seq, int64_t hidden,
                                          const void* ada_scale, const void* ada_shift,

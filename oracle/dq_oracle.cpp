@@ -473,7 +473,7 @@ int oracle_dequant_per_group(const void* y, int y_dtype, int64_t rows, int64_t c
 int oracle_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
                      const float* a_scale, const float* b_scale, int out_dtype, int accumulate, void* out) {
   if (m < 0 || n < 0 || k < 1) return ORACLE_ERR_SHAPE;
-  if (k > (int64_t(1) << 17)) return ORACLE_ERR_SHAPE;  // |acc| < 2^31 for any int8 codes
+  if (k >= (int64_t(1) << 17)) return ORACLE_ERR_SHAPE;  // |acc| <= k * 2^14 < 2^31 for any int8 codes
   if (!is_float_dtype(out_dtype)) return ORACLE_ERR_DTYPE;
   if (accumulate && out_dtype != ORACLE_F32) return ORACLE_ERR_ARGUMENT;
   if (m > 0 && n > 0 && (a == nullptr || b == nullptr || a_scale == nullptr || b_scale == nullptr || out == nullptr))

@@ -169,6 +169,36 @@ def test_ada_layernorm_quant_validation(dq_lib):
         assert _ada(d, **kw) == want, kw
 
 
+def _ada_noalloc(d, **kw):
+    args = dict(x=FAKE, x_dtype=d.DQ_BF16, batch=2, seq=8, hidden=64, ada_scale=FAKE, ada_shift=FAKE, weight=None,
+                bias=None, smooth=None, param_dtype=d.DQ_BF16, epsilon=1e-6, out=FAKE, quant_scale=FAKE,
+                stream=None)
+    args.update(kw)
+    return d.dq_ada_layernorm_quant_noalloc(**args)
+
+
+def test_noalloc_checks_follow_the_regular_order(dq_lib):
+    """The no-allocation AdaLN entry point validates in the regular entry
+    point's order (shapes, epsilon, empty input, pointers), with its array's
+    size limit where the regular one checks the workspace; every case here is
+    rejected (or empty) on the host, before any CUDA call."""
+    d = dq_lib
+    too_big = dict(batch=33, seq=1, hidden=4096)  # 33 * 4096 > DQ_ADA_NOALLOC_MAX_TABLE
+    cases = [
+        (dict(batch=0, epsilon=float("nan")), d.DQ_ERR_BAD_ARGUMENT, d.DQ_ERR_BAD_ARGUMENT),
+        (dict(seq=0, epsilon=-1.0), d.DQ_ERR_BAD_ARGUMENT, d.DQ_ERR_BAD_ARGUMENT),
+        (dict(batch=0, x=None, out=None), d.DQ_OK, d.DQ_OK),
+        (dict(hidden=0, epsilon=float("nan")), d.DQ_ERR_BAD_SHAPE, d.DQ_ERR_BAD_SHAPE),
+        (dict(too_big, x=None), d.DQ_ERR_NULL_POINTER, d.DQ_ERR_NULL_POINTER),
+        (dict(too_big, quant_scale=None), d.DQ_ERR_NULL_POINTER, d.DQ_ERR_NULL_POINTER),
+        (dict(too_big, epsilon=float("inf")), d.DQ_ERR_BAD_ARGUMENT, d.DQ_ERR_BAD_ARGUMENT),
+        (dict(too_big), d.DQ_ERR_UNSUPPORTED, d.DQ_ERR_WORKSPACE_TOO_SMALL),
+    ]
+    for kw, want_noalloc, want_regular in cases:
+        assert _ada_noalloc(d, **kw) == want_noalloc, kw
+        assert _ada(d, **dict(kw, workspace=None, workspace_bytes=0)) == want_regular, kw
+
+
 def _deq(d, **kw):
     args = dict(y=FAKE, y_dtype=d.DQ_INT8, rows=4, cols=64, scale=FAKE, offset=None, scale_dtype=d.DQ_F32,
                 out=FAKE, out_dtype=d.DQ_BF16, stream=None)
@@ -245,6 +275,7 @@ def test_w8a8_gemm_validation(dq_lib):
     cases = [
         (dict(k=0), d.DQ_ERR_BAD_SHAPE),
         (dict(k=(1 << 17) + 16), d.DQ_ERR_BAD_SHAPE),  # int32 sums could overflow
+        (dict(k=1 << 17), d.DQ_ERR_BAD_SHAPE),  # all codes -128: the sum 2^31 does not fit int32
         (dict(m=-1), d.DQ_ERR_BAD_SHAPE),
         (dict(out_dtype=d.DQ_INT8), d.DQ_ERR_BAD_DTYPE),
         (dict(accumulate=2), d.DQ_ERR_BAD_ARGUMENT),

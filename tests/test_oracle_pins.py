@@ -719,6 +719,19 @@ def test_w8a8_operand_roles_transpose(oracle_mod):
     np.testing.assert_array_equal(x, y.T)
 
 
+def test_w8a8_largest_k_fits_int32_and_2_pow_17_is_rejected(oracle_mod):
+    """|sum| <= k * 128 * 128, so k < 2^17 keeps every int32 sum exact: at the
+    largest accepted multiple of 16, all codes -128 give 2^31 - 2^18 (exact in
+    binary32); at k = 2^17 that sum would be 2^31, one past INT32_MAX."""
+    k = (1 << 17) - 16
+    a = np.full((1, k), -128, dtype=np.int8)
+    out = oracle_mod.w8a8_gemm(a, a, np.ones(1, np.float32), np.ones(1, np.float32), out_dtype="f32")
+    assert out[0, 0] == float(k * 128 * 128) == 2.0 ** 31 - 2.0 ** 18
+    big = np.full((1, 1 << 17), -128, dtype=np.int8)
+    with pytest.raises(Exception):
+        oracle_mod.w8a8_gemm(big, big, np.ones(1, np.float32), np.ones(1, np.float32), out_dtype="f32")
+
+
 def test_w8a8_scale_product_is_taken_first(oracle_mod):
     """The formula multiplies the sum by (scale1 * scale2): rounded products in
     that order. Cases where (acc * s1) * s2 would round differently pin it."""

@@ -9,6 +9,7 @@ denormals for results identical to the formulas' binary32 evaluation.
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -46,24 +47,45 @@ def is_stale() -> bool:
     return any(os.path.getmtime(p) > t for p in _inputs() + [os.path.abspath(__file__)])
 
 
+def _run(cmd: list[str]) -> subprocess.CompletedProcess:
+    return subprocess.run(cmd, capture_output=True, text=True)
+
+
 def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
-    """Compile every .cu under csrc/ into one shared library (static cudart)."""
+    """Compile every .cu under csrc/ (one object each, in parallel) and link
+    them into one shared library with a static CUDA runtime."""
     if not force and not is_stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [
-        _nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17",
-        "-Xcompiler", "-fPIC,-O2", "-shared", "--cudart", "static",
-        "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources(),
-    ]
+    nvcc = _nvcc()
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    common = [*ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC]
     if ptxas_verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError(f"nvcc failed ({res.returncode}) building {LIB}")
+        common.insert(0, "-Xptxas=-v")
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.splitext(os.path.basename(src))[0] + f".{os.getpid()}.o")
+        jobs.append((obj, [nvcc, *common, "-c", src, "-o", obj]))
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+        results = list(pool.map(lambda j: _run(j[1]), jobs))
+    log = "".join(r.stdout + r.stderr for r in results)
+    failed = [j[1][-3] for j, r in zip(jobs, results) if r.returncode != 0]
+    if failed:
+        sys.stderr.write(log)
+        raise RuntimeError(f"nvcc failed compiling {', '.join(os.path.basename(f) for f in failed)}")
+    tmp = LIB + f".tmp{os.getpid()}"
+    link = _run([nvcc, *ARCH_FLAGS, "-shared", "--cudart", "static", "-o", tmp, *(j[0] for j in jobs)])
+    for obj, _ in jobs:
+        try:
+            os.remove(obj)
+        except OSError:
+            pass
+    if link.returncode != 0:
+        sys.stderr.write(log + link.stdout + link.stderr)
+        raise RuntimeError(f"nvcc failed linking {LIB}")
     if not quiet or ptxas_verbose:
-        sys.stderr.write(res.stdout + res.stderr)
+        sys.stderr.write(log + link.stdout + link.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -37,35 +37,15 @@
 //   * steps 4-5 are the DynamicQuant quantizer (exact IEEE semantics).
 #pragma once
 
+#include "dq_args.cuh"
 #include "dq_device.cuh"
 #include "tma_pipeline.cuh"
 
 namespace dq {
 
-struct AdaArgs {
-  const void* x;
-  int64_t batch, seq, hidden;
-  const void* ada_scale;  // [batch, hidden]
-  const void* ada_shift;  // [batch, hidden]
-  const void* weight;     // [hidden] or nullptr
-  const void* bias;       // [hidden] or nullptr
-  const void* smooth;     // [hidden] or nullptr
-  int param_dtype;
-  float epsilon;
-  double inv_hidden;      // 1 / hidden, rounded once in double
-  float* table;           // workspace: A [batch][hidden], then B [batch][hidden]
-  int8_t* out;
-  float* quant_scale;
-  int tpr;
-  int groups;
-  int stages;
-  uint32_t stage_stride;
-};
-
 __host__ __device__ inline size_t ada_smem_bytes(int groups, int stages, uint32_t stride) {
   return static_cast<size_t>(groups) * stages * stride + static_cast<size_t>(groups) * stages * 8;
 }
-
 
 // ============================================================ affine table
 

@@ -24,27 +24,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "dq_args.cuh"
 #include "dq_device.cuh"
 
 namespace dq {
-
-struct DequantArgs {
-  const void* y;       // codes
-  int64_t rows, cols;
-  const void* scale;   // scale table of scale_dtype (layout below)
-  const void* offset;  // table of the same shape and dtype, or nullptr
-  int scale_dtype;     // kF32 / kF16 / kBF16
-  void* out;           // [rows, cols] of the output type
-  int64_t group_size;  // group layouts only
-  int64_t table_cols;  // row length of the scale table
-};
-
-enum : int { kOutF32 = 0, kOutF16 = 1, kOutBF16 = 2 };
-
-// Scale-table layouts (AntiQuantize policies): PER_TOKEN [rows]; PER_GROUP
-// with k along a row (kDim 1) [rows, ceil(cols/g)], entry (i, j / g); PER_GROUP
-// with k down a column (kDim 0) [ceil(rows/g), cols], entry (i / g, j).
-enum : int { kPerToken = 0, kGroupAlongRow = 1, kGroupDownColumn = 2 };
 
 // Output element storage and pair narrowing (round to nearest even).
 template <int OUT>

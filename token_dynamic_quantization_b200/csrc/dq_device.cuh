@@ -19,10 +19,9 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
-namespace dq {
+#include "dq_args.cuh"
 
-// Element type tags (mirror the dq_dtype values of the C ABI).
-enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
+namespace dq {
 
 // Compile-time flag carried through generic lambdas.
 template <bool B>

@@ -12,8 +12,12 @@
 // through CUDA nor through any library.
 //
 // Set-up: the array's device address is looked up with cudaGetSymbolAddress
-// once per device, on the first call made while that device is current, and
-// cached. Every other call only reads the cache.
+// on the first call made while a device is current, and cached together with
+// the identity of that device's current context. A later call that finds a
+// different context (the device was reset with cudaDeviceReset, which
+// reloads the library's device code) repeats the look-up; every other call
+// only reads the cache. A call that does the look-up should come before any
+// stream capture.
 //
 // Nothing in the array has to start at zero: every call writes each table
 // entry it reads (the table kernel runs first on the same stream and the row
@@ -22,10 +26,11 @@
 // threads) race on it; such callers use the regular entry point with
 // separate workspaces.
 
-#include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "dq.h"
@@ -37,10 +42,44 @@ namespace {
 static __device__ __align__(256) float2 g_ada_noalloc_table[DQ_ADA_NOALLOC_MAX_TABLE];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_table_addr[kMaxDevices];
+
+struct Cached {
+  void* addr;
+  unsigned long long ctx_id;  // 0: not set up
+};
+Cached g_table[kMaxDevices];
 std::mutex g_setup_mutex;
 
-// Device address of this device's table (set up on first use).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (never 0), or 0 when the
+// driver cannot report one; then the cached address is kept as it is.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    cudaGetLastError();
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id + 1;  // keep 0 for "unknown"
+}
+
+// Device address of this device's table (set up on first use, and again
+// after the device's context has changed).
 dq_status noalloc_table(void** addr) {
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) {
@@ -48,19 +87,19 @@ dq_status noalloc_table(void** addr) {
     return DQ_ERR_CUDA;
   }
   if (device < 0 || device >= kMaxDevices) return DQ_ERR_UNSUPPORTED;
-  void* p = g_table_addr[device].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    p = g_table_addr[device].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      if (cudaGetSymbolAddress(&p, g_ada_noalloc_table) != cudaSuccess || p == nullptr) {
-        cudaGetLastError();
-        return DQ_ERR_CUDA;
-      }
-      g_table_addr[device].store(p, std::memory_order_release);
+  const unsigned long long ctx = current_context_id();
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  Cached& c = g_table[device];
+  if (c.addr == nullptr || (ctx != 0 && c.ctx_id != ctx)) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ada_noalloc_table) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return DQ_ERR_CUDA;
     }
+    c.addr = p;
+    c.ctx_id = ctx;
   }
-  *addr = p;
+  *addr = c.addr;
   return DQ_OK;
 }
 
@@ -71,10 +110,15 @@ extern "C" dq_status dq_ada_layernorm_quant_noalloc(const void* x, dq_dtype x_dt
                                                     const void* weight, const void* bias, const void* smooth,
                                                     dq_dtype param_dtype, float epsilon, int8_t* out,
                                                     float* quant_scale, cudaStream_t stream) {
+  // the checks of dq_ada_layernorm_quant, in its order, with the array's
+  // size limit in place of its workspace check
   size_t needed = 0;
   const dq_status st = dq_ada_layernorm_quant_get_workspace_size(batch, seq, hidden, x_dtype, param_dtype, &needed);
   if (st != DQ_OK) return st;
+  if (!(epsilon >= 0.0f) || epsilon == INFINITY) return DQ_ERR_BAD_ARGUMENT;  // NaN, negative or infinite
   if (needed == 0) return DQ_OK;  // batch * seq == 0: nothing to do, no set-up
+  if (x == nullptr || ada_scale == nullptr || ada_shift == nullptr || out == nullptr || quant_scale == nullptr)
+    return DQ_ERR_NULL_POINTER;
   if (batch > DQ_ADA_NOALLOC_MAX_TABLE / hidden) return DQ_ERR_UNSUPPORTED;  // table larger than the array
   void* table = nullptr;
   const dq_status ts = noalloc_table(&table);

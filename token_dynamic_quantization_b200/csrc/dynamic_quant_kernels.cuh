@@ -16,31 +16,11 @@
 //     two passes over the row (the second one mostly hits L2).
 #pragma once
 
+#include "dq_args.cuh"
 #include "dq_device.cuh"
 #include "tma_pipeline.cuh"
 
 namespace dq {
-
-enum : int { kSym = 0, kAsym = 1 };
-enum : int { kOutInt8 = 0, kOutInt4 = 1 };  // kOutInt4: INT4X2 and INT32 share bytes
-
-struct RowQuantArgs {
-  const void* x;
-  int64_t rows;
-  int64_t cols;
-  const void* smooth;          // nullptr, [cols] or [num_groups, cols]
-  int smooth_dtype;
-  const int32_t* group_index;  // nullptr or [num_groups] cumulative end rows
-  int num_groups;
-  void* y;
-  float* scale;
-  float* offset;               // asymmetric only
-  uint32_t* status;            // workspace status word (with a group index)
-  int tpr;                     // threads per row group (bulk-copy kernel)
-  int groups;                  // row groups per CTA (bulk-copy kernel)
-  int stages;                  // ring depth per group (bulk-copy kernel)
-  uint32_t stage_stride;       // bytes between stages (multiple of 128)
-};
 
 template <int MODE, int OUT>
 struct QuantConsts {

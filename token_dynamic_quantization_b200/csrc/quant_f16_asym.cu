@@ -1,0 +1,4 @@
+// DynamicQuant dispatch for f16 input, asym mode (aclnnDynamicQuantV2, "Formula").
+#include "quant_launch.cuh"
+
+DQ_DEFINE_QUANT_DISPATCH(quant_f16_asym, __half, dq::kAsym)

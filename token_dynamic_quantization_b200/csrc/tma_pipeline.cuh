@@ -8,17 +8,27 @@
 // shared memory, and the next copy into that stage is issued only after the
 // whole group has passed a barrier that follows those reads.
 //
-// Every wait is bounded: after kMaxWaitIterations unsuccessful try_wait
-// rounds the caller gets `false` and must take its error path (no GPU hang).
+// Every wait is bounded in time: after kWaitLimitNs without completion the
+// caller gets `false` and must take its error path (no GPU hang).
 #pragma once
 
 #include <stdint.h>
 
 namespace dq {
 
-// try_wait suspends for a hardware-defined interval per round; this bound is
-// seconds, far above any legitimate wait for one row copy.
-constexpr uint32_t kMaxWaitIterations = 1u << 22;
+// Every wait gives up after DQ_WAIT_LIMIT_NS nanoseconds of the global timer
+// (one second: far above any legitimate wait for a copy or an MMA, short
+// enough that a lost copy ends the kernel instead of hanging the GPU).
+#ifndef DQ_WAIT_LIMIT_NS
+#define DQ_WAIT_LIMIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = DQ_WAIT_LIMIT_NS;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,21 +72,57 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst_smem, const void* src_gm
       : "memory");
 }
 
-// Bounded wait for phase `parity` of `bar` to complete. Returns false on timeout.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait for phase `parity` of `bar` to complete. Returns false after
+// kWaitLimitNs without completion.
 __device__ __forceinline__ bool mbar_wait_parity(uint64_t* bar, uint32_t parity) {
   const uint32_t addr = smem_addr(bar);
-  for (uint32_t it = 0; it < kMaxWaitIterations; ++it) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
   }
-  return false;
+}
+
+// Bounded wait with an explicit limit in nanoseconds.
+__device__ __forceinline__ bool mbar_wait_parity_for(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t addr = smem_addr(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// The same wait that also gives up as soon as *abort (shared memory) is
+// non-zero: another warp of the CTA has met a failed wait.
+__device__ __forceinline__ bool mbar_wait_parity_or_abort(uint64_t* bar, uint32_t parity,
+                                                          const volatile uint32_t* abort) {
+  const uint32_t addr = smem_addr(bar);
+  if (mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(addr, parity)) return true;
+    if (*abort != 0u || global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Plain arrival (count 1) on `bar`.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // Group barrier over `nthreads` (a multiple of 32) that also ORs a predicate

@@ -250,13 +250,19 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         tc_commit(empty + s);  // the stage is free once these MMAs have read it
       }
       tc_commit(acc_ready);  // every MMA issued above is complete when this arrives
+      // this warp frees the TMEM below: it sees the MMAs complete itself, so
+      // the accumulator is never released under MMAs still in flight (even
+      // when the epilogue's wait has run out)
+      dq::mbar_wait_parity_for(acc_ready, 0, dq::kWaitLimitNs * (ktiles + 1));
     }
   } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
     // the tile's column scales, staged once by the 128 epilogue threads
 #pragma unroll
     for (int j = threadIdx.x - 64; j < kBN; j += 128) col_scale[j] = n0 + j < a.n ? a.b_scale[n0 + j] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    const bool ready = dq::mbar_wait_parity(acc_ready, 0) && *mma_failed == 0u;
+    // the MMA lane may take up to one wait limit per stage: the epilogue's
+    // budget covers the whole K loop
+    const bool ready = dq::mbar_wait_parity_for(acc_ready, 0, dq::kWaitLimitNs * (ktiles + 1)) && *mma_failed == 0u;
     tc_fence_after();
     const int quarter = warp & 3;
     const int64_t row = m0 + 32 * quarter + lane;
@@ -441,7 +447,8 @@ dq_status launch_tc(const W8A8Args& args, int device, cudaStream_t stream) {
 extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
                                   const float* a_scale, const float* b_scale, void* out, dq_dtype out_dtype,
                                   int32_t accumulate, cudaStream_t stream) {
-  if (m < 0 || n < 0 || k < 1 || k > (int64_t(1) << 17) || m > (int64_t(1) << 31) || n > (int64_t(1) << 31))
+  // k < 2^17: |sum| <= k * 128 * 128 < 2^31 for any int8 codes (-128 included)
+  if (m < 0 || n < 0 || k < 1 || k >= (int64_t(1) << 17) || m > (int64_t(1) << 31) || n > (int64_t(1) << 31))
     return DQ_ERR_BAD_SHAPE;
   if (out_dtype != DQ_F32 && out_dtype != DQ_F16 && out_dtype != DQ_BF16) return DQ_ERR_BAD_DTYPE;
   if (accumulate != 0 && accumulate != 1) return DQ_ERR_BAD_ARGUMENT;
