@@ -120,3 +120,29 @@ def test_bench_reference_arm_under_torchrun():
     rec = json.loads(lines[0])
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_gpus_n_starts_its_own_ranks():
+    """`bench.py --gpus 2` started as one plain process re-runs itself under
+    torch.distributed.run with two ranks: the line reports n_gpus 2."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "3",
+           "--warmup", "3", "--cpu-seconds", "0.3", "--workload", "sym_int8_f16_64x1024"]
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env["OMP_NUM_THREADS"] = "1"
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+
+
+def test_bench_refuses_a_world_size_that_differs_from_gpus():
+    """Under a launcher whose WORLD_SIZE is not --gpus, bench.py exits non-zero
+    instead of timing the wrong number of ranks."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2", "--steps", "3",
+           "--warmup", "3", "--cpu-seconds", "0.3", "--workload", "sym_int8_f16_64x1024"]
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0", OMP_NUM_THREADS="1")
+    res = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert res.returncode != 0
+    assert "WORLD_SIZE" in res.stderr
