@@ -120,6 +120,41 @@ def test_dynamic_quant_smooth(dq, smooth_dtype, mode, cols):
     assert_dq_equal(run_gpu(dq, x, smooth=smooth, mode=mode), want, "int8")
 
 
+# Row counts around the dispatch limits: the one-warp-per-row kernel serves at
+# most 2 rows per SM of one-warp rows (296 on 148 SMs); beyond that the ring
+# kernel runs with one CTA per SM, and its ring of at most 32 row slots is
+# reused when a CTA owns more rows than slots (5920 rows: 40 per CTA).
+RING_SHAPES = [(296, 1024), (297, 1024), (5920, 1024), (4500, 4096), (1200, 7168), (601, 16384)]
+
+
+@pytest.mark.parametrize("shape", RING_SHAPES, ids=[f"{r}x{c}" for r, c in RING_SHAPES])
+@pytest.mark.parametrize("mode", ["symmetric", "asymmetric"])
+@pytest.mark.parametrize("smooth_dtype", [None, torch.float32, torch.bfloat16], ids=["plain", "f32", "bf16"])
+def test_ring_slot_reuse_and_dispatch_limits(dq, shape, mode, smooth_dtype):
+    rows, cols = shape
+    x = rows_mix(rows, cols, torch.bfloat16, seed=rows + 3 * cols)
+    sm = None
+    if smooth_dtype is not None:
+        sm = (torch.rand(cols, generator=torch.Generator().manual_seed(cols)) * 1.5 + 0.5).to(smooth_dtype)
+    for y_dtype in ("int8", "int4"):
+        want = oracle.dynamic_quant(x, smooth=sm, mode=mode, y_dtype=y_dtype)
+        got = run_gpu(dq, x, smooth=sm, mode=mode, y_dtype=y_dtype)
+        assert_dq_equal(got, want, y_dtype)
+
+
+@pytest.mark.parametrize("rows,cols,experts", [(5920, 1024, 16), (3000, 4096, 64), (296, 1024, 8)])
+def test_ring_moe_many_rows_per_cta(dq, rows, cols, experts):
+    g = torch.Generator().manual_seed(rows)
+    x = rows_mix(rows, cols, torch.bfloat16, seed=rows + cols)
+    sm = torch.rand(experts, cols, generator=g) * 1.5 + 0.5
+    counts = torch.bincount(torch.randint(0, experts, (rows,), generator=g), minlength=experts)
+    gi = torch.cumsum(counts, 0).to(torch.int32)
+    want = oracle.dynamic_quant(x, smooth=sm, group_index=gi.numpy())
+    got = run_gpu(dq, x, smooth=sm, group_index=gi)
+    assert_dq_equal(got, want, "int8")
+    assert got[3] == 0
+
+
 @pytest.mark.parametrize("mode", ["symmetric", "asymmetric"])
 @pytest.mark.parametrize("y_dtype", ["int8", "int4"])
 def test_misaligned_pointers_take_the_scalar_path(dq, mode, y_dtype):
@@ -368,6 +403,20 @@ ADA_SHAPES = [(1, 1, 8), (2, 3, 64), (1, 3, 256), (1, 3, 512), (2, 7, 1024), (3,
 def test_ada_layernorm_quant_shapes(dq, shape, dtype, pdtype):
     b, s, h = shape
     x, sc, sh, w, bias, sm = _ada_inputs(b, s, h, dtype, pdtype, seed=h + s)
+    want = oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6)
+    got = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
+    assert_ada_close(got, want)
+
+
+# Many rows per CTA (ring slots reused), batch boundaries inside a CTA's rows,
+# and many small batches per CTA (the staged table holds several batches).
+ADA_RING_SHAPES = [(3, 1000, 1024), (64, 7, 1024), (2, 2500, 3072), (5, 1111, 2048), (300, 3, 256)]
+
+
+@pytest.mark.parametrize("shape", ADA_RING_SHAPES, ids=[f"{b}x{s}x{h}" for b, s, h in ADA_RING_SHAPES])
+def test_ada_ring_batches_across_ctas(dq, shape):
+    b, s, h = shape
+    x, sc, sh, w, bias, sm = _ada_inputs(b, s, h, torch.bfloat16, torch.bfloat16, seed=b * 31 + s + h)
     want = oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6)
     got = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
     assert_ada_close(got, want)

@@ -40,10 +40,10 @@ def _inputs() -> list[str]:
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def is_stale() -> bool:
-    if not os.path.exists(LIB):
+def is_stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _inputs() + [os.path.abspath(__file__)])
 
 
@@ -51,15 +51,19 @@ def _run(cmd: list[str]) -> subprocess.CompletedProcess:
     return subprocess.run(cmd, capture_output=True, text=True)
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True, lib: str = LIB,
+          defines: tuple[str, ...] = ()) -> str:
     """Compile every .cu under csrc/ (one object each, in parallel) and link
-    them into one shared library with a static CUDA runtime."""
-    if not force and not is_stale():
-        return LIB
+    them into one shared library with a static CUDA runtime. `lib` and
+    `defines` (extra -D flags) serve test builds of the same sources."""
+    if not force and not is_stale(lib):
+        return lib
     nvcc = _nvcc()
-    objdir = os.path.join(PKG, "_build")
+    objdir = os.path.join(PKG, "_build", os.path.basename(lib).replace(".so", ""))
     os.makedirs(objdir, exist_ok=True)
-    common = [*ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC]
+    common = [*ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-Xfatbin=-compress-all",
+              "-I", INCLUDE, "-I", CSRC,
+              *(f"-D{d}" for d in defines)]
     if ptxas_verbose:
         common.insert(0, "-Xptxas=-v")
     jobs = []
@@ -74,7 +78,7 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
     if failed:
         sys.stderr.write(log)
         raise RuntimeError(f"nvcc failed compiling {', '.join(os.path.basename(f) for f in failed)}")
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     link = _run([nvcc, *ARCH_FLAGS, "-shared", "--cudart", "static", "-o", tmp, *(j[0] for j in jobs)])
     for obj, _ in jobs:
         try:
@@ -83,11 +87,24 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
             pass
     if link.returncode != 0:
         sys.stderr.write(log + link.stdout + link.stderr)
-        raise RuntimeError(f"nvcc failed linking {LIB}")
+        raise RuntimeError(f"nvcc failed linking {lib}")
     if not quiet or ptxas_verbose:
         sys.stderr.write(log + link.stdout + link.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+# Test build: the same sources with a 2 ms wait limit and one row copy (global
+# row 777 of the quantizers) and one W8A8 operand stage (tile row 1, k-tile 2)
+# left out, so that the tests can run the kernels' timeout paths. Only the
+# tests load it; the product library has none of these flags.
+WAIT_TEST_LIB = os.path.join(PKG, "libdq_waittest.so")
+WAIT_TEST_DEFINES = ("DQ_WAIT_LIMIT_NS=2000000ull", "DQ_TEST_SKIP_COPY_ROW=777", "DQ_TEST_SKIP_W8A8_TILE_M=1",
+                     "DQ_TEST_SKIP_W8A8_KTILE=2")
+
+
+def build_wait_test(force: bool = False) -> str:
+    return build(force=force, lib=WAIT_TEST_LIB, defines=WAIT_TEST_DEFINES)
 
 
 def main(argv=None) -> int:

@@ -4,6 +4,7 @@
 #include <cstdlib>
 
 #include "ada_layernorm_quant_kernels.cuh"
+#include "ada_layernorm_quant_ring.cuh"
 #include "dq_launch.cuh"
 
 namespace dq_host {
@@ -24,42 +25,78 @@ dq_status launch_ada_table(const dq::AdaArgs& a, int sms, cudaStream_t stream) {
   return launch_programmatic(dq::ada_affine_table_kernel, a, static_cast<int>(grid), dq::kTableBlock, 0, stream);
 }
 
-template <typename InT, int VPT, bool kRagged>
-dq_status launch_ada_tma(dq::AdaArgs a, int device, int sms, cudaStream_t stream) {
-  void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_tma_kernel<InT, VPT, kRagged>;
+// Largest dynamic shared memory of one CTA on sm_100 (227 KB), less the
+// ring kernel's static shared memory and a reserve; the part of it the staged
+// affine table may take.
+constexpr size_t kAdaRingSmemBudget = 232448 - 2048;
+#ifndef DQ_ADA_TABLE_BUDGET
+#define DQ_ADA_TABLE_BUDGET (64 * 1024)
+#endif
+#ifndef DQ_ADA_RING_MAX_SLOTS
+#define DQ_ADA_RING_MAX_SLOTS 32
+#endif
+
+// Ring kernel launch: one CTA per SM (fewer for few rows), NC consumer groups
+// of G warps (as many as the registers allow, at most 15 with G > 1), the
+// table rows of the CTA's batches staged when they fit DQ_ADA_TABLE_BUDGET,
+// NS row slots in the rest of the shared memory.
+template <typename InT, int VPT, bool kRagged, bool kStaged>
+dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batches, cudaStream_t stream) {
+  void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_ring_kernel<InT, VPT, kRagged, kStaged>;
   const void* k = reinterpret_cast<const void*>(kfn);
-  const size_t smem = dq::ada_smem_bytes(a.groups, a.stages, a.stage_stride);
-  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return kNotLaunchable;
-  const int block = a.tpr * a.groups;
+  if (!allow_smem_bytes(k, device, kAdaRingSmemBudget)) return kNotLaunchable;
+  const int regs = kernel_registers(k, device);
+  if (regs <= 0) return kNotLaunchable;
+  const int G = a.tpr / 32;
   const int64_t rows = a.batch * a.seq;
-  const int64_t wanted = (rows + a.groups - 1) / a.groups;
-  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
-  if (resident < 1) return kNotLaunchable;
-  const int grid = static_cast<int>(wanted < resident ? wanted : resident);
+  const int64_t grid = rows < sms ? rows : sms;
+  const int64_t per_cta = (rows + grid - 1) / grid;
+  int64_t nc = (65536 / (32 * ((regs + 7) / 8 * 8)) - 1) / G;
+  if (nc > (dq::kRingMaxThreads / 32 - 1) / G) nc = (dq::kRingMaxThreads / 32 - 1) / G;
+  if (G > 1 && nc > 15) nc = 15;
+  if (nc > per_cta) nc = per_cta;
+  a.table_batches = kStaged ? static_cast<int>(table_batches) : 0;
+  const size_t fixed = dq::ada_ring_smem_bytes(0, a.stage_stride, a.table_batches, a.hidden);
+  if (fixed >= kAdaRingSmemBudget) return kNotLaunchable;
+  int64_t ns = static_cast<int64_t>((kAdaRingSmemBudget - fixed) / (a.stage_stride + 16));
+  if (ns > DQ_ADA_RING_MAX_SLOTS) ns = DQ_ADA_RING_MAX_SLOTS;
+  if (ns > per_cta) ns = per_cta;
+  if (nc > ns) nc = ns;
+  if (nc < 1) return kNotLaunchable;
+  a.groups = static_cast<int>(nc);
+  a.stages = static_cast<int>(ns);
+  const size_t smem = dq::ada_ring_smem_bytes(a.stages, a.stage_stride, a.table_batches, a.hidden);
+  const int block = 32 + a.tpr * a.groups;
+  if (blocks_per_sm(k, block, smem, device) < 1) return kNotLaunchable;
   dq_status st = launch_ada_table(a, sms, stream);
   if (st != DQ_OK) return st;
-  return launch_programmatic(kfn, a, grid, block, smem, stream);
+  return launch_programmatic(kfn, a, static_cast<int>(grid), block, smem, stream);
 }
 
 template <typename InT, int VPT>
 dq_status launch_ada_ragged(dq::AdaArgs a, int device, int sms, cudaStream_t stream) {
-  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds checks
-  if ((a.hidden >> 3) == static_cast<int64_t>(a.tpr) * VPT) return launch_ada_tma<InT, VPT, false>(a, device, sms, stream);
-  return launch_ada_tma<InT, VPT, true>(a, device, sms, stream);
+  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds
+  // checks; the table rows of a CTA's batches are staged when they fit
+  const bool exact = (a.hidden >> 3) == static_cast<int64_t>(a.tpr) * VPT;
+  const int64_t rows = a.batch * a.seq;
+  const int64_t grid = rows < sms ? rows : sms;
+  const int64_t per_cta = (rows + grid - 1) / grid;
+  int64_t nb = (per_cta - 1) / a.seq + 2;  // batches a range of per_cta rows can touch
+  if (nb > a.batch) nb = a.batch;
+  const bool staged = static_cast<size_t>(nb) * static_cast<size_t>(a.hidden) * 8 <= DQ_ADA_TABLE_BUDGET;
+  if (exact) {
+    return staged ? launch_ada_ring<InT, VPT, false, true>(a, device, sms, nb, stream)
+                  : launch_ada_ring<InT, VPT, false, false>(a, device, sms, nb, stream);
+  }
+  return staged ? launch_ada_ring<InT, VPT, true, true>(a, device, sms, nb, stream)
+                : launch_ada_ring<InT, VPT, true, false>(a, device, sms, nb, stream);
 }
 
 // AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8}, fewest wasted lanes,
 // then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
-// two row reductions; the row share stays in registers). DQ_ADA_STAGES row
-// buffers per group, one of them holding the row being processed.
+// row reductions; the row share stays in registers).
 #ifndef DQ_ADA_TARGET_VPT
-#define DQ_ADA_TARGET_VPT 6  // hidden 3072: 2 warps x 6 vectors per row (2811 GB/s) over 3 x 4 (2652)
-#endif
-#ifndef DQ_ADA_CTA_BYTES
-#define DQ_ADA_CTA_BYTES 147456  // 8 row groups of 64 threads at hidden 3072: 16 warps per SM
-#endif
-#ifndef DQ_ADA_STAGES
-#define DQ_ADA_STAGES 3
+#define DQ_ADA_TARGET_VPT 6  // hidden 3072: 2 warps x 6 vectors per row
 #endif
 
 GroupShape pick_ada_shape(int64_t nvec) {
@@ -88,17 +125,9 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
   if (vector_ok) {
     const GroupShape gs = pick_ada_shape(a.hidden >> 3);
     if (gs.vpt > 0) {
-      const uint32_t stride = static_cast<uint32_t>((a.hidden * 2 + 127) / 128 * 128);
-      const int stages = DQ_ADA_STAGES;
-      int64_t groups = DQ_ADA_CTA_BYTES / (static_cast<int64_t>(stages) * stride);
-      const int64_t max_groups = dq::kAdaMaxBlock / gs.tpr;
-      groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
-      groups = groups > 15 ? 15 : groups;
+      a.stage_stride = static_cast<uint32_t>((a.hidden * 2 + 127) / 128 * 128);
       a.tpr = gs.tpr;
-      a.groups = static_cast<int>(groups);
-      a.stages = stages;
-      a.stage_stride = stride;
-      if (dq::ada_smem_bytes(a.groups, stages, stride) <= kMaxDynamicSmem) {
+      {
         dq_status st;
         switch (gs.vpt) {
           case 2: st = launch_ada_ragged<InT, 2>(a, device, sms, stream); break;

@@ -1,0 +1,354 @@
+// Fused AdaLayerNorm + symmetric INT8 dynamic quantization, ring kernel
+// (aclnnAdaLayerNormQuant, "Formula" steps 1-5), sm_100a.
+//
+// The row kernel of the fused path, on the structure of the DynamicQuant ring
+// kernel (dynamic_quant_ring.cuh): one persistent CTA per SM owns a
+// contiguous range of rows; warp 0 lane 0 streams them with cp.async.bulk
+// into a CTA-wide ring of NS slots; NC consumer groups of G warps take rows
+// c, c + NC, ... and release each slot as soon as its row is in registers.
+// The folded affine table (A, B per batch and column, written by
+// ada_affine_table_kernel) is staged in shared memory for the batches the
+// CTA's rows belong to, so the per-element reads of steps 1-3 are shared
+// loads instead of L1/L2 loads on every row.
+//
+// Arithmetic per row, as in ada_layernorm_quant_tma_kernel: both moments of
+// d = x - K (K the mean of the row's first 8 elements) from one reduction,
+// fp32 partial sums per thread and warp, double across warps, a centred second
+// pass for rows whose first elements sit far from the mean; then
+// n = fma(d, rstd, -(E(x) - K) * rstd), y = n * A + B, absmax, and the exact
+// symmetric INT8 quantizer.
+//
+// Failure handling as in the DynamicQuant ring kernel: every wait is bounded
+// in time and gives up on the shared abort flag; a group whose row never
+// arrives writes NaN quant scales for its remaining rows and stops.
+#pragma once
+
+#include "ada_layernorm_quant_kernels.cuh"
+#include "dq_args.cuh"
+#include "dq_device.cuh"
+#include "tma_pipeline.cuh"
+
+namespace dq {
+
+// Shared memory of the AdaLN ring kernel: NS row slots of `stride` bytes;
+// full[NS], empty[NS]; a 16-byte abort word; then, when staged,
+// A[table_batches][hidden] and B[table_batches][hidden] (fp32).
+__host__ __device__ inline size_t ada_ring_smem_bytes(int slots, uint32_t stride, int table_batches, int64_t hidden) {
+  return static_cast<size_t>(slots) * stride + static_cast<size_t>(slots) * 16 + 16 +
+         static_cast<size_t>(table_batches) * static_cast<size_t>(hidden) * 8;
+}
+
+#ifndef DQ_ADA_RING_MAX_REGS
+#define DQ_ADA_RING_MAX_REGS 128
+#endif
+
+template <typename InT, int VPT, bool kRagged, bool kStaged>
+__global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kernel(const AdaArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ double red_d[2][3][32];  // [parity][sum | sq | centred sq][warp]
+  __shared__ float red_f[2][32];      // [parity][warp] absmax
+
+  const int NS = a.stages;
+  const uint32_t stride = a.stage_stride;
+  const int tpr = a.tpr;
+  const int G = tpr >> 5;
+  const int NC = a.groups;
+  const int64_t H = a.hidden;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * stride);
+  uint64_t* empty = full + NS;
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + NS);
+  float* table_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(empty + NS) + 16);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = a.batch * a.seq;
+  const int64_t r_begin = static_cast<int64_t>(blockIdx.x) * rows / gridDim.x;
+  const int n = static_cast<int>((static_cast<int64_t>(blockIdx.x) + 1) * rows / gridDim.x - r_begin);
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, static_cast<uint32_t>(G));
+    }
+    *abort_flag = 0u;
+    fence_mbarrier_init();
+  }
+
+  // Producer state (thread 0). The first NS copies go out before the wait for
+  // the table kernel: that kernel waited for the work before it before it let
+  // this one start, so x is already final.
+  int issued = 0;
+  const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  uint64_t policy = 0;
+  auto issue = [&](int s) {
+#ifdef DQ_TEST_SKIP_COPY_ROW
+    // test builds only: leave one row's copy out (see dynamic_quant_ring.cuh)
+    if (r_begin + issued == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) {
+      x_next += row_bytes;
+      ++issued;
+      return;
+    }
+#endif
+    mbar_arrive_expect_tx(full + s, row_bytes);
+    bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_next, row_bytes, full + s, policy);
+    x_next += row_bytes;
+    ++issued;
+  };
+  if (threadIdx.x == 0 && n > 0) {
+    policy = l2_evict_first_policy();
+    while (issued < NS && issued < n) issue(issued);
+  }
+  pdl_wait_primary();  // the affine table is complete and visible from here on
+  pdl_launch_dependents();
+
+  // the table rows of the batches this CTA's rows belong to
+  const int64_t b_lo = n > 0 ? r_begin / a.seq : 0;
+  if (kStaged && n > 0) {
+    const int64_t nb = (r_begin + n - 1) / a.seq - b_lo + 1;  // <= table_batches (host)
+    const int64_t per = H / 4;                                // float4 per table row
+    const float4* A_g = reinterpret_cast<const float4*>(a.table + b_lo * H);
+    const float4* B_g = reinterpret_cast<const float4*>(a.table + a.batch * H + b_lo * H);
+    float4* A_s = reinterpret_cast<float4*>(table_s);
+    float4* B_s = reinterpret_cast<float4*>(table_s + static_cast<int64_t>(a.table_batches) * H);
+    for (int64_t i = threadIdx.x; i < nb * per; i += blockDim.x) {
+      A_s[i] = __ldg(A_g + i);
+      B_s[i] = __ldg(B_g + i);
+    }
+  }
+  __syncthreads();
+  if (n <= 0) return;
+
+  // ------------------------------------------------------------ producer
+  if (warp == 0) {
+    if (lane != 0) return;
+    int s = issued % NS;
+    uint32_t k = static_cast<uint32_t>(issued / NS);
+    while (issued < n) {
+      if (!mbar_wait_parity_or_abort(empty + s, (k - 1u) & 1u, abort_flag)) {
+        *abort_flag = 1u;
+        break;
+      }
+      fence_proxy_async_smem();
+      issue(s);
+      if (++s == NS) {
+        s = 0;
+        ++k;
+      }
+    }
+    for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
+      mbar_wait_parity(full + (j % NS), static_cast<uint32_t>(j / NS) & 1u);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int cw = warp - 1;
+  const int c = cw / G;
+  const int wg = cw - c * G;
+  const int lane_g = wg * 32 + lane;
+  const int warp_g0 = 1 + c * G;
+  if (c >= NC || c >= n) return;
+  const int nvec = static_cast<int>(H >> 3);
+  const int vbase = wg * (32 * VPT) + lane;
+  auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
+  const int64_t table_b_stride4 = H / 4;  // float4 per batch row
+  const float4* A_base = kStaged ? reinterpret_cast<const float4*>(table_s)
+                                 : reinterpret_cast<const float4*>(a.table);
+  const float4* B_base = kStaged ? reinterpret_cast<const float4*>(table_s + static_cast<int64_t>(a.table_batches) * H)
+                                 : reinterpret_cast<const float4*>(a.table + a.batch * H);
+  const int64_t b_origin = kStaged ? b_lo : 0;
+
+  int s = c;
+  uint32_t par = 0u;
+  int parity = 0;
+  int64_t b = -1, b_end = -1;
+  const float4* A4 = nullptr;
+  const float4* B4 = nullptr;
+  int8_t* orow = a.out + (r_begin + c) * H;
+  const int64_t o_step = H * NC;
+  for (int j = c; j < n; j += NC, orow += o_step) {
+    const int64_t r = r_begin + j;
+    if (r >= b_end) {
+      b = r / a.seq;
+      b_end = (b + 1) * a.seq;
+      A4 = A_base + (b - b_origin) * table_b_stride4 + 2 * vbase;
+      B4 = B_base + (b - b_origin) * table_b_stride4 + 2 * vbase;
+    }
+    const bool ok = mbar_wait_parity_or_abort(full + s, par, abort_flag);
+    const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
+
+    // ---- pass 1: load, widen, shift by K, both moments of d = x - K
+    constexpr int NACC = VPT < 4 ? VPT : 4;
+    float K;
+    {
+      float f[8];
+      InTraits<InT>::widen8(srow[0], f);
+      K = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(f[0], f[1]), __fadd_rn(f[2], f[3])),
+                              __fadd_rn(__fadd_rn(f[4], f[5]), __fadd_rn(f[6], f[7]))),
+                    0.125f);
+    }
+    float v[VPT][8];
+    float2 acc[NACC], acq[NACC];
+#pragma unroll
+    for (int t = 0; t < NACC; ++t) acc[t] = acq[t] = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const bool active = in_row(k);
+      InTraits<InT>::widen8(active ? srow[vbase + 32 * k] : make_uint4(0, 0, 0, 0), v[k]);
+      float2 d[4];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        d[p] = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-K));
+        if (kRagged && !active) d[p] = make_float2(0.0f, 0.0f);
+        v[k][2 * p] = d[p].x;
+        v[k][2 * p + 1] = d[p].y;
+        acq[(k + p) % NACC] = __ffma2_rn(d[p], d[p], acq[(k + p) % NACC]);
+      }
+      acc[k % NACC] = __fadd2_rn(acc[k % NACC], __fadd2_rn(__fadd2_rn(d[0], d[1]), __fadd2_rn(d[2], d[3])));
+    }
+#pragma unroll
+    for (int t = 1; t < NACC; ++t) {
+      acc[0] = __fadd2_rn(acc[0], acc[t]);
+      acq[0] = __fadd2_rn(acq[0], acq[t]);
+    }
+    float s1 = __fadd_rn(acc[0].x, acc[0].y), s2 = __fadd_rn(acq[0].x, acq[0].y);
+    // butterflies: every lane ends with the same bits; the lane shuffles also
+    // make every lane's shared loads of the slot complete
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
+      s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
+    }
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(empty + s);
+    s += NC;
+    if (s >= NS) {
+      s -= NS;
+      par ^= 1u;
+    }
+    double sum = s1, sq = s2;
+    bool failed;
+    if (G > 1) {
+      if (lane == 0) {
+        red_d[parity][0][warp] = sum;
+        red_d[parity][1][warp] = sq;
+      }
+      failed = group_barrier_or(1 + c, tpr, !ok);
+      sum = 0.0;
+      sq = 0.0;
+      for (int w = 0; w < G; ++w) {
+        sum += red_d[parity][0][warp_g0 + w];
+        sq += red_d[parity][1][warp_g0 + w];
+      }
+    } else {
+      failed = __any_sync(0xffffffffu, !ok);
+    }
+    if (failed) {
+      *abort_flag = 1u;
+      for (int jj = j + lane_g * NC; jj < n; jj += tpr * NC) a.quant_scale[r_begin + jj] = __int_as_float(0x7fc00000);
+      return;
+    }
+    const double m1 = sum * a.inv_hidden;  // E(d)
+    const double m2 = sq * a.inv_hidden;   // E(d^2)
+    const float mean_f = __double2float_rn(static_cast<double>(K) + m1);
+    const float c_f = __fsub_rn(mean_f, K);
+    double var_d;
+    if (m1 * m1 <= 0.75 * m2) {
+      var_d = m2 - m1 * m1;
+    } else {
+      // ---- centred second pass (rows whose first elements sit far from the mean)
+#pragma unroll
+      for (int t = 0; t < NACC; ++t) acq[t] = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        const bool active = in_row(k);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          float2 e = __fadd2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(-c_f));
+          if (kRagged && !active) e = make_float2(0.0f, 0.0f);
+          acq[(k + p) % NACC] = __ffma2_rn(e, e, acq[(k + p) % NACC]);
+        }
+      }
+#pragma unroll
+      for (int t = 1; t < NACC; ++t) acq[0] = __fadd2_rn(acq[0], acq[t]);
+      double sc = warp_sum(static_cast<double>(acq[0].x) + static_cast<double>(acq[0].y));
+      if (G > 1) {
+        if (lane == 0) red_d[parity][2][warp] = sc;
+        group_barrier(1 + c, tpr);
+        sc = 0.0;
+        for (int w = 0; w < G; ++w) sc += red_d[parity][2][warp_g0 + w];
+      }
+      const double dm = m1 - static_cast<double>(c_f);
+      var_d = sc * a.inv_hidden - dm * dm;
+    }
+    var_d = var_d > 0.0 ? var_d : 0.0;
+    const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__double2float_rn(var_d), a.epsilon)));
+    const float nb = -__fmul_rn(c_f, rstd);
+
+    // ---- pass 2: y = n * A + B, absmax
+    float amx[NACC];
+#pragma unroll
+    for (int t = 0; t < NACC; ++t) amx[t] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      if (in_row(k)) {
+        const float4 a0 = kStaged ? A4[64 * k] : __ldg(A4 + 64 * k);
+        const float4 a1 = kStaged ? A4[64 * k + 1] : __ldg(A4 + 64 * k + 1);
+        const float4 b0 = kStaged ? B4[64 * k] : __ldg(B4 + 64 * k);
+        const float4 b1 = kStaged ? B4[64 * k + 1] : __ldg(B4 + 64 * k + 1);
+        const float Av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 nn = __ffma2_rn(make_float2(v[k][2 * p], v[k][2 * p + 1]), f2(rstd), f2(nb));
+          const float2 y =
+              __ffma2_rn(nn, make_float2(Av[2 * p], Av[2 * p + 1]), make_float2(Bv[2 * p], Bv[2 * p + 1]));
+          v[k][2 * p] = y.x;
+          v[k][2 * p + 1] = y.y;
+        }
+        amx[k % NACC] = fmaxf(amx[k % NACC], absmax8(v[k]));
+      }
+    }
+    float amax = warp_max(tree<NACC, true>(amx));
+    if (G > 1) {
+      if (lane == 0) red_f[parity][warp] = amax;
+      group_barrier(1 + c, tpr);
+      amax = warp_max(lane < G ? red_f[parity][warp_g0 + lane] : 0.0f);
+      parity ^= 1;
+    }
+
+    // ---- steps 4-5
+    const RowQuant q = make_sym<127>(amax);
+    if (lane_g == 0) __stcs(a.quant_scale + r, q.scale);
+    uint2* ov = reinterpret_cast<uint2*>(orow) + vbase;
+    if (q.zero_scale) {
+      const uint2 zeros = make_uint2(0u, 0u);
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        if (in_row(k)) __stcs(ov + 32 * k, zeros);
+      }
+      continue;
+    }
+    if (q.exact_row) {
+      // rare (quant_scale below 2^-40): the IEEE division for every element
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        if (!in_row(k)) continue;
+        uint32_t bits[8];
+        quant8_exact<false>(v[k], q, -127.0f, 127.0f, bits);
+        __stcs(ov + 32 * k, pack8_int8(bits));
+      }
+      continue;
+    }
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      if (!in_row(k)) continue;
+      uint32_t bits[8];
+      quant8<false, false>(v[k], q, -127.0f, 127.0f, bits);
+      __stcs(ov + 32 * k, pack8_int8(bits));
+    }
+  }
+}
+
+}  // namespace dq

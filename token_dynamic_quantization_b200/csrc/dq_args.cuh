@@ -6,6 +6,9 @@
 
 namespace dq {
 
+// Largest CTA of the ring kernels: one producer warp and up to 31 consumer warps.
+constexpr int kRingMaxThreads = 1024;
+
 // Element type tags (mirror the dq_dtype values of the C ABI).
 enum : int { kF32 = 0, kF16 = 1, kBF16 = 2 };
 
@@ -50,6 +53,7 @@ struct AdaArgs {
   int groups;
   int stages;
   uint32_t stage_stride;
+  int table_batches;      // ring kernel: batches of the table staged in shared memory per CTA (0: read from L2)
 };
 
 // ---- dequantization (AntiQuantize)

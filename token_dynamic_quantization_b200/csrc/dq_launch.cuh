@@ -97,6 +97,52 @@ inline bool allow_smem(const void* kernel, int device) {
   return true;
 }
 
+// The same opt-in for an explicit number of bytes.
+inline bool allow_smem_bytes(const void* kernel, int device, size_t bytes) {
+  struct Entry {
+    const void* k;
+    int device;
+    size_t bytes;
+  };
+  static Entry done[512];
+  static int used = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i) {
+    if (done[i].k == kernel && done[i].device == device && done[i].bytes >= bytes) return true;
+  }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (used < 512) done[used++] = Entry{kernel, device, bytes};
+  return true;
+}
+
+// Registers per thread of a compiled kernel (0 if unknown); cached.
+inline int kernel_registers(const void* kernel, int device) {
+  struct Entry {
+    const void* k;
+    int device;
+    int regs;
+  };
+  static Entry cache[512];
+  static int used = 0;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i) {
+    if (cache[i].k == kernel && cache[i].device == device) return cache[i].regs;
+  }
+  cudaFuncAttributes attr{};
+  if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (used < 512) cache[used++] = Entry{kernel, device, attr.numRegs};
+  return attr.numRegs;
+}
+
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 inline dq_status launch_status() {

@@ -1,5 +1,5 @@
-// DynamicQuant launch selection (aclnnDynamicQuantV2): the bulk-copy row
-// kernel's shape for a row width, or the generic kernel. Included by one
+// DynamicQuant launch selection (aclnnDynamicQuantV2): the ring kernel's
+// shape for a row width, or the generic kernel. Included by one
 // translation unit per (input type, mode) so the instantiations compile in
 // parallel.
 #pragma once
@@ -8,6 +8,7 @@
 
 #include "dq_launch.cuh"
 #include "dynamic_quant_kernels.cuh"
+#include "dynamic_quant_ring.cuh"
 
 namespace dq_host {
 
@@ -17,29 +18,16 @@ struct GroupShape {
   int tpr;
 };
 
-// Row-group geometry of the bulk-copy DynamicQuant kernel: a group of
-// tpr = 32 * G threads owns a row, VPT in {2, 4, 6, 7, 8} vectors per thread;
-// the shape wasting the fewest lanes wins, then the one whose VPT is closest
-// to the target VPT (8 by default: more elements per thread amortize the
-// per-row work; with smooth scales the fp32 products of pass 1 stay in
-// registers for pass 2). DQ_WARP_STAGES row buffers per group; groups per CTA
-// so that a CTA holds about DQ_WARP_CTA_BYTES_SMOOTH / _PLAIN of rows
-// (measured: the smooth-scale path prefers several groups sharing a CTA, the
-// plain path smaller CTAs).
+// Row-group geometry of the ring kernel: a group of tpr = 32 * G threads owns
+// a row, VPT in {2, 4, 6, 7, 8} 16-byte vectors per thread; the shape wasting
+// the fewest lanes wins, then the one whose VPT is closest to the target VPT
+// (8: more elements per thread amortize the per-row work, and with smooth
+// scales the fp32 products of pass 1 stay in registers for pass 2).
 #ifndef DQ_TARGET_VPT_SMOOTH
 #define DQ_TARGET_VPT_SMOOTH 8
 #endif
 #ifndef DQ_TARGET_VPT_PLAIN
 #define DQ_TARGET_VPT_PLAIN 8
-#endif
-#ifndef DQ_WARP_STAGES
-#define DQ_WARP_STAGES 2
-#endif
-#ifndef DQ_WARP_CTA_BYTES_SMOOTH
-#define DQ_WARP_CTA_BYTES_SMOOTH 65536
-#endif
-#ifndef DQ_WARP_CTA_BYTES_PLAIN
-#define DQ_WARP_CTA_BYTES_PLAIN 32768
 #endif
 
 inline GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
@@ -61,26 +49,80 @@ inline GroupShape pick_dq_shape(int64_t nvec, int target_vpt) {
   return best;
 }
 
-template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged>
-dq_status launch_dq_tma(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
-  const void* k = reinterpret_cast<const void*>(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>);
-  const size_t smem = dq::dq_smem_bytes(a.groups, a.stages, a.stage_stride, a.group_index ? a.num_groups : 0);
-  if (smem > kMaxDynamicSmem || !allow_smem(k, device)) return kNotLaunchable;
-  const int block = a.tpr * a.groups;
-  const int64_t wanted = (a.rows + a.groups - 1) / a.groups;
-  const int64_t resident = static_cast<int64_t>(sms) * blocks_per_sm(k, block, smem, device);
-  if (resident < 1) return kNotLaunchable;
-  const int grid = static_cast<int>(wanted < resident ? wanted : resident);
-  return launch_programmatic(dq::dynamic_quant_tma_kernel<InT, MODE, OUT, SMK, VPT, kRagged>, a, grid, block, smem,
-                             stream);
+// Largest dynamic shared memory of one CTA on sm_100 (227 KB), less the
+// ring kernel's static shared memory and a reserve.
+constexpr size_t kRingSmemBudget = 232448 - 1024;
+#ifndef DQ_RING_MAX_SLOTS
+#define DQ_RING_MAX_SLOTS 32
+#endif
+
+// Ring kernel launch: one CTA per SM (fewer for few rows), NC consumer groups
+// of G = tpr / 32 warps, as many as the kernel's registers allow (at most 15
+// with G > 1: one named barrier each), and NS row slots filling the shared
+// memory (NC <= NS <= rows of a CTA).
+template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged, bool kSS>
+dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
+  void (*kfn)(const dq::RowQuantArgs) = dq::dynamic_quant_ring_kernel<InT, MODE, OUT, SMK, VPT, kRagged, kSS>;
+  const void* k = reinterpret_cast<const void*>(kfn);
+  if (!allow_smem_bytes(k, device, kRingSmemBudget)) return kNotLaunchable;
+  const int regs = kernel_registers(k, device);
+  if (regs <= 0) return kNotLaunchable;
+  const int G = a.tpr / 32;
+  const int64_t grid = a.rows < sms ? a.rows : sms;
+  const int64_t per_cta = (a.rows + grid - 1) / grid;
+  int64_t nc = (65536 / (32 * ((regs + 7) / 8 * 8)) - 1) / G;  // warps the register file holds, less the producer
+  if (nc > (dq::kRingMaxThreads / 32 - 1) / G) nc = (dq::kRingMaxThreads / 32 - 1) / G;
+  if (G > 1 && nc > 15) nc = 15;
+  if (nc > per_cta) nc = per_cta;
+  const size_t smooth_bytes = kSS ? static_cast<size_t>(a.cols) * (SMK == dq::kSmF32 ? 4 : 2) : 0;
+  const size_t fixed = dq::ring_smem_bytes(0, a.stage_stride, smooth_bytes, a.group_index ? a.num_groups : 0);
+  if (fixed >= kRingSmemBudget) return kNotLaunchable;
+  int64_t ns = static_cast<int64_t>((kRingSmemBudget - fixed) / (a.stage_stride + 16));
+  if (ns > DQ_RING_MAX_SLOTS) ns = DQ_RING_MAX_SLOTS;
+  if (ns > per_cta) ns = per_cta;
+  if (nc > ns) nc = ns;
+  if (nc < 1) return kNotLaunchable;
+  a.groups = static_cast<int>(nc);
+  a.stages = static_cast<int>(ns);
+  const size_t smem = dq::ring_smem_bytes(a.stages, a.stage_stride, smooth_bytes, a.group_index ? a.num_groups : 0);
+  const int block = 32 + a.tpr * a.groups;
+  if (blocks_per_sm(k, block, smem, device) < 1) return kNotLaunchable;
+  return launch_programmatic(kfn, a, static_cast<int>(grid), block, smem, stream);
 }
+
+// Few short rows: one warp per row, one warp per CTA (see
+// dynamic_quant_warp_kernel).
+template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged>
+dq_status launch_dq_warp(const dq::RowQuantArgs& a, int sms, cudaStream_t stream) {
+  const int64_t cap = static_cast<int64_t>(sms) * 16;
+  const int grid = static_cast<int>(a.rows < cap ? a.rows : cap);
+  return launch_programmatic(dq::dynamic_quant_warp_kernel<InT, MODE, OUT, SMK, VPT, kRagged>, a, grid,
+                             dq::kWarpRowThreads, 0, stream);
+}
+
+// The warp kernel serves rows of one warp (tpr == 32) when there are at most
+// DQ_WARP_KERNEL_MAX_ROWS_PER_SM rows per SM: too few for the ring's per-CTA
+// set-up and copy pipeline to pay off.
+#ifndef DQ_WARP_KERNEL_MAX_ROWS_PER_SM
+#define DQ_WARP_KERNEL_MAX_ROWS_PER_SM 2
+#endif
 
 template <typename InT, int MODE, int OUT, int SMK, int VPT>
 dq_status launch_dq_ragged(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
-  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds checks
-  if ((a.cols >> 3) == static_cast<int64_t>(a.tpr) * VPT)
-    return launch_dq_tma<InT, MODE, OUT, SMK, VPT, false>(a, device, sms, stream);
-  return launch_dq_tma<InT, MODE, OUT, SMK, VPT, true>(a, device, sms, stream);
+  // exact tiling (the row is G * 32 * VPT vectors) needs no per-vector bounds
+  // checks; a dense smooth table is staged in shared memory
+  const bool exact = (a.cols >> 3) == static_cast<int64_t>(a.tpr) * VPT;
+  if (a.tpr == 32 && a.rows <= static_cast<int64_t>(sms) * DQ_WARP_KERNEL_MAX_ROWS_PER_SM) {
+    return exact ? launch_dq_warp<InT, MODE, OUT, SMK, VPT, false>(a, sms, stream)
+                 : launch_dq_warp<InT, MODE, OUT, SMK, VPT, true>(a, sms, stream);
+  }
+  const bool staged = SMK != dq::kSmNone && a.group_index == nullptr;
+  if (exact) {
+    return staged ? launch_dq_ring<InT, MODE, OUT, SMK, VPT, false, SMK != dq::kSmNone>(a, device, sms, stream)
+                  : launch_dq_ring<InT, MODE, OUT, SMK, VPT, false, false>(a, device, sms, stream);
+  }
+  return staged ? launch_dq_ring<InT, MODE, OUT, SMK, VPT, true, SMK != dq::kSmNone>(a, device, sms, stream)
+                : launch_dq_ring<InT, MODE, OUT, SMK, VPT, true, false>(a, device, sms, stream);
 }
 
 template <typename InT, int MODE, int OUT, int SMK>
@@ -103,18 +145,9 @@ dq_status launch_dynamic_quant(dq::RowQuantArgs a, bool vector_ok, cudaStream_t 
         pick_dq_shape(a.cols >> 3, a.smooth != nullptr ? DQ_TARGET_VPT_SMOOTH : DQ_TARGET_VPT_PLAIN);
     if (gs.vpt > 0) {
       const int64_t row_bytes = a.cols * 2;
-      const uint32_t stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
-      const int stages = DQ_WARP_STAGES;
-      const int64_t cta_bytes = a.smooth != nullptr ? DQ_WARP_CTA_BYTES_SMOOTH : DQ_WARP_CTA_BYTES_PLAIN;
-      int64_t groups = cta_bytes / (static_cast<int64_t>(stages) * stride);
-      const int64_t max_groups = dq::kWarpKernelMaxThreads / gs.tpr;
-      groups = groups < 1 ? 1 : (groups > max_groups ? max_groups : groups);
-      groups = groups > 15 ? 15 : groups;  // named barriers 1..15
-      a.groups = static_cast<int>(groups);
-      a.stages = stages;
-      a.stage_stride = stride;
+      a.stage_stride = static_cast<uint32_t>((row_bytes + 127) / 128 * 128);
       a.tpr = gs.tpr;
-      if (dq::dq_smem_bytes(a.groups, stages, stride, a.group_index ? a.num_groups : 0) <= kMaxDynamicSmem) {
+      {
         dq_status st;
         if (a.smooth == nullptr) {
           st = launch_dq_vpt<InT, MODE, OUT, dq::kSmNone>(a, gs.vpt, device, sms, stream);

@@ -62,6 +62,13 @@ constexpr int kBM = 128, kBK = 128;
 constexpr uint32_t kTileABytes = kBM * kBK;  // 16 KB
 constexpr int kThreads = 192;
 
+// Instruction descriptor of tcgen05.mma kind::i8 for an M = 128 x N tile:
+// int32 accumulator (format 2), signed A and B (format 1), both K-major,
+// N / 8 and M / 16.
+constexpr uint32_t i8_idesc(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+}
+
 template <int BN, int STAGES>
 struct TileConfig {
   static constexpr uint32_t kTileBBytes = BN * kBK;
@@ -69,10 +76,7 @@ struct TileConfig {
   static constexpr uint32_t kTmemCols = BN;  // one int32 accumulator column per output column
   // slack for 1024-byte alignment, ring, barriers, column scales
   static constexpr size_t kSmemBytes = 1024 + STAGES * kStageBytes + 256 + BN * 4;
-  // kind::i8: int32 accumulator (format 2), signed A and B (format 1), both
-  // K-major, N / 8 and M / 16.
-  static constexpr uint32_t kIdesc =
-      (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+  static constexpr uint32_t kIdesc = i8_idesc(BN);
 };
 
 struct W8A8Args {
@@ -105,6 +109,58 @@ __device__ __forceinline__ void store_out(const W8A8Args& a, int64_t e, float t)
     static_cast<__half*>(a.out)[e] = __float2half_rn(t);
   } else {
     static_cast<__nv_bfloat16*>(a.out)[e] = __float2bfloat16_rn(t);
+  }
+}
+
+// Epilogue of one 32-column chunk of one output row: out = float(acc) *
+// (a_scale[row] * b_scale[col]) (+ out), narrowed, with 16-byte stores when
+// the whole chunk is in range and rows start 16-byte aligned. `cs` holds the
+// chunk's 32 column scales.
+__device__ __forceinline__ void epilogue_chunk(const W8A8Args& a, int64_t row, int64_t c0, const uint32_t (&r)[32],
+                                               float sa_row, const float* cs) {
+  float t[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float scales = __fmul_rn(sa_row, cs[j]);
+    t[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
+  }
+  const int64_t e0 = row * a.n + c0;  // 32 consecutive outputs of this row
+  if (a.vec_out && c0 + 32 <= a.n) {
+    if (a.out_kind == 0) {
+      float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + e0);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float4 v = make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
+        if (a.accumulate) {
+          const float4 y = o[q];
+          v = make_float4(__fadd_rn(v.x, y.x), __fadd_rn(v.y, y.y), __fadd_rn(v.z, y.z), __fadd_rn(v.w, y.w));
+        }
+        o[q] = v;
+      }
+    } else {
+      uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + e0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float x0 = t[8 * q + 2 * h], x1 = t[8 * q + 2 * h + 1];
+          if (a.out_kind == 1) {
+            const __half2 p2 = __floats2half2_rn(x0, x1);
+            w[h] = *reinterpret_cast<const uint32_t*>(&p2);
+          } else {
+            const __nv_bfloat162 p2 = __floats2bfloat162_rn(x0, x1);
+            w[h] = *reinterpret_cast<const uint32_t*>(&p2);
+          }
+        }
+        o[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (c0 + j < a.n) store_out(a, e0 + j, t[j]);
+    }
   }
 }
 
@@ -158,6 +214,43 @@ __device__ __forceinline__ void tc_ld_32cols(uint32_t taddr, uint32_t (&r)[32]) 
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---------------------------------------------------------------- bounded waits
+
+__device__ __forceinline__ bool wait_or_abort_for(uint64_t* bar, uint32_t parity, const volatile uint32_t* abort,
+                                                  uint64_t limit_ns) {
+  const uint32_t addr = dq::smem_addr(bar);
+  if (dq::mbar_try_wait(addr, parity)) return true;
+  const uint64_t t0 = dq::global_ns();
+  while (true) {
+    if (dq::mbar_try_wait(addr, parity)) return true;
+    if (*abort != 0u || dq::global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Wait for an accumulator that the MMA lane is still building: gives up only
+// after kWaitLimitNs without the lane's stage counter `progress` moving (or
+// on the abort flag), so a long K loop that keeps moving is never cut off,
+// while a stuck one ends within the limit.
+__device__ __forceinline__ bool wait_while_progress(uint64_t* bar, uint32_t parity, const volatile uint32_t* abort,
+                                                    const volatile uint32_t* progress) {
+  const uint32_t addr = dq::smem_addr(bar);
+  if (dq::mbar_try_wait(addr, parity)) return true;
+  uint64_t t0 = dq::global_ns();
+  uint32_t seen = *progress;
+  while (true) {
+    if (dq::mbar_try_wait(addr, parity)) return true;
+    if (abort != nullptr && *abort != 0u) return false;
+    const uint32_t now_seen = *progress;
+    const uint64_t now = dq::global_ns();
+    if (now_seen != seen) {
+      seen = now_seen;
+      t0 = now;
+    } else if (now - t0 > dq::kWaitLimitNs) {
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- kernels
 
 template <int BN, int STAGES>
@@ -177,6 +270,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   uint64_t* acc_ready = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 1);
   volatile uint32_t* mma_failed = tmem_slot + 1;  // set when the MMA lane gave up on a stage
+  volatile uint32_t* mma_progress = tmem_slot + 2;  // stages the MMA lane has consumed
   float* col_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // the tile's b_scale
 
   const int warp = threadIdx.x >> 5;
@@ -192,6 +286,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
     }
     dq::mbar_init(acc_ready, 1);
     *mma_failed = 0u;
+    *mma_progress = 0u;
     dq::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -217,6 +312,11 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         const int s = kt % kStages;
         const uint32_t ph = static_cast<uint32_t>(kt / kStages) & 1u;
         if (!dq::mbar_wait_parity(empty + s, ph ^ 1u)) break;
+#if defined(DQ_TEST_SKIP_W8A8_TILE_M) && defined(DQ_TEST_SKIP_W8A8_KTILE)
+        // test builds only: leave one operand stage of one tile out, so that
+        // the MMA lane's bounded wait runs out and the failure path runs
+        if (blockIdx.y == DQ_TEST_SKIP_W8A8_TILE_M && blockIdx.x == 0 && kt == DQ_TEST_SKIP_W8A8_KTILE) continue;
+#endif
         dq::mbar_arrive_expect_tx(full + s, Cfg::kStageBytes);
         tma_load_2d(sa + s * kTileABytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
         tma_load_2d(sb + s * Cfg::kTileBBytes, &map_b, kt * kBK, static_cast<int>(n0), full + s);
@@ -248,21 +348,22 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
           tc_mma_i8(tmem, ad + 2 * kk, bd + 2 * kk, Cfg::kIdesc, (kt | kk) != 0 ? 1u : 0u);
         }
         tc_commit(empty + s);  // the stage is free once these MMAs have read it
+        *mma_progress = static_cast<uint32_t>(kt + 1);
       }
       tc_commit(acc_ready);  // every MMA issued above is complete when this arrives
       // this warp frees the TMEM below: it sees the MMAs complete itself, so
       // the accumulator is never released under MMAs still in flight (even
       // when the epilogue's wait has run out)
-      dq::mbar_wait_parity_for(acc_ready, 0, dq::kWaitLimitNs * (ktiles + 1));
+      dq::mbar_wait_parity(acc_ready, 0);
     }
   } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
     // the tile's column scales, staged once by the 128 epilogue threads
 #pragma unroll
     for (int j = threadIdx.x - 64; j < kBN; j += 128) col_scale[j] = n0 + j < a.n ? a.b_scale[n0 + j] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");
-    // the MMA lane may take up to one wait limit per stage: the epilogue's
-    // budget covers the whole K loop
-    const bool ready = dq::mbar_wait_parity_for(acc_ready, 0, dq::kWaitLimitNs * (ktiles + 1)) && *mma_failed == 0u;
+    // the MMA lane may take up to one wait limit per stage: the epilogue
+    // gives up only when the lane has stopped moving for that long
+    const bool ready = wait_while_progress(acc_ready, 0, nullptr, mma_progress) && *mma_failed == 0u;
     tc_fence_after();
     const int quarter = warp & 3;
     const int64_t row = m0 + 32 * quarter + lane;
@@ -281,50 +382,7 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
         }
         continue;
       }
-      float t[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float scales = __fmul_rn(sa_row, col_scale[32 * c + j]);
-        t[j] = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), scales);
-      }
-      const int64_t e0 = row * a.n + c0;  // 32 consecutive outputs of this row
-      if (a.vec_out && c0 + 32 <= a.n) {
-        if (a.out_kind == 0) {
-          float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + e0);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 v = make_float4(t[4 * q], t[4 * q + 1], t[4 * q + 2], t[4 * q + 3]);
-            if (a.accumulate) {
-              const float4 y = o[q];
-              v = make_float4(__fadd_rn(v.x, y.x), __fadd_rn(v.y, y.y), __fadd_rn(v.z, y.z), __fadd_rn(v.w, y.w));
-            }
-            o[q] = v;
-          }
-        } else {
-          uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + e0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float x0 = t[8 * q + 2 * h], x1 = t[8 * q + 2 * h + 1];
-              if (a.out_kind == 1) {
-                const __half2 p2 = __floats2half2_rn(x0, x1);
-                w[h] = *reinterpret_cast<const uint32_t*>(&p2);
-              } else {
-                const __nv_bfloat162 p2 = __floats2bfloat162_rn(x0, x1);
-                w[h] = *reinterpret_cast<const uint32_t*>(&p2);
-              }
-            }
-            o[q] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (c0 + j < a.n) store_out(a, e0 + j, t[j]);
-        }
-      }
+      epilogue_chunk(a, row, c0, r, sa_row, col_scale + 32 * c);
     }
   }
 
@@ -333,6 +391,224 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- persistent kernel
+
+// One CTA per SM walks a list of output tiles: 128 x 256 tiles first, then the
+// last r of them split into two 128 x 128 tiles each, when that evens out the
+// SMs (every SM gets q wide tiles, 2r <= SMs of them one narrow tile: the
+// last wave is half as long). The ring is 4 stages of 48 KB; the int32
+// accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of
+// one tile overlaps the MMAs of the next.
+#ifndef DQ_W8A8_PSTAGES
+#define DQ_W8A8_PSTAGES 4
+#endif
+constexpr int kPStages = DQ_W8A8_PSTAGES;
+constexpr uint32_t kPTileBBytes = 256 * kBK;                     // 32 KB (a narrow tile uses 16)
+constexpr uint32_t kPStageBytes = kTileABytes + kPTileBBytes;   // 48 KB
+constexpr uint32_t kPTmemCols = 512;
+// ring, barriers and flags (256 B), two buffers of 256 column scales
+constexpr size_t kPSmemBytes = 1024 + kPStages * kPStageBytes + 256 + 2 * 256 * 4;
+constexpr uint32_t kIdescN256 = i8_idesc(256);
+constexpr uint32_t kIdescN128 = i8_idesc(128);
+
+struct PersistSched {
+  int64_t n_tiles;  // 256-wide column tiles
+  int64_t wide;     // list items that are whole 128 x 256 tiles
+  int64_t items;    // wide + 2 * (tiles split in two)
+};
+
+__device__ __forceinline__ void decode_item(const PersistSched& ps, int64_t item, int64_t& m0, int64_t& n0,
+                                            bool& wide) {
+  int64_t t, half = 0;
+  if (item < ps.wide) {
+    t = item;
+    wide = true;
+  } else {
+    t = ps.wide + (item - ps.wide) / 2;
+    half = (item - ps.wide) & 1;
+    wide = false;
+  }
+  m0 = (t / ps.n_tiles) * kBM;
+  n0 = (t % ps.n_tiles) * 256 + half * 128;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+w8a8_gemm_persistent_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b256,
+                            const __grid_constant__ CUtensorMap map_b128, const W8A8Args a, const PersistSched ps) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sa = smem;                                   // kPStages x 16 KB (A tiles)
+  uint8_t* sb = smem + kPStages * kTileABytes;          // kPStages x 32 KB (B tiles)
+  uint64_t* full = reinterpret_cast<uint64_t*>(sb + kPStages * kPTileBBytes);
+  uint64_t* empty = full + kPStages;
+  uint64_t* acc_full = empty + kPStages;   // [2]: the accumulator holds a finished tile
+  uint64_t* acc_empty = acc_full + 2;      // [2]: the epilogue has read it out
+  uint64_t* mma_done = acc_empty + 2;      // every MMA this CTA issued has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile uint32_t* mma_progress = tmem_slot + 2;  // stages the MMA lane has consumed
+  float* col_scale = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // [2][256]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ktiles = static_cast<int>((a.k + kBK - 1) / kBK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      dq::mbar_init(full + s, 1);
+      dq::mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      dq::mbar_init(acc_full + b, 1);
+      dq::mbar_init(acc_empty + b, 4);  // one arrival per epilogue warp
+    }
+    dq::mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    *mma_progress = 0u;
+    dq::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dq::smem_addr(tmem_slot)),
+                 "r"(kPTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // launched as a programmatic dependent: the codes may come from the
+  // previous kernel, so no global memory is read before this
+  asm volatile("griddepcontrol.launch_dependents;");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  if (warp == 0) {
+    if (lane == 0) {  // producer
+      uint32_t slice = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; ok && item < ps.items; item += gridDim.x) {
+        int64_t m0, n0;
+        bool wide;
+        decode_item(ps, item, m0, n0, wide);
+        for (int kt = 0; kt < ktiles; ++kt, ++slice) {
+          const int s = static_cast<int>(slice % kPStages);
+          const uint32_t ph = (slice / kPStages) & 1u;
+          if (!wait_or_abort_for(empty + s, ph ^ 1u, abort_flag, dq::kWaitLimitNs)) {
+            *abort_flag = 1u;
+            ok = false;
+            break;
+          }
+#if defined(DQ_TEST_SKIP_W8A8_TILE_M) && defined(DQ_TEST_SKIP_W8A8_KTILE)
+          // test builds only: leave one operand stage of one tile out, so that
+          // the MMA lane's bounded wait runs out and the failure path runs
+          if (m0 == int64_t(kBM) * DQ_TEST_SKIP_W8A8_TILE_M && n0 == 0 && kt == DQ_TEST_SKIP_W8A8_KTILE) continue;
+#endif
+          dq::mbar_arrive_expect_tx(full + s, kTileABytes + (wide ? kPTileBBytes : kPTileBBytes / 2));
+          tma_load_2d(sa + s * kTileABytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
+          tma_load_2d(sb + s * kPTileBBytes, wide ? &map_b256 : &map_b128, kt * kBK, static_cast<int>(n0), full + s);
+        }
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (uint32_t j = slice > kPStages ? slice - kPStages : 0; j < slice; ++j) {
+        dq::mbar_wait_parity(full + j % kPStages, (j / kPStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      uint32_t slice = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t item = blockIdx.x; ok && item < ps.items; item += gridDim.x, ++i) {
+        int64_t m0, n0;
+        bool wide;
+        decode_item(ps, item, m0, n0, wide);
+        const int acc = i & 1;
+        if (!wait_or_abort_for(acc_empty + acc, ((i >> 1) & 1) ^ 1u, abort_flag, dq::kWaitLimitNs)) {
+          *abort_flag = 1u;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * 256);
+        const uint32_t idesc = wide ? kIdescN256 : kIdescN128;
+        for (int kt = 0; kt < ktiles; ++kt, ++slice) {
+          const int s = static_cast<int>(slice % kPStages);
+          const uint32_t ph = (slice / kPStages) & 1u;
+          if (!wait_or_abort_for(full + s, ph, abort_flag, dq::kWaitLimitNs)) {
+            *abort_flag = 1u;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_k_sw128(sa + s * kTileABytes);
+          const uint64_t bd = smem_desc_k_sw128(sb + s * kPTileBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 32; ++kk) {
+            tc_mma_i8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kt | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(empty + s);
+          *mma_progress = slice + 1;
+        }
+        if (ok) tc_commit(acc_full + acc);
+      }
+      // this warp frees the TMEM below: it sees every MMA it issued complete
+      tc_commit(mma_done);
+      dq::mbar_wait_parity(mma_done, 0);
+    }
+  } else {  // epilogue: warps 2..5 cover TMEM lane quarters (warp % 4)
+    const int quarter = warp & 3;
+    const int et = threadIdx.x - 64;
+    bool dead = false;
+    int i = 0;
+    for (int64_t item = blockIdx.x; item < ps.items; item += gridDim.x, ++i) {
+      int64_t m0, n0;
+      bool wide;
+      decode_item(ps, item, m0, n0, wide);
+      const int bn = wide ? 256 : 128;
+      const int acc = i & 1;
+      float* cs = col_scale + acc * 256;
+      for (int j = et; j < bn; j += 128) cs[j] = n0 + j < a.n ? a.b_scale[n0 + j] : 0.0f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!dead) dead = !wait_while_progress(acc_full + acc, (i >> 1) & 1, abort_flag, mma_progress);
+      // lanes can see a wait's deadline differently: the warp agrees, so the
+      // collective TMEM loads below are taken by all of its lanes or none
+      dead = __any_sync(0xffffffffu, dead);
+      tc_fence_after();
+      const int64_t row = m0 + 32 * quarter + lane;
+      const bool row_ok = row < a.m;
+      const float sa_row = row_ok ? a.a_scale[row] : 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < bn / 32; ++c) {
+        const int64_t c0 = n0 + 32 * c;
+        if (c0 >= a.n) break;  // warp-uniform
+        if (dead) {  // a wait ran out in this CTA: NaN marks this and its remaining tiles
+          if (row_ok) {
+            for (int j = 0; j < 32; ++j) {
+              if (c0 + j < a.n) store_nan(a, row * a.n + c0 + j);
+            }
+          }
+          continue;
+        }
+        uint32_t r[32];
+        tc_ld_32cols(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(acc * 256 + 32 * c),
+                     r);
+        if (row_ok) epilogue_chunk(a, row, c0, r, sa_row, cs + 32 * c);
+      }
+      if (dead) *abort_flag = 1u;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dq::mbar_arrive(acc_empty + acc);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPTmemCols) : "memory");
   }
 }
 
@@ -442,6 +718,39 @@ dq_status launch_tc(const W8A8Args& args, int device, cudaStream_t stream) {
                     static_cast<unsigned>((args.m + kBM - 1) / kBM)), kThreads, Cfg::kSmemBytes, stream, ma, mb, args);
 }
 
+// Persistent launch: one CTA per SM over the tile list (see
+// w8a8_gemm_persistent_kernel); kNotLaunchable when the tensor maps or the
+// shared-memory opt-in are unavailable.
+dq_status launch_persistent(const W8A8Args& args, int device, cudaStream_t stream) {
+  CUtensorMap ma, mb256, mb128;
+  if (!make_map(&ma, args.a, args.m, args.k, kBM) || !make_map(&mb256, args.b, args.n, args.k, 256) ||
+      !make_map(&mb128, args.b, args.n, args.k, 128))
+    return kNotLaunchable;
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  static int sms[kMaxDevices];
+  if (device < 0 || device >= kMaxDevices) return kNotLaunchable;
+  std::call_once(once[device], [device] {
+    ok[device] = cudaFuncSetAttribute(w8a8_gemm_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(kPSmemBytes)) == cudaSuccess &&
+                 cudaDeviceGetAttribute(&sms[device], cudaDevAttrMultiProcessorCount, device) == cudaSuccess &&
+                 sms[device] > 0;
+    if (!ok[device]) cudaGetLastError();
+  });
+  if (!ok[device]) return kNotLaunchable;
+  const int64_t P = sms[device];
+  PersistSched ps;
+  ps.n_tiles = (args.n + 255) / 256;
+  const int64_t T = ((args.m + kBM - 1) / kBM) * ps.n_tiles;
+  const int64_t r = T % P;  // tiles of the last, partial wave
+  const int64_t split = 2 * r <= P ? r : 0;  // halve them when every half gets its own SM
+  ps.wide = T - split;
+  ps.items = T + split;
+  const int64_t grid = ps.items < P ? ps.items : P;
+  return launch_pdl(w8a8_gemm_persistent_kernel, dim3(static_cast<unsigned>(grid)), kThreads, kPSmemBytes, stream,
+                    ma, mb256, mb128, args, ps);
+}
+
 }  // namespace
 
 extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, int64_t n, int64_t k,
@@ -467,6 +776,10 @@ extern "C" dq_status dq_w8a8_gemm(const int8_t* a, const int8_t* b, int64_t m, i
   const bool tiles = k % 16 == 0 && (m + kBM - 1) / kBM <= 65535 && aligned_to(a, 16) && aligned_to(b, 16);
   if (tiles) {
     const int device = current_device();
+#ifndef DQ_W8A8_NO_PERSISTENT
+    const dq_status pst = launch_persistent(args, device, stream);
+    if (pst != kNotLaunchable) return pst;
+#endif
     // 256-wide tiles unless a 128-wide last tile would waste less
     if (DQ_W8A8_BN >= 256 && (n % 256 == 0 || n % 256 > 128)) {
       const dq_status st = launch_tc<256, DQ_W8A8_STAGES_256>(args, device, stream);
