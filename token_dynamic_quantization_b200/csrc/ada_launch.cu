@@ -36,8 +36,8 @@ constexpr size_t kAdaRingSmemBudget = 232448 - 2048;
 #define DQ_ADA_RING_MAX_SLOTS 32
 #endif
 
-// Ring kernel launch: one CTA per SM (fewer for few rows), NC consumer groups
-// of G warps (as many as the registers allow, at most 15 with G > 1), the
+// Ring kernel launch: one CTA per SM (fewer for few rows), NC row groups of G
+// warps (as many as the kernel's largest block holds, at most 15 with G > 1), the
 // table rows of the CTA's batches staged when they fit DQ_ADA_TABLE_BUDGET,
 // NS row slots in the rest of the shared memory.
 template <typename InT, int VPT, bool kRagged, bool kStaged>
@@ -45,14 +45,12 @@ dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batc
   void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_ring_kernel<InT, VPT, kRagged, kStaged>;
   const void* k = reinterpret_cast<const void*>(kfn);
   if (!allow_smem_bytes(k, device, kAdaRingSmemBudget)) return kNotLaunchable;
-  const int regs = kernel_registers(k, device);
-  if (regs <= 0) return kNotLaunchable;
+  const int max_threads = kernel_max_threads(k, device);
   const int G = a.tpr / 32;
   const int64_t rows = a.batch * a.seq;
   const int64_t grid = rows < sms ? rows : sms;
   const int64_t per_cta = (rows + grid - 1) / grid;
-  int64_t nc = (65536 / (32 * ((regs + 7) / 8 * 8)) - 1) / G;
-  if (nc > (dq::kRingMaxThreads / 32 - 1) / G) nc = (dq::kRingMaxThreads / 32 - 1) / G;
+  int64_t nc = max_threads / a.tpr;
   if (G > 1 && nc > 15) nc = 15;
   if (nc > per_cta) nc = per_cta;
   a.table_batches = kStaged ? static_cast<int>(table_batches) : 0;
@@ -66,7 +64,7 @@ dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batc
   a.groups = static_cast<int>(nc);
   a.stages = static_cast<int>(ns);
   const size_t smem = dq::ada_ring_smem_bytes(a.stages, a.stage_stride, a.table_batches, a.hidden);
-  const int block = 32 + a.tpr * a.groups;
+  const int block = a.tpr * a.groups;
   if (blocks_per_sm(k, block, smem, device) < 1) return kNotLaunchable;
   dq_status st = launch_ada_table(a, sms, stream);
   if (st != DQ_OK) return st;
@@ -92,24 +90,21 @@ dq_status launch_ada_ragged(dq::AdaArgs a, int device, int sms, cudaStream_t str
                 : launch_ada_ring<InT, VPT, true, false>(a, device, sms, nb, stream);
 }
 
-// AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8}, fewest wasted lanes,
-// then VPT closest to DQ_ADA_TARGET_VPT (more elements per thread amortize the
-// row reductions; the row share stays in registers).
-#ifndef DQ_ADA_TARGET_VPT
-#define DQ_ADA_TARGET_VPT 6  // hidden 3072: 2 warps x 6 vectors per row
-#endif
-
+// AdaLayerNorm row-group shape: VPT in {2, 3, 4, 6, 8, 12}, fewest wasted
+// lanes, then the fewest warps per row. The per-row work (three row
+// reductions, the row statistics and constants) is repeated by every warp of
+// a row, and one warp per row needs no cross-warp combine: hidden 3072 runs
+// one warp of 12 vectors per lane.
 GroupShape pick_ada_shape(int64_t nvec) {
   GroupShape best{0, 0};
   double best_eff = -1.0;
-  static const int kVpts[5] = {2, 3, 4, 6, 8};
+  static const int kVpts[6] = {2, 3, 4, 6, 8, 12};
   for (int vpt : kVpts) {
     const int64_t warps = (nvec + 32 * vpt - 1) / (32 * vpt);
     if (warps > 16) continue;
     const int64_t tpr = warps * 32;
     const double eff = static_cast<double>(nvec) / static_cast<double>(tpr * vpt);
-    const bool better = eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && std::abs(vpt - DQ_ADA_TARGET_VPT) <
-                                                                             std::abs(best.vpt - DQ_ADA_TARGET_VPT));
+    const bool better = eff > best_eff + 1e-9 || (eff > best_eff - 1e-9 && tpr <= best.tpr);
     if (better) {
       best_eff = eff;
       best = GroupShape{vpt, static_cast<int>(tpr)};
@@ -134,7 +129,8 @@ dq_status launch_ada(dq::AdaArgs a, bool vector_ok, cudaStream_t stream) {
           case 3: st = launch_ada_ragged<InT, 3>(a, device, sms, stream); break;
           case 4: st = launch_ada_ragged<InT, 4>(a, device, sms, stream); break;
           case 6: st = launch_ada_ragged<InT, 6>(a, device, sms, stream); break;
-          default: st = launch_ada_ragged<InT, 8>(a, device, sms, stream); break;
+          case 8: st = launch_ada_ragged<InT, 8>(a, device, sms, stream); break;
+          default: st = launch_ada_ragged<InT, 12>(a, device, sms, stream); break;
         }
         if (st != kNotLaunchable) return st;
       }

@@ -3,15 +3,15 @@
 //
 // The row kernel of the fused path, on the structure of the DynamicQuant ring
 // kernel (dynamic_quant_ring.cuh): one persistent CTA per SM owns a
-// contiguous range of rows; warp 0 lane 0 streams them with cp.async.bulk
-// into a CTA-wide ring of NS slots; NC consumer groups of G warps take rows
-// c, c + NC, ... and release each slot as soon as its row is in registers.
+// contiguous range of rows and a CTA-wide ring of NS slots filled with
+// cp.async.bulk; NC row groups of G warps take rows c, c + NC, ..., and the
+// last warp of a group to have its row in registers refills the slot.
 // The folded affine table (A, B per batch and column, written by
 // ada_affine_table_kernel) is staged in shared memory for the batches the
 // CTA's rows belong to, so the per-element reads of steps 1-3 are shared
 // loads instead of L1/L2 loads on every row.
 //
-// Arithmetic per row, as in ada_layernorm_quant_tma_kernel: both moments of
+// Arithmetic per row: both moments of
 // d = x - K (K the mean of the row's first 8 elements) from one reduction,
 // fp32 partial sums per thread and warp, double across warps, a centred second
 // pass for rows whose first elements sit far from the mean; then
@@ -20,7 +20,8 @@
 //
 // Failure handling as in the DynamicQuant ring kernel: every wait is bounded
 // in time and gives up on the shared abort flag; a group whose row never
-// arrives writes NaN quant scales for its remaining rows and stops.
+// arrives writes NaN quant scales for its remaining rows and stops, and the
+// CTA waits (bounded) for its copies in flight before it exits.
 #pragma once
 
 #include "ada_layernorm_quant_kernels.cuh"
@@ -31,7 +32,8 @@
 namespace dq {
 
 // Shared memory of the AdaLN ring kernel: NS row slots of `stride` bytes;
-// full[NS], empty[NS]; a 16-byte abort word; then, when staged,
+// full[NS] mbarriers; per slot a release counter and the fill round of its
+// last copy; a 16-byte abort word; then, when staged,
 // A[table_batches][hidden] and B[table_batches][hidden] (fp32).
 __host__ __device__ inline size_t ada_ring_smem_bytes(int slots, uint32_t stride, int table_batches, int64_t hidden) {
   return static_cast<size_t>(slots) * stride + static_cast<size_t>(slots) * 16 + 16 +
@@ -55,9 +57,10 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   const int NC = a.groups;
   const int64_t H = a.hidden;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * stride);
-  uint64_t* empty = full + NS;
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + NS);
-  float* table_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(empty + NS) + 16);
+  uint32_t* rel_count = reinterpret_cast<uint32_t*>(full + NS);      // warps of the group done with the slot
+  int32_t* last_round = reinterpret_cast<int32_t*>(rel_count + NS);  // fill round of the slot's last copy
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(last_round + NS);
+  float* table_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(last_round + NS) + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -69,35 +72,31 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, static_cast<uint32_t>(G));
+      rel_count[s] = 0u;
+      last_round[s] = -1;
     }
     *abort_flag = 0u;
     fence_mbarrier_init();
   }
 
-  // Producer state (thread 0). The first NS copies go out before the wait for
-  // the table kernel: that kernel waited for the work before it before it let
-  // this one start, so x is already final.
-  int issued = 0;
-  const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
-  uint64_t policy = 0;
-  auto issue = [&](int s) {
+  // local row j of the CTA into slot s (= j % NS), completing full[s]
+  const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  const uint64_t policy = l2_evict_first_policy();
+  auto issue = [&](int s, int j) {
+    last_round[s] = j / NS;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out (see dynamic_quant_ring.cuh)
-    if (r_begin + issued == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) {
-      x_next += row_bytes;
-      ++issued;
-      return;
-    }
+    if (r_begin + j == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) return;
 #endif
     mbar_arrive_expect_tx(full + s, row_bytes);
-    bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_next, row_bytes, full + s, policy);
-    x_next += row_bytes;
-    ++issued;
+    bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes,
+                  full + s, policy);
   };
-  if (threadIdx.x == 0 && n > 0) {
-    policy = l2_evict_first_policy();
-    while (issued < NS && issued < n) issue(issued);
+  // The whole ring goes out before the wait for the table kernel: that kernel
+  // waited for the work before it before it let this one start, so x is
+  // already final.
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < NS && j < n; ++j) issue(j, j);
   }
   pdl_wait_primary();  // the affine table is complete and visible from here on
   pdl_launch_dependents();
@@ -119,36 +118,11 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   __syncthreads();
   if (n <= 0) return;
 
-  // ------------------------------------------------------------ producer
-  if (warp == 0) {
-    if (lane != 0) return;
-    int s = issued % NS;
-    uint32_t k = static_cast<uint32_t>(issued / NS);
-    while (issued < n) {
-      if (!mbar_wait_parity_or_abort(empty + s, (k - 1u) & 1u, abort_flag)) {
-        *abort_flag = 1u;
-        break;
-      }
-      fence_proxy_async_smem();
-      issue(s);
-      if (++s == NS) {
-        s = 0;
-        ++k;
-      }
-    }
-    for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
-      mbar_wait_parity(full + (j % NS), static_cast<uint32_t>(j / NS) & 1u);
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int cw = warp - 1;
-  const int c = cw / G;
-  const int wg = cw - c * G;
+  // ------------------------------------------------------------ row groups
+  const int c = warp / G;
+  const int wg = warp - c * G;
   const int lane_g = wg * 32 + lane;
-  const int warp_g0 = 1 + c * G;
-  if (c >= NC || c >= n) return;
+  const int warp_g0 = c * G;
   const int nvec = static_cast<int>(H >> 3);
   const int vbase = wg * (32 * VPT) + lane;
   auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
@@ -167,7 +141,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   const float4* B4 = nullptr;
   int8_t* orow = a.out + (r_begin + c) * H;
   const int64_t o_step = H * NC;
-  for (int j = c; j < n; j += NC, orow += o_step) {
+  for (int j = c; j < n && c < NC; j += NC, orow += o_step) {
     const int64_t r = r_begin + j;
     if (r >= b_end) {
       b = r / a.seq;
@@ -220,8 +194,20 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
       s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
     }
+    // the group's last warp to get here refills the slot with the row NS on
     __syncwarp();
-    if (ok && lane == 0) mbar_arrive(empty + s);
+    if (lane == 0) {
+      bool last = true;
+      if (G > 1) {
+        __threadfence_block();
+        last = atomicAdd(rel_count + s, 1u) == static_cast<uint32_t>(G - 1);
+        if (last) rel_count[s] = 0u;
+      }
+      if (last && ok && j + NS < n) {
+        fence_proxy_async_smem();
+        issue(s, j + NS);
+      }
+    }
     s += NC;
     if (s >= NS) {
       s -= NS;
@@ -247,7 +233,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     if (failed) {
       *abort_flag = 1u;
       for (int jj = j + lane_g * NC; jj < n; jj += tpr * NC) a.quant_scale[r_begin + jj] = __int_as_float(0x7fc00000);
-      return;
+      break;
     }
     const double m1 = sum * a.inv_hidden;  // E(d)
     const double m2 = sq * a.inv_hidden;   // E(d^2)
@@ -347,6 +333,14 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       uint32_t bits[8];
       quant8<false, false>(v[k], q, -127.0f, 127.0f, bits);
       __stcs(ov + 32 * k, pack8_int8(bits));
+    }
+  }
+  // after a failed wait, wait (bounded) for every slot's last copy before the
+  // CTA's shared memory is released; on the normal path all were consumed
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag != 0u) {
+    for (int t = 0; t < NS; ++t) {
+      if (last_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(last_round[t]) & 1u);
     }
   }
 }

@@ -120,27 +120,28 @@ inline bool allow_smem_bytes(const void* kernel, int device, size_t bytes) {
   return true;
 }
 
-// Registers per thread of a compiled kernel (0 if unknown); cached.
-inline int kernel_registers(const void* kernel, int device) {
+// Largest block a compiled kernel can be launched with (its registers per
+// thread, rounded as the hardware allocates them; 0 if unknown); cached.
+inline int kernel_max_threads(const void* kernel, int device) {
   struct Entry {
     const void* k;
     int device;
-    int regs;
+    int threads;
   };
   static Entry cache[512];
   static int used = 0;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
   for (int i = 0; i < used; ++i) {
-    if (cache[i].k == kernel && cache[i].device == device) return cache[i].regs;
+    if (cache[i].k == kernel && cache[i].device == device) return cache[i].threads;
   }
   cudaFuncAttributes attr{};
   if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
-  if (used < 512) cache[used++] = Entry{kernel, device, attr.numRegs};
-  return attr.numRegs;
+  if (used < 512) cache[used++] = Entry{kernel, device, attr.maxThreadsPerBlock};
+  return attr.maxThreadsPerBlock;
 }
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }

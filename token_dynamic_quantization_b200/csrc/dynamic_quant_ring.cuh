@@ -2,20 +2,20 @@
 // and "Description"), sm_100a.
 //
 // One persistent CTA per SM owns a contiguous range of rows and one ring of
-// NS shared-memory row slots:
-//   * warp 0, lane 0 is the producer: it streams the CTA's rows in order into
-//     the ring with cp.async.bulk (TMA) copies, each completing the slot's
-//     `full` mbarrier (transaction count), and refills a slot as soon as its
-//     `empty` mbarrier says every warp of the consuming group has read it.
-//     At launch it issues NS copies at once, so the CTA's first rows are in
-//     flight before any consumer starts.
-//   * the other warps form C consumer groups of G warps; group c takes the
-//     CTA's local rows c, c + C, c + 2C, ... A group reads its row once from
-//     the slot into registers (pass 1: widen, multiply by the smooth scales,
-//     reduce), releases the slot, combines the warps' partial reductions,
-//     derives the row constants and quantizes from registers (pass 2).
+// NS shared-memory row slots; local row j lives in slot j % NS.
+//   * At launch, thread 0 issues NS cp.async.bulk (TMA) copies at once, each
+//     completing its slot's `full` mbarrier (transaction count), so the
+//     CTA's first NS rows are in flight before any row is processed.
+//   * The warps form NC row groups of G warps; group c takes the CTA's rows
+//     c, c + NC, c + 2NC, ... A group reads its row once from the slot into
+//     registers (pass 1: widen, multiply by the smooth scales, reduce). The
+//     last of its warps to finish reading (a shared-memory counter) refills
+//     the slot at once with the row NS further on. The group then combines
+//     its warps' partial reductions, derives the row constants and quantizes
+//     from registers (pass 2).
 // Because the slots are shared by the whole CTA, copies run ahead of every
-// group by up to NS rows, independently of which group is slowest.
+// group by up to NS rows, independently of which group is slowest, and no
+// warp is set aside for issuing copies.
 //
 // Dense smooth-scale tables are staged once per CTA in shared memory; MoE
 // tables (one row per expert) are read through L1.
@@ -23,8 +23,9 @@
 // Failure handling: every wait is bounded in time (tma_pipeline.cuh) and also
 // gives up when a shared abort flag is set. A group whose row copy never
 // completes writes NaN scales for its remaining rows, sets the flag and
-// stops; the producer stops issuing, waits (bounded) for the copies it has in
-// flight, and the CTA exits. No thread waits forever.
+// stops; the other groups stop at their next row that has not landed; before
+// the CTA exits, thread 0 waits (bounded) for every slot's last copy. No
+// thread waits forever.
 #pragma once
 
 #include "dq_args.cuh"
@@ -35,8 +36,9 @@
 namespace dq {
 
 // Shared memory of the ring kernel, in this order: NS row slots of `stride`
-// bytes; full[NS] and empty[NS] mbarriers; a 16-byte abort word; the staged
-// smooth table (`smooth_bytes`, a multiple of 16); the MoE group index.
+// bytes; full[NS] mbarriers; per slot a release counter and the fill round
+// of its last copy; a 16-byte abort word; the staged smooth table
+// (`smooth_bytes`, a multiple of 16); the MoE group index.
 __host__ __device__ inline size_t ring_smem_bytes(int slots, uint32_t stride, size_t smooth_bytes, int num_groups) {
   return static_cast<size_t>(slots) * stride + static_cast<size_t>(slots) * 16 + 16 + smooth_bytes +
          static_cast<size_t>(num_groups) * 4;
@@ -79,9 +81,10 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   const int G = tpr >> 5;
   const int NC = a.groups;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * stride);
-  uint64_t* empty = full + NS;
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + NS);
-  uint8_t* smooth_s = reinterpret_cast<uint8_t*>(empty + NS) + 16;
+  uint32_t* rel_count = reinterpret_cast<uint32_t*>(full + NS);  // warps of the group done with the slot
+  int32_t* last_round = reinterpret_cast<int32_t*>(rel_count + NS);  // fill round of the slot's last copy
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(last_round + NS);
+  uint8_t* smooth_s = reinterpret_cast<uint8_t*>(last_round + NS) + 16;
   const size_t smooth_bytes = kSmemSmooth ? static_cast<size_t>(a.cols) * kSmoothElem : 0;
   int32_t* gi_s = reinterpret_cast<int32_t*>(smooth_s + smooth_bytes);
 
@@ -95,7 +98,8 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, static_cast<uint32_t>(G));
+      rel_count[s] = 0u;
+      last_round[s] = -1;
     }
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -105,28 +109,23 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   pdl_launch_dependents();
   pdl_wait_primary();
 
-  // producer state (thread 0): the first NS copies go out before anything else
-  int issued = 0;
-  const uint8_t* x_next = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
-  uint64_t policy = 0;
-  auto issue = [&](int s) {
+  // local row j of the CTA into slot s (= j % NS), completing full[s]
+  const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  const uint64_t policy = l2_evict_first_policy();
+  auto issue = [&](int s, int j) {
+    last_round[s] = j / NS;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out, so that its consumer's
     // bounded wait runs out and the failure path runs
-    if (r_begin + issued == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) {
-      x_next += row_bytes;
-      ++issued;
-      return;
-    }
+    if (r_begin + j == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) return;
 #endif
     mbar_arrive_expect_tx(full + s, row_bytes);
-    bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_next, row_bytes, full + s, policy);
-    x_next += row_bytes;
-    ++issued;
+    bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes,
+                  full + s, policy);
   };
-  if (threadIdx.x == 0 && n > 0) {
-    policy = l2_evict_first_policy();
-    while (issued < NS && issued < n) issue(issued);
+  // the whole ring is in flight before anything else
+  if (threadIdx.x == 0) {
+    for (int j = 0; j < NS && j < n; ++j) issue(j, j);
   }
   if (kSmemSmooth) {
     const uint4* src = static_cast<const uint4*>(a.smooth);
@@ -140,39 +139,11 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   write_group_status(a);
   if (n <= 0) return;
 
-  // ------------------------------------------------------------ producer
-  if (warp == 0) {
-    if (lane != 0) return;
-    int s = issued % NS;
-    uint32_t k = static_cast<uint32_t>(issued / NS);  // fill round of row `issued`
-    while (issued < n) {
-      // slot s was last filled in round k - 1; its consumers released it
-      if (!mbar_wait_parity_or_abort(empty + s, (k - 1u) & 1u, abort_flag)) {
-        *abort_flag = 1u;
-        break;
-      }
-      fence_proxy_async_smem();
-      issue(s);
-      if (++s == NS) {
-        s = 0;
-        ++k;
-      }
-    }
-    // before the CTA can exit, every copy it issued must have landed (on the
-    // normal path the consumers have already seen them all)
-    for (int j = issued - 1; j >= 0 && j >= issued - NS; --j) {
-      mbar_wait_parity(full + (j % NS), static_cast<uint32_t>(j / NS) & 1u);
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int cw = warp - 1;             // consumer warp index
-  const int c = cw / G;                // group
-  const int wg = cw - c * G;           // warp within the group
+  // ------------------------------------------------------------ row groups
+  const int c = warp / G;              // group
+  const int wg = warp - c * G;         // warp within the group
   const int lane_g = wg * 32 + lane;   // thread within the group
-  const int warp_g0 = 1 + c * G;       // first warp of the group
-  if (c >= NC || c >= n) return;
+  const int warp_g0 = c * G;           // first warp of the group
   const int nvec = static_cast<int>(a.cols >> 3);
   const int vbase = wg * (32 * VPT) + lane;  // this thread's vector k is vbase + 32 * k
   auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
@@ -188,7 +159,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   int s = c;           // slot of local row j (NC <= NS)
   uint32_t par = 0u;   // parity of its fill round
   int parity = 0;      // red[] buffer
-  for (int j = c; j < n; j += NC, yrow += y_step) {
+  for (int j = c; j < n && c < NC; j += NC, yrow += y_step) {
     const int64_t r = r_begin + j;
     const bool ok = mbar_wait_parity_or_abort(full + s, par, abort_flag);
     const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
@@ -282,9 +253,21 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
     m0 = warp_max(m0);
     if (kA) m1 = warp_min(m1);
     // every lane's shared loads of the slot are complete (their values fed the
-    // warp reduction): release the slot for the producer's next copy
+    // warp reduction): the group's last warp to get here refills the slot
+    // with the row NS further on
     __syncwarp();
-    if (ok && lane == 0) mbar_arrive(empty + s);
+    if (lane == 0) {
+      bool last = true;
+      if (G > 1) {
+        __threadfence_block();
+        last = atomicAdd(rel_count + s, 1u) == static_cast<uint32_t>(G - 1);
+        if (last) rel_count[s] = 0u;
+      }
+      if (last && ok && j + NS < n) {
+        fence_proxy_async_smem();
+        issue(s, j + NS);
+      }
+    }
     s += NC;  // slot and fill round of local row j + NC (NC <= NS)
     if (s >= NS) {
       s -= NS;
@@ -309,10 +292,10 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
     if (failed) {
       // A row copy never completed (not a data-dependent condition): mark this
       // and the group's remaining rows with NaN scales and stop; the abort
-      // flag stops the producer and the other groups.
+      // flag stops the other groups at their next row that has not landed.
       *abort_flag = 1u;
       for (int jj = j + lane_g * NC; jj < n; jj += tpr * NC) a.scale[r_begin + jj] = __int_as_float(0x7fc00000);
-      return;
+      break;
     }
 
     RowQuant q = kA ? make_asym<C::kDivisor, C::kOffsetOptInt>(m0, m1) : make_sym<C::kDivisor>(m0);
@@ -385,6 +368,15 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
       pass2(BoolTag<true>{});
     } else {
       pass2(BoolTag<false>{});
+    }
+  }
+  // After a failed wait, copies issued for rows that nobody consumed may still
+  // be landing: wait (bounded) for every slot's last copy before the CTA's
+  // shared memory is released. On the normal path every copy was consumed.
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag != 0u) {
+    for (int t = 0; t < NS; ++t) {
+      if (last_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(last_round[t]) & 1u);
     }
   }
 }

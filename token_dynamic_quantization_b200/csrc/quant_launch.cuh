@@ -56,8 +56,8 @@ constexpr size_t kRingSmemBudget = 232448 - 1024;
 #define DQ_RING_MAX_SLOTS 32
 #endif
 
-// Ring kernel launch: one CTA per SM (fewer for few rows), NC consumer groups
-// of G = tpr / 32 warps, as many as the kernel's registers allow (at most 15
+// Ring kernel launch: one CTA per SM (fewer for few rows), NC row groups of
+// G = tpr / 32 warps, as many as the kernel's largest block holds (at most 15
 // with G > 1: one named barrier each), and NS row slots filling the shared
 // memory (NC <= NS <= rows of a CTA).
 template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged, bool kSS>
@@ -65,13 +65,11 @@ dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t s
   void (*kfn)(const dq::RowQuantArgs) = dq::dynamic_quant_ring_kernel<InT, MODE, OUT, SMK, VPT, kRagged, kSS>;
   const void* k = reinterpret_cast<const void*>(kfn);
   if (!allow_smem_bytes(k, device, kRingSmemBudget)) return kNotLaunchable;
-  const int regs = kernel_registers(k, device);
-  if (regs <= 0) return kNotLaunchable;
+  const int max_threads = kernel_max_threads(k, device);
   const int G = a.tpr / 32;
   const int64_t grid = a.rows < sms ? a.rows : sms;
   const int64_t per_cta = (a.rows + grid - 1) / grid;
-  int64_t nc = (65536 / (32 * ((regs + 7) / 8 * 8)) - 1) / G;  // warps the register file holds, less the producer
-  if (nc > (dq::kRingMaxThreads / 32 - 1) / G) nc = (dq::kRingMaxThreads / 32 - 1) / G;
+  int64_t nc = max_threads / a.tpr;
   if (G > 1 && nc > 15) nc = 15;
   if (nc > per_cta) nc = per_cta;
   const size_t smooth_bytes = kSS ? static_cast<size_t>(a.cols) * (SMK == dq::kSmF32 ? 4 : 2) : 0;
@@ -85,7 +83,7 @@ dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t s
   a.groups = static_cast<int>(nc);
   a.stages = static_cast<int>(ns);
   const size_t smem = dq::ring_smem_bytes(a.stages, a.stage_stride, smooth_bytes, a.group_index ? a.num_groups : 0);
-  const int block = 32 + a.tpr * a.groups;
+  const int block = a.tpr * a.groups;
   if (blocks_per_sm(k, block, smem, device) < 1) return kNotLaunchable;
   return launch_programmatic(kfn, a, static_cast<int>(grid), block, smem, stream);
 }
