@@ -142,6 +142,28 @@ def test_ring_slot_reuse_and_dispatch_limits(dq, shape, mode, smooth_dtype):
         assert_dq_equal(got, want, y_dtype)
 
 
+def test_ring_repeated_calls_stay_exact(dq):
+    """Many calls of a shape whose rows cycle through every ring slot many
+    times, with fewer row groups than slots and slots not a multiple of the
+    groups (16384 rows of 8192 fp16 values, asymmetric INT4: 110 rows per CTA,
+    14 slots, 4 groups). A group reaching a slot's next fill round before that
+    round was issued must wait for it; every call is checked for NaN scales
+    (a wait that ran out) and on sampled rows against the oracle."""
+    rows, cols = 16384, 8192
+    x = workloads.normal((rows, cols), torch.float16, 71, mean=0.5, std=2.0)
+    xg = x.cuda()
+    pick = torch.randperm(rows, generator=torch.Generator().manual_seed(72))[:48].sort().values
+    want = oracle.dynamic_quant(x[pick], mode="asymmetric", y_dtype="int4")
+    out = None
+    for call in range(40):
+        out = dq.dynamic_quant(xg, mode="asymmetric", y_dtype="int4", out=out)
+        if call % 8 == 7:
+            torch.cuda.synchronize()
+            y, s, o = (t.cpu().numpy() for t in out[:3])
+            assert not np.isnan(s).any(), f"call {call}: a row's wait ran out"
+            assert_dq_equal((y[pick.numpy()], s[pick.numpy()], o[pick.numpy()]), want, "int4")
+
+
 @pytest.mark.parametrize("rows,cols,experts", [(5920, 1024, 16), (3000, 4096, 64), (296, 1024, 8)])
 def test_ring_moe_many_rows_per_cta(dq, rows, cols, experts):
     g = torch.Generator().manual_seed(rows)

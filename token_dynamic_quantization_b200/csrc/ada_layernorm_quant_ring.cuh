@@ -57,10 +57,12 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   const int NC = a.groups;
   const int64_t H = a.hidden;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * stride);
-  uint32_t* rel_count = reinterpret_cast<uint32_t*>(full + NS);      // warps of the group done with the slot
-  int32_t* last_round = reinterpret_cast<int32_t*>(rel_count + NS);  // fill round of the slot's last copy
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(last_round + NS);
-  float* table_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(last_round + NS) + 16);
+  // fill round of the slot's last issued copy (-1: none); a group reaching
+  // round k of a slot waits for it before the phase parity (see the
+  // DynamicQuant ring kernel)
+  volatile int32_t* issued_round = reinterpret_cast<volatile int32_t*>(full + NS);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(issued_round + 2 * NS);
+  float* table_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(const_cast<int32_t*>(issued_round) + 2 * NS) + 16);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -72,8 +74,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      rel_count[s] = 0u;
-      last_round[s] = -1;
+      issued_round[s] = -1;
     }
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -83,7 +84,8 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   const uint64_t policy = l2_evict_first_policy();
   auto issue = [&](int s, int j) {
-    last_round[s] = j / NS;
+    __threadfence_block();
+    issued_round[s] = j / NS;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out (see dynamic_quant_ring.cuh)
     if (r_begin + j == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) return;
@@ -101,18 +103,24 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   pdl_wait_primary();  // the affine table is complete and visible from here on
   pdl_launch_dependents();
 
-  // the table rows of the batches this CTA's rows belong to
+  // The table rows of the batches this CTA's rows belong to. Each row is
+  // staged as two planes (elements 0-3 and 4-7 of every 8-column vector), so
+  // that 32 lanes reading consecutive vectors read consecutive 16-byte words:
+  // no bank conflicts.
   const int64_t b_lo = n > 0 ? r_begin / a.seq : 0;
   if (kStaged && n > 0) {
     const int64_t nb = (r_begin + n - 1) / a.seq - b_lo + 1;  // <= table_batches (host)
     const int64_t per = H / 4;                                // float4 per table row
+    const int64_t nv = H / 8;
     const float4* A_g = reinterpret_cast<const float4*>(a.table + b_lo * H);
     const float4* B_g = reinterpret_cast<const float4*>(a.table + a.batch * H + b_lo * H);
     float4* A_s = reinterpret_cast<float4*>(table_s);
     float4* B_s = reinterpret_cast<float4*>(table_s + static_cast<int64_t>(a.table_batches) * H);
     for (int64_t i = threadIdx.x; i < nb * per; i += blockDim.x) {
-      A_s[i] = __ldg(A_g + i);
-      B_s[i] = __ldg(B_g + i);
+      const int64_t row = i / per, w = i - row * per;
+      const int64_t d = row * per + (w & 1) * nv + (w >> 1);
+      A_s[d] = __ldg(A_g + i);
+      B_s[d] = __ldg(B_g + i);
     }
   }
   __syncthreads();
@@ -127,6 +135,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   const int vbase = wg * (32 * VPT) + lane;
   auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
   const int64_t table_b_stride4 = H / 4;  // float4 per batch row
+  const int64_t nv4 = H / 8;              // staged: offset of the second plane
   const float4* A_base = kStaged ? reinterpret_cast<const float4*>(table_s)
                                  : reinterpret_cast<const float4*>(a.table);
   const float4* B_base = kStaged ? reinterpret_cast<const float4*>(table_s + static_cast<int64_t>(a.table_batches) * H)
@@ -146,10 +155,10 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     if (r >= b_end) {
       b = r / a.seq;
       b_end = (b + 1) * a.seq;
-      A4 = A_base + (b - b_origin) * table_b_stride4 + 2 * vbase;
-      B4 = B_base + (b - b_origin) * table_b_stride4 + 2 * vbase;
+      A4 = A_base + (b - b_origin) * table_b_stride4 + (kStaged ? vbase : 2 * vbase);
+      B4 = B_base + (b - b_origin) * table_b_stride4 + (kStaged ? vbase : 2 * vbase);
     }
-    const bool ok = mbar_wait_parity_or_abort(full + s, par, abort_flag);
+    const bool ok = wait_round(issued_round + s, j / NS, abort_flag) && mbar_wait_parity_or_abort(full + s, par, abort_flag);
     const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
 
     // ---- pass 1: load, widen, shift by K, both moments of d = x - K
@@ -194,25 +203,6 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
       s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
     }
-    // the group's last warp to get here refills the slot with the row NS on
-    __syncwarp();
-    if (lane == 0) {
-      bool last = true;
-      if (G > 1) {
-        __threadfence_block();
-        last = atomicAdd(rel_count + s, 1u) == static_cast<uint32_t>(G - 1);
-        if (last) rel_count[s] = 0u;
-      }
-      if (last && ok && j + NS < n) {
-        fence_proxy_async_smem();
-        issue(s, j + NS);
-      }
-    }
-    s += NC;
-    if (s >= NS) {
-      s -= NS;
-      par ^= 1u;
-    }
     double sum = s1, sq = s2;
     bool failed;
     if (G > 1) {
@@ -229,6 +219,18 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       }
     } else {
       failed = __any_sync(0xffffffffu, !ok);
+    }
+    // every warp of the group is done with the slot (its shared loads fed the
+    // butterflies before the barrier): the group's first lane refills it with
+    // the row NS further on
+    if (lane_g == 0 && !failed && j + NS < n) {
+      fence_proxy_async_smem();
+      issue(s, j + NS);
+    }
+    s += NC;
+    if (s >= NS) {
+      s -= NS;
+      par ^= 1u;
     }
     if (failed) {
       *abort_flag = 1u;
@@ -279,10 +281,10 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       if (in_row(k)) {
-        const float4 a0 = kStaged ? A4[64 * k] : __ldg(A4 + 64 * k);
-        const float4 a1 = kStaged ? A4[64 * k + 1] : __ldg(A4 + 64 * k + 1);
-        const float4 b0 = kStaged ? B4[64 * k] : __ldg(B4 + 64 * k);
-        const float4 b1 = kStaged ? B4[64 * k + 1] : __ldg(B4 + 64 * k + 1);
+        const float4 a0 = kStaged ? A4[32 * k] : __ldg(A4 + 64 * k);
+        const float4 a1 = kStaged ? A4[32 * k + nv4] : __ldg(A4 + 64 * k + 1);
+        const float4 b0 = kStaged ? B4[32 * k] : __ldg(B4 + 64 * k);
+        const float4 b1 = kStaged ? B4[32 * k + nv4] : __ldg(B4 + 64 * k + 1);
         const float Av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
         const float Bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -340,7 +342,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag != 0u) {
     for (int t = 0; t < NS; ++t) {
-      if (last_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(last_round[t]) & 1u);
+      if (issued_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(issued_round[t]) & 1u);
     }
   }
 }

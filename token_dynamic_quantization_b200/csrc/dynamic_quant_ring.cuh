@@ -44,12 +44,15 @@ __host__ __device__ inline size_t ring_smem_bytes(int slots, uint32_t stride, si
          static_cast<size_t>(num_groups) * 4;
 }
 
-// Smooth scales of vector vi from the staged shared-memory copy.
+// Smooth scales of vector vi from the staged shared-memory copy. An fp32
+// table is staged as two planes (elements 0-3 and 4-7 of every 8-column
+// vector), so that 32 lanes reading consecutive vectors read consecutive
+// 16-byte words: no bank conflicts. `nvec` is the number of vectors.
 template <int SMK>
-__device__ __forceinline__ void load_smooth8_smem(const uint8_t* s, int vi, float (&v)[8]) {
+__device__ __forceinline__ void load_smooth8_smem(const uint8_t* s, int vi, int nvec, float (&v)[8]) {
   if (SMK == kSmF32) {
-    const float4* p = reinterpret_cast<const float4*>(s) + 2 * vi;
-    const float4 a = p[0], b = p[1];
+    const float4* p = reinterpret_cast<const float4*>(s);
+    const float4 a = p[vi], b = p[nvec + vi];
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   } else if (SMK == kSmBF16) {
@@ -81,10 +84,13 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   const int G = tpr >> 5;
   const int NC = a.groups;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NS) * stride);
-  uint32_t* rel_count = reinterpret_cast<uint32_t*>(full + NS);  // warps of the group done with the slot
-  int32_t* last_round = reinterpret_cast<int32_t*>(rel_count + NS);  // fill round of the slot's last copy
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(last_round + NS);
-  uint8_t* smooth_s = reinterpret_cast<uint8_t*>(last_round + NS) + 16;
+  // fill round of the slot's last issued copy (-1: none). An mbarrier only
+  // exposes the parity of its current phase, so a group that reaches round k
+  // of a slot first waits until round k has been issued, and only then for
+  // the phase's parity: it can never mistake a pending round k - 1 for k.
+  volatile int32_t* issued_round = reinterpret_cast<volatile int32_t*>(full + NS);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(issued_round + 2 * NS);
+  uint8_t* smooth_s = reinterpret_cast<uint8_t*>(const_cast<int32_t*>(issued_round) + 2 * NS) + 16;
   const size_t smooth_bytes = kSmemSmooth ? static_cast<size_t>(a.cols) * kSmoothElem : 0;
   int32_t* gi_s = reinterpret_cast<int32_t*>(smooth_s + smooth_bytes);
 
@@ -98,8 +104,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      rel_count[s] = 0u;
-      last_round[s] = -1;
+      issued_round[s] = -1;
     }
     *abort_flag = 0u;
     fence_mbarrier_init();
@@ -113,7 +118,8 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   const uint64_t policy = l2_evict_first_policy();
   auto issue = [&](int s, int j) {
-    last_round[s] = j / NS;
+    __threadfence_block();
+    issued_round[s] = j / NS;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out, so that its consumer's
     // bounded wait runs out and the failure path runs
@@ -130,7 +136,13 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   if (kSmemSmooth) {
     const uint4* src = static_cast<const uint4*>(a.smooth);
     uint4* dst = reinterpret_cast<uint4*>(smooth_s);
-    for (int i = threadIdx.x; i < static_cast<int>(smooth_bytes / 16); i += blockDim.x) dst[i] = __ldg(src + i);
+    const int words = static_cast<int>(smooth_bytes / 16);
+    const int nv = static_cast<int>(a.cols >> 3);
+    for (int i = threadIdx.x; i < words; i += blockDim.x) {
+      // fp32: word i is half (i & 1) of vector i / 2 -> plane (i & 1)
+      const int d = SMK == kSmF32 ? (i & 1) * nv + (i >> 1) : i;
+      dst[d] = __ldg(src + i);
+    }
   }
   if (moe) {
     for (int i = threadIdx.x; i < a.num_groups; i += blockDim.x) gi_s[i] = a.group_index[i];
@@ -161,7 +173,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   int parity = 0;      // red[] buffer
   for (int j = c; j < n && c < NC; j += NC, yrow += y_step) {
     const int64_t r = r_begin + j;
-    const bool ok = mbar_wait_parity_or_abort(full + s, par, abort_flag);
+    const bool ok = wait_round(issued_round + s, j / NS, abort_flag) && mbar_wait_parity_or_abort(full + s, par, abort_flag);
     const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
 
     bool row_valid = true;
@@ -196,7 +208,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
           float v[8], sm[8];
           InTraits<InT>::widen8(raw[k], v);
           if (kSmemSmooth) {
-            load_smooth8_smem<SMK>(smooth_s, vbase + 32 * k, sm);
+            load_smooth8_smem<SMK>(smooth_s, vbase + 32 * k, nvec, sm);
           } else {
             load_smooth8<SMK>(smooth_row, vbase + 32 * k, sm);
           }
@@ -253,27 +265,9 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
     m0 = warp_max(m0);
     if (kA) m1 = warp_min(m1);
     // every lane's shared loads of the slot are complete (their values fed the
-    // warp reduction): the group's last warp to get here refills the slot
+    // warp reduction); once the whole group is past this point (its barrier
+    // below, or this warp alone), the group's first lane refills the slot
     // with the row NS further on
-    __syncwarp();
-    if (lane == 0) {
-      bool last = true;
-      if (G > 1) {
-        __threadfence_block();
-        last = atomicAdd(rel_count + s, 1u) == static_cast<uint32_t>(G - 1);
-        if (last) rel_count[s] = 0u;
-      }
-      if (last && ok && j + NS < n) {
-        fence_proxy_async_smem();
-        issue(s, j + NS);
-      }
-    }
-    s += NC;  // slot and fill round of local row j + NC (NC <= NS)
-    if (s >= NS) {
-      s -= NS;
-      par ^= 1u;
-    }
-
     bool failed;
     if (G > 1) {
       if (lane == 0) {
@@ -281,13 +275,24 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
         if (kA) red[parity][1][warp] = m1;
       }
       failed = group_barrier_or(1 + c, tpr, !ok);
+    } else {
+      failed = __any_sync(0xffffffffu, !ok);
+    }
+    if (lane_g == 0 && !failed && j + NS < n) {
+      fence_proxy_async_smem();
+      issue(s, j + NS);
+    }
+    s += NC;  // slot and fill round of local row j + NC (NC <= NS)
+    if (s >= NS) {
+      s -= NS;
+      par ^= 1u;
+    }
+    if (G > 1) {
       // lane i takes warp i's partial; one more warp reduction combines them
       const bool has = lane < G;
       m0 = warp_max(has ? red[parity][0][warp_g0 + lane] : (kA ? -INFINITY : 0.0f));
       if (kA) m1 = warp_min(has ? red[parity][1][warp_g0 + lane] : INFINITY);
       parity ^= 1;
-    } else {
-      failed = __any_sync(0xffffffffu, !ok);
     }
     if (failed) {
       // A row copy never completed (not a data-dependent condition): mark this
@@ -376,7 +381,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag != 0u) {
     for (int t = 0; t < NS; ++t) {
-      if (last_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(last_round[t]) & 1u);
+      if (issued_round[t] >= 0) mbar_wait_parity(full + t, static_cast<uint32_t>(issued_round[t]) & 1u);
     }
   }
 }

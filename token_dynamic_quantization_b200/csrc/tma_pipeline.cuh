@@ -120,6 +120,22 @@ __device__ __forceinline__ bool mbar_wait_parity_or_abort(uint64_t* bar, uint32_
   }
 }
 
+// Bounded wait until *round (shared memory, written by another warp of the
+// CTA) equals `want`; gives up on the abort flag or after kWaitLimitNs. The
+// fence orders what the writer did before its write (it had observed the
+// slot's previous phase complete) before anything this thread does next.
+__device__ __forceinline__ bool wait_round(const volatile int32_t* round, int32_t want,
+                                           const volatile uint32_t* abort) {
+  if (*round != want) {
+    const uint64_t t0 = global_ns();
+    while (*round != want) {
+      if (*abort != 0u || global_ns() - t0 > kWaitLimitNs) return false;
+    }
+  }
+  __threadfence_block();
+  return true;
+}
+
 // Plain arrival (count 1) on `bar`.
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
