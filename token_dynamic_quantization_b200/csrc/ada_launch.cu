@@ -35,11 +35,16 @@ constexpr size_t kAdaRingSmemBudget = 232448 - 2048;
 #ifndef DQ_ADA_RING_MAX_SLOTS
 #define DQ_ADA_RING_MAX_SLOTS 32
 #endif
+// Bytes of row slots per CTA (hidden 3072, 16 one-warp groups: 16 slots of
+// 6 KB 38.6 us, 20 slots 38.9 us, 29 slots 41.8 us).
+#ifndef DQ_ADA_RING_BYTES
+#define DQ_ADA_RING_BYTES (100 * 1024)
+#endif
 
 // Ring kernel launch: one CTA per SM (fewer for few rows), NC row groups of G
 // warps (as many as the kernel's largest block holds, at most 15 with G > 1), the
 // table rows of the CTA's batches staged when they fit DQ_ADA_TABLE_BUDGET,
-// NS row slots in the rest of the shared memory.
+// NS row slots of about DQ_ADA_RING_BYTES in all.
 template <typename InT, int VPT, bool kRagged, bool kStaged>
 dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batches, cudaStream_t stream) {
   void (*kfn)(const dq::AdaArgs) = dq::ada_layernorm_quant_ring_kernel<InT, VPT, kRagged, kStaged>;
@@ -56,7 +61,10 @@ dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batc
   a.table_batches = kStaged ? static_cast<int>(table_batches) : 0;
   const size_t fixed = dq::ada_ring_smem_bytes(0, a.stage_stride, a.table_batches, a.hidden);
   if (fixed >= kAdaRingSmemBudget) return kNotLaunchable;
-  int64_t ns = static_cast<int64_t>((kAdaRingSmemBudget - fixed) / (a.stage_stride + 16));
+  const int64_t ns_fit = static_cast<int64_t>((kAdaRingSmemBudget - fixed) / (a.stage_stride + 16));
+  int64_t ns = DQ_ADA_RING_BYTES / a.stage_stride;
+  if (ns < nc) ns = nc;  // at least one slot per group
+  if (ns > ns_fit) ns = ns_fit;
   if (ns > DQ_ADA_RING_MAX_SLOTS) ns = DQ_ADA_RING_MAX_SLOTS;
   if (ns > per_cta) ns = per_cta;
   if (nc > ns) nc = ns;

@@ -83,9 +83,9 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   // local row j of the CTA into slot s (= j % NS), completing full[s]
   const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   const uint64_t policy = l2_evict_first_policy();
-  auto issue = [&](int s, int j) {
+  auto issue = [&](int s, int j, int round) {  // round = j / NS
     __threadfence_block();
-    issued_round[s] = j / NS;
+    issued_round[s] = round;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out (see dynamic_quant_ring.cuh)
     if (r_begin + j == static_cast<int64_t>(DQ_TEST_SKIP_COPY_ROW)) return;
@@ -98,7 +98,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   // waited for the work before it before it let this one start, so x is
   // already final.
   if (threadIdx.x == 0) {
-    for (int j = 0; j < NS && j < n; ++j) issue(j, j);
+    for (int j = 0; j < NS && j < n; ++j) issue(j, j, 0);
   }
   pdl_wait_primary();  // the affine table is complete and visible from here on
   pdl_launch_dependents();
@@ -142,8 +142,8 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
                                  : reinterpret_cast<const float4*>(a.table + a.batch * H);
   const int64_t b_origin = kStaged ? b_lo : 0;
 
-  int s = c;
-  uint32_t par = 0u;
+  int s = c;       // slot of local row j (NC <= NS)
+  int round = 0;   // its fill round, j / NS
   int parity = 0;
   int64_t b = -1, b_end = -1;
   const float4* A4 = nullptr;
@@ -158,7 +158,8 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       A4 = A_base + (b - b_origin) * table_b_stride4 + (kStaged ? vbase : 2 * vbase);
       B4 = B_base + (b - b_origin) * table_b_stride4 + (kStaged ? vbase : 2 * vbase);
     }
-    const bool ok = wait_round(issued_round + s, j / NS, abort_flag) && mbar_wait_parity_or_abort(full + s, par, abort_flag);
+    const bool ok = wait_round(issued_round + s, round, abort_flag) &&
+                    mbar_wait_parity_or_abort(full + s, static_cast<uint32_t>(round) & 1u, abort_flag);
     const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
 
     // ---- pass 1: load, widen, shift by K, both moments of d = x - K
@@ -225,12 +226,12 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     // the row NS further on
     if (lane_g == 0 && !failed && j + NS < n) {
       fence_proxy_async_smem();
-      issue(s, j + NS);
+      issue(s, j + NS, round + 1);
     }
     s += NC;
     if (s >= NS) {
       s -= NS;
-      par ^= 1u;
+      ++round;
     }
     if (failed) {
       *abort_flag = 1u;

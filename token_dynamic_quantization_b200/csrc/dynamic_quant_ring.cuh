@@ -117,9 +117,9 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   // local row j of the CTA into slot s (= j % NS), completing full[s]
   const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   const uint64_t policy = l2_evict_first_policy();
-  auto issue = [&](int s, int j) {
+  auto issue = [&](int s, int j, int round) {  // round = j / NS
     __threadfence_block();
-    issued_round[s] = j / NS;
+    issued_round[s] = round;
 #ifdef DQ_TEST_SKIP_COPY_ROW
     // test builds only: leave one row's copy out, so that its consumer's
     // bounded wait runs out and the failure path runs
@@ -131,7 +131,7 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   };
   // the whole ring is in flight before anything else
   if (threadIdx.x == 0) {
-    for (int j = 0; j < NS && j < n; ++j) issue(j, j);
+    for (int j = 0; j < NS && j < n; ++j) issue(j, j, 0);
   }
   if (kSmemSmooth) {
     const uint4* src = static_cast<const uint4*>(a.smooth);
@@ -169,11 +169,12 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   uint8_t* yrow = static_cast<uint8_t*>(a.y) + (r_begin + c) * y_row_bytes;
 
   int s = c;           // slot of local row j (NC <= NS)
-  uint32_t par = 0u;   // parity of its fill round
+  int round = 0;       // its fill round, j / NS
   int parity = 0;      // red[] buffer
   for (int j = c; j < n && c < NC; j += NC, yrow += y_step) {
     const int64_t r = r_begin + j;
-    const bool ok = wait_round(issued_round + s, j / NS, abort_flag) && mbar_wait_parity_or_abort(full + s, par, abort_flag);
+    const bool ok = wait_round(issued_round + s, round, abort_flag) &&
+                    mbar_wait_parity_or_abort(full + s, static_cast<uint32_t>(round) & 1u, abort_flag);
     const uint4* srow = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stride);
 
     bool row_valid = true;
@@ -280,12 +281,12 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
     }
     if (lane_g == 0 && !failed && j + NS < n) {
       fence_proxy_async_smem();
-      issue(s, j + NS);
+      issue(s, j + NS, round + 1);
     }
     s += NC;  // slot and fill round of local row j + NC (NC <= NS)
     if (s >= NS) {
       s -= NS;
-      par ^= 1u;
+      ++round;
     }
     if (G > 1) {
       // lane i takes warp i's partial; one more warp reduction combines them

@@ -55,11 +55,19 @@ constexpr size_t kRingSmemBudget = 232448 - 1024;
 #ifndef DQ_RING_MAX_SLOTS
 #define DQ_RING_MAX_SLOTS 32
 #endif
+// Bytes of row slots per CTA. Measured on the 8192 x 4096 workload (one CTA
+// per SM, 8 row groups): 12 slots of 8 KB 20.1 us, 16 slots 22.2 us, 26 slots
+// 23.6 us; on 32768 rows 8 slots 67.7 us, 26 slots 73.9 us. A deeper ring
+// puts more rows in flight than the HBM needs and makes each row's copy
+// slower to land.
+#ifndef DQ_RING_BYTES
+#define DQ_RING_BYTES (100 * 1024)
+#endif
 
 // Ring kernel launch: one CTA per SM (fewer for few rows), NC row groups of
 // G = tpr / 32 warps, as many as the kernel's largest block holds (at most 15
-// with G > 1: one named barrier each), and NS row slots filling the shared
-// memory (NC <= NS <= rows of a CTA).
+// with G > 1: one named barrier each), and NS row slots of about
+// DQ_RING_BYTES in all (NC <= NS <= rows of a CTA).
 template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged, bool kSS>
 dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t stream) {
   void (*kfn)(const dq::RowQuantArgs) = dq::dynamic_quant_ring_kernel<InT, MODE, OUT, SMK, VPT, kRagged, kSS>;
@@ -75,7 +83,10 @@ dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t s
   const size_t smooth_bytes = kSS ? static_cast<size_t>(a.cols) * (SMK == dq::kSmF32 ? 4 : 2) : 0;
   const size_t fixed = dq::ring_smem_bytes(0, a.stage_stride, smooth_bytes, a.group_index ? a.num_groups : 0);
   if (fixed >= kRingSmemBudget) return kNotLaunchable;
-  int64_t ns = static_cast<int64_t>((kRingSmemBudget - fixed) / (a.stage_stride + 16));
+  const int64_t ns_fit = static_cast<int64_t>((kRingSmemBudget - fixed) / (a.stage_stride + 16));
+  int64_t ns = DQ_RING_BYTES / a.stage_stride;
+  if (ns < nc) ns = nc;  // at least one slot per group
+  if (ns > ns_fit) ns = ns_fit;
   if (ns > DQ_RING_MAX_SLOTS) ns = DQ_RING_MAX_SLOTS;
   if (ns > per_cta) ns = per_cta;
   if (nc > ns) nc = ns;
