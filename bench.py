@@ -133,8 +133,8 @@ def measured_peaks(tensor: bool = False):
 KERNEL_SOURCES = {
     "dynamic_quant": ("dynamic_quant_kernels.cuh", "dynamic_quant_ring.cuh", "dq_device.cuh", "tma_pipeline.cuh",
                       "dq_args.cuh", "quant_launch.cuh", "dq_launch.cuh"),
-    "ada_layernorm_quant": ("ada_layernorm_quant_kernels.cuh", "dq_device.cuh", "tma_pipeline.cuh", "dq_args.cuh",
-                            "ada_launch.cu", "dq_launch.cuh"),
+    "ada_layernorm_quant": ("ada_layernorm_quant_kernels.cuh", "ada_layernorm_quant_ring.cuh", "dq_device.cuh",
+                            "tma_pipeline.cuh", "dq_args.cuh", "ada_launch.cu", "dq_launch.cuh"),
     "dequant_per_token": ("dequant_kernels.cuh", "dq_device.cuh", "dq_args.cuh", "dequant_launch.cu", "dq_launch.cuh"),
     "dequant_per_group": ("dequant_kernels.cuh", "dq_device.cuh", "dq_args.cuh", "dequant_launch.cu", "dq_launch.cuh"),
     "w8a8_gemm": ("w8a8_gemm.cu", "tma_pipeline.cuh"),

@@ -17,7 +17,7 @@
 //
 // Arithmetic of the ring kernel:
 //   * E(x), Var(x) from one row reduction: each thread sums d = x - K and d^2
-//     over its share, with K the mean of the row's first 8 elements (the same
+//     over its share, with K the mean of the row's first 4 elements (the same
 //     value in every thread; d is exact when x and K are within a factor 2,
 //     as on rows whose mean is far above their spread). Partial sums are fp32,
 //     the sums across warps double; E(x) = K + E(d), Var = E(d^2) - E(d)^2.
@@ -25,7 +25,7 @@
 //     relative accuracy. Rows past the bound (first elements far from the
 //     mean) take a centred second pass about RN(E(x)). E(x) is rounded to
 //     fp32 once, as the formula's mean is.
-//   * n = (x - E(x)) * rstd with rstd = RN(1 / RN(sqrt(Var + eps))), as
+//   * n = (x - E(x)) * rstd with rstd = RN(1 / sqrt(Var + eps)), as
 //     fma(d, rstd, -(E(x) - K) * rstd), then y = n * A + B. Against a
 //     sequential evaluation that rounds every printed operation separately
 //     and divides by the square root, this moves y by a few ulps:

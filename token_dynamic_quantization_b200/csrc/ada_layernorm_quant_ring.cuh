@@ -12,11 +12,12 @@
 // loads instead of L1/L2 loads on every row.
 //
 // Arithmetic per row: both moments of
-// d = x - K (K the mean of the row's first 8 elements) from one reduction,
+// d = x - K (K the mean of the row's first 4 elements) from one reduction,
 // fp32 partial sums per thread and warp, double across warps, a centred second
 // pass for rows whose first elements sit far from the mean; then
-// n = fma(d, rstd, -(E(x) - K) * rstd), y = n * A + B, absmax, and the exact
-// symmetric INT8 quantizer.
+// rstd = RN(1 / sqrt(Var + eps)) (one correctly rounded reciprocal square
+// root), n = fma(d, rstd, -(E(x) - K) * rstd), y = n * A + B, absmax, and the
+// exact symmetric INT8 quantizer.
 //
 // Failure handling as in the DynamicQuant ring kernel: every wait is bounded
 // in time and gives up on the shared abort flag; a group whose row never
@@ -164,13 +165,12 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
 
     // ---- pass 1: load, widen, shift by K, both moments of d = x - K
     constexpr int NACC = VPT < 4 ? VPT : 4;
-    float K;
+    float K;  // the mean of the row's first 4 elements (the same bits in every thread)
     {
+      const uint2 w2 = reinterpret_cast<const uint2*>(srow)[0];
       float f[8];
-      InTraits<InT>::widen8(srow[0], f);
-      K = __fmul_rn(__fadd_rn(__fadd_rn(__fadd_rn(f[0], f[1]), __fadd_rn(f[2], f[3])),
-                              __fadd_rn(__fadd_rn(f[4], f[5]), __fadd_rn(f[6], f[7]))),
-                    0.125f);
+      InTraits<InT>::widen8(make_uint4(w2.x, w2.y, 0u, 0u), f);
+      K = __fmul_rn(__fadd_rn(__fadd_rn(f[0], f[1]), __fadd_rn(f[2], f[3])), 0.25f);
     }
     float v[VPT][8];
     float2 acc[NACC], acq[NACC];
@@ -196,14 +196,15 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       acc[0] = __fadd2_rn(acc[0], acc[t]);
       acq[0] = __fadd2_rn(acq[0], acq[t]);
     }
-    float s1 = __fadd_rn(acc[0].x, acc[0].y), s2 = __fadd_rn(acq[0].x, acq[0].y);
-    // butterflies: every lane ends with the same bits; the lane shuffles also
-    // make every lane's shared loads of the slot complete
+    // butterflies on (sum d, sum d^2) as one pair: every lane ends with the
+    // same bits (each step adds the same two operands on both lanes of a pair)
+    float2 s12 = make_float2(__fadd_rn(acc[0].x, acc[0].y), __fadd_rn(acq[0].x, acq[0].y));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s1 = __fadd_rn(s1, __shfl_xor_sync(0xffffffffu, s1, o));
-      s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, o));
+      const float2 t = make_float2(__shfl_xor_sync(0xffffffffu, s12.x, o), __shfl_xor_sync(0xffffffffu, s12.y, o));
+      s12 = __fadd2_rn(s12, t);
     }
+    const float s1 = s12.x, s2 = s12.y;
     double sum = s1, sq = s2;
     bool failed;
     if (G > 1) {
@@ -272,7 +273,7 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
       var_d = sc * a.inv_hidden - dm * dm;
     }
     var_d = var_d > 0.0 ? var_d : 0.0;
-    const float rstd = __frcp_rn(__fsqrt_rn(__fadd_rn(__double2float_rn(var_d), a.epsilon)));
+    const float rstd = __frsqrt_rn(__fadd_rn(__double2float_rn(var_d), a.epsilon));  // RN(1 / sqrt(var + eps))
     const float nb = -__fmul_rn(c_f, rstd);
 
     // ---- pass 2: y = n * A + B, absmax
