@@ -95,11 +95,14 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes,
                   full + s, policy);
   };
-  // The whole ring goes out before the wait for the table kernel: that kernel
-  // waited for the work before it before it let this one start, so x is
-  // already final.
+  // The first ceil(NC / 2) rows go out before the wait for the table kernel
+  // (that kernel waited for the work before it before it let this one start,
+  // so x is already final), the rest of the ring once the table is staged:
+  // copies in flight together land at about the same time, so a few issued
+  // first let the row groups start early (see dynamic_quant_ring.cuh).
+  const int first_fill = (NC + 1) / 2;
   if (threadIdx.x == 0) {
-    for (int j = 0; j < NS && j < n; ++j) issue(j, j, 0);
+    for (int j = 0; j < first_fill && j < n; ++j) issue(j, j, 0);
   }
   pdl_wait_primary();  // the affine table is complete and visible from here on
   pdl_launch_dependents();
@@ -125,6 +128,9 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int j = first_fill; j < NS && j < n; ++j) issue(j, j, 0);
+  }
   if (n <= 0) return;
 
   // ------------------------------------------------------------ row groups

@@ -178,6 +178,13 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(const void* tile) {
   return start | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
+// The same for the 64-byte swizzle layout: rows of 64 bytes, groups of 8
+// rows 512 bytes apart, layout type 4.
+__device__ __forceinline__ uint64_t smem_desc_k_sw64(const void* tile) {
+  const uint64_t start = (dq::smem_addr(tile) >> 4) & 0x3FFFu;
+  return start | (uint64_t(1) << 16) | (uint64_t(512 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(4) << 61);
+}
+
 __device__ __forceinline__ void tc_mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
   asm volatile(
@@ -399,18 +406,29 @@ w8a8_gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_cons
 // One CTA per SM walks a list of output tiles: 128 x 256 tiles first, then the
 // last r of them split into two 128 x 128 tiles each, when that evens out the
 // SMs (every SM gets q wide tiles, 2r <= SMs of them one narrow tile: the
-// last wave is half as long). The ring is 4 stages of 48 KB; the int32
-// accumulator is double-buffered in TMEM (2 x 256 columns), so the epilogue of
-// one tile overlaps the MMAs of the next.
+// last wave is half as long). The ring holds 192 KB of K slices of kPBK bytes
+// (4 stages of 48 KB at 128 bytes, 8 of 24 KB at 64); the int32 accumulator is
+// double-buffered in TMEM (2 x 256 columns), so the epilogue of one tile
+// overlaps the MMAs of the next.
+#ifndef DQ_W8A8_PBK
+#define DQ_W8A8_PBK 128
+#endif
+constexpr int kPBK = DQ_W8A8_PBK;  // K slice per stage: 128 (128-byte swizzle) or 64 (64-byte swizzle)
+static_assert(kPBK == 128 || kPBK == 64, "K slice of 64 or 128 bytes");
 #ifndef DQ_W8A8_PSTAGES
-#define DQ_W8A8_PSTAGES 4
+#define DQ_W8A8_PSTAGES (kPBK == 128 ? 4 : 8)
 #endif
 constexpr int kPStages = DQ_W8A8_PSTAGES;
-constexpr uint32_t kPTileBBytes = 256 * kBK;                     // 32 KB (a narrow tile uses 16)
-constexpr uint32_t kPStageBytes = kTileABytes + kPTileBBytes;   // 48 KB
+constexpr uint32_t kPTileABytes = kBM * kPBK;                     // 16 KB at 128
+constexpr uint32_t kPTileBBytes = 256 * kPBK;                     // 32 KB at 128 (a narrow tile uses half)
+constexpr uint32_t kPStageBytes = kPTileABytes + kPTileBBytes;   // 48 KB at 128
 constexpr uint32_t kPTmemCols = 512;
 // ring, barriers and flags (256 B), two buffers of 256 column scales
 constexpr size_t kPSmemBytes = 1024 + kPStages * kPStageBytes + 256 + 2 * 256 * 4;
+
+__device__ __forceinline__ uint64_t smem_desc_k_p(const void* tile) {
+  return kPBK == 128 ? smem_desc_k_sw128(tile) : smem_desc_k_sw64(tile);
+}
 constexpr uint32_t kIdescN256 = i8_idesc(256);
 constexpr uint32_t kIdescN128 = i8_idesc(128);
 
@@ -440,8 +458,8 @@ w8a8_gemm_persistent_kernel(const __grid_constant__ CUtensorMap map_a, const __g
                             const __grid_constant__ CUtensorMap map_b128, const W8A8Args a, const PersistSched ps) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sa = smem;                                   // kPStages x 16 KB (A tiles)
-  uint8_t* sb = smem + kPStages * kTileABytes;          // kPStages x 32 KB (B tiles)
+  uint8_t* sa = smem;                                   // kPStages x kPTileABytes (A tiles)
+  uint8_t* sb = smem + kPStages * kPTileABytes;         // kPStages x kPTileBBytes (B tiles)
   uint64_t* full = reinterpret_cast<uint64_t*>(sb + kPStages * kPTileBBytes);
   uint64_t* empty = full + kPStages;
   uint64_t* acc_full = empty + kPStages;   // [2]: the accumulator holds a finished tile
@@ -454,7 +472,7 @@ w8a8_gemm_persistent_kernel(const __grid_constant__ CUtensorMap map_a, const __g
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ktiles = static_cast<int>((a.k + kBK - 1) / kBK);
+  const int ktiles = static_cast<int>((a.k + kPBK - 1) / kPBK);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPStages; ++s) {
@@ -507,9 +525,9 @@ w8a8_gemm_persistent_kernel(const __grid_constant__ CUtensorMap map_a, const __g
           // the MMA lane's bounded wait runs out and the failure path runs
           if (m0 == int64_t(kBM) * DQ_TEST_SKIP_W8A8_TILE_M && n0 == 0 && kt == DQ_TEST_SKIP_W8A8_KTILE) continue;
 #endif
-          dq::mbar_arrive_expect_tx(full + s, kTileABytes + (wide ? kPTileBBytes : kPTileBBytes / 2));
-          tma_load_2d(sa + s * kTileABytes, &map_a, kt * kBK, static_cast<int>(m0), full + s);
-          tma_load_2d(sb + s * kPTileBBytes, wide ? &map_b256 : &map_b128, kt * kBK, static_cast<int>(n0), full + s);
+          dq::mbar_arrive_expect_tx(full + s, kPTileABytes + (wide ? kPTileBBytes : kPTileBBytes / 2));
+          tma_load_2d(sa + s * kPTileABytes, &map_a, kt * kPBK, static_cast<int>(m0), full + s);
+          tma_load_2d(sb + s * kPTileBBytes, wide ? &map_b256 : &map_b128, kt * kPBK, static_cast<int>(n0), full + s);
         }
       }
       // no copy may still be landing in shared memory when the CTA exits
@@ -543,10 +561,10 @@ w8a8_gemm_persistent_kernel(const __grid_constant__ CUtensorMap map_a, const __g
             break;
           }
           tc_fence_after();
-          const uint64_t ad = smem_desc_k_sw128(sa + s * kTileABytes);
-          const uint64_t bd = smem_desc_k_sw128(sb + s * kPTileBBytes);
+          const uint64_t ad = smem_desc_k_p(sa + s * kPTileABytes);
+          const uint64_t bd = smem_desc_k_p(sb + s * kPTileBBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 32; ++kk) {
+          for (int kk = 0; kk < kPBK / 32; ++kk) {
             tc_mma_i8(d, ad + 2 * kk, bd + 2 * kk, idesc, (kt | kk) != 0 ? 1u : 0u);
           }
           tc_commit(empty + s);
@@ -651,16 +669,18 @@ EncodeTiledFn encode_tiled() {
 }
 
 // [rows, k] int8, k contiguous: 128-byte x box_rows boxes, 128-byte swizzle.
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k, uint32_t box_rows) {
+// Boxes of box_k bytes of K (128: 128-byte swizzle, 64: 64-byte swizzle) by
+// box_rows rows.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t k, uint32_t box_rows, uint32_t box_k = kBK) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};  // bytes between rows
-  const cuuint32_t box[2] = {kBK, box_rows};
+  const cuuint32_t box[2] = {box_k, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, box_k == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool aligned_to(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) & (n - 1)) == 0; }
@@ -723,8 +743,8 @@ dq_status launch_tc(const W8A8Args& args, int device, cudaStream_t stream) {
 // shared-memory opt-in are unavailable.
 dq_status launch_persistent(const W8A8Args& args, int device, cudaStream_t stream) {
   CUtensorMap ma, mb256, mb128;
-  if (!make_map(&ma, args.a, args.m, args.k, kBM) || !make_map(&mb256, args.b, args.n, args.k, 256) ||
-      !make_map(&mb128, args.b, args.n, args.k, 128))
+  if (!make_map(&ma, args.a, args.m, args.k, kBM, kPBK) || !make_map(&mb256, args.b, args.n, args.k, 256, kPBK) ||
+      !make_map(&mb128, args.b, args.n, args.k, 128, kPBK))
     return kNotLaunchable;
   static std::once_flag once[kMaxDevices];
   static bool ok[kMaxDevices];
