@@ -107,10 +107,48 @@ def workload_config(wl) -> dict:
             "cols": wl.cols, "mode": wl.mode if wl.kind == "dynamic_quant" else "symmetric", "y_dtype": wl.y_dtype}
 
 
+SMS = 148
+
+
+def ada_table_staged(wl) -> bool:
+    """Whether the library's AdaLayerNormQuant launch takes the ring kernel
+    that folds the affine table rows of its CTA's batches in shared memory
+    (hidden a multiple of 8, and those rows within 64 KB): one launch per
+    call. Otherwise the affine-table kernel runs first: two launches."""
+    b, s, h = wl.primary.shape
+    rows = b * s
+    if h % 8 or rows == 0:
+        return False
+    grid = min(rows, SMS)
+    per_cta = -(-rows // grid)
+    nb = min((per_cta - 1) // s + 2, b)
+    return nb * h * 8 <= 64 * 1024
+
+
 def launches_per_call(wl) -> int:
-    """Kernels one C-ABI call launches: DynamicQuant and the dequantizer one;
-    AdaLayerNormQuant two (the per-batch affine table, then the row kernel)."""
-    return 2 if wl.kind == "ada_layernorm_quant" else 1
+    """Kernels one C-ABI call launches: DynamicQuant, the dequantizers and the
+    W8A8 product one; AdaLayerNormQuant one when its ring kernel folds the
+    affine table itself, else two (the affine table, then the row kernel)."""
+    if wl.kind == "ada_layernorm_quant":
+        return 1 if ada_table_staged(wl) else 2
+    return 1
+
+
+def timed_kernel(wl) -> str:
+    """The kernel the timed region runs (the roofline's subject)."""
+    if wl.kind == "dynamic_quant":
+        # few short rows (one warp each, at most 2 per SM) take the warp kernel
+        nvec = wl.cols // 8
+        one_warp = wl.cols % 8 == 0 and any(nvec == 32 * v for v in (2, 4, 6, 7, 8))
+        return "dynamic_quant_warp_kernel" if one_warp and wl.rows <= 2 * SMS else "dynamic_quant_ring_kernel"
+    if wl.kind == "ada_layernorm_quant":
+        return ("ada_layernorm_quant_ring_kernel (one launch per call: the affine table folded in the kernel)"
+                if ada_table_staged(wl) else
+                "ada_layernorm_quant_ring_kernel (time of the whole call: affine-table kernel included)")
+    if wl.kind == "w8a8_gemm":
+        return "w8a8_gemm_persistent_kernel"
+    return {"dequant_per_token": "dequant_vec_kernel (per-token layout)",
+            "dequant_per_group": "dequant_vec_kernel (per-group layout)"}[wl.kind]
 
 
 def measured_peaks(tensor: bool = False):
@@ -502,11 +540,7 @@ def run_ours(args, world, rank, local):
                               if tensor else "measured (MEASURED_PEAKS.json hbm_gbs, copy kernel)")
                 if peak_kind == "measured" else "fallback",
                 "traffic": traffic,
-                "kernel": {"dynamic_quant": "dynamic_quant_tma_kernel", "w8a8_gemm": "w8a8_gemm_tc_kernel",
-                           "dequant_per_token": "dequant_vec_kernel (per-token layout)",
-                           "dequant_per_group": "dequant_vec_kernel (per-group layout)",
-                           "ada_layernorm_quant": "ada_layernorm_quant_tma_kernel (time of the whole call: "
-                                                  "affine-table kernel included)"}[wl.kind],
+                "kernel": timed_kernel(wl),
             },
             "clocks": clocks,
             "gpu_launches": args.steps * launches_per_call(wl),

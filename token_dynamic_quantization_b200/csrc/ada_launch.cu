@@ -1,6 +1,7 @@
-// AdaLayerNormQuant launch selection (aclnnAdaLayerNormQuant): the affine
-// table kernel, then the bulk-copy row kernel for the row width (or the
-// generic kernel), as its programmatic dependent.
+// AdaLayerNormQuant launch selection (aclnnAdaLayerNormQuant): the bulk-copy
+// ring kernel for the row width, which folds its batches' affine table rows
+// itself when they fit in shared memory; otherwise the affine table kernel,
+// then the ring kernel (or the generic kernel) as its programmatic dependent.
 #include <cstdlib>
 
 #include "ada_layernorm_quant_kernels.cuh"
@@ -74,8 +75,11 @@ dq_status launch_ada_ring(dq::AdaArgs a, int device, int sms, int64_t table_batc
   const size_t smem = dq::ada_ring_smem_bytes(a.stages, a.stage_stride, a.table_batches, a.hidden);
   const int block = a.tpr * a.groups;
   if (blocks_per_sm(k, block, smem, device) < 1) return kNotLaunchable;
-  dq_status st = launch_ada_table(a, sms, stream);
-  if (st != DQ_OK) return st;
+  if (!kStaged) {
+    // the ring kernel reads the table through L1: the table kernel writes it
+    const dq_status st = launch_ada_table(a, sms, stream);
+    if (st != DQ_OK) return st;
+  }
   return launch_programmatic(kfn, a, static_cast<int>(grid), block, smem, stream);
 }
 

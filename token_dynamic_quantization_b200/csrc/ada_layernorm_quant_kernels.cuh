@@ -1,19 +1,21 @@
 // Fused AdaLayerNorm + symmetric INT8 dynamic quantization
 // (aclnnAdaLayerNormQuant, "Formula" steps 1-5), sm_100a.
 //
-// Two launches per call:
-//   1. ada_affine_table_kernel folds the per-(batch, column) parameters of
-//      steps 1-3 into a table in the caller's workspace,
-//        A[b][c] = (w[c] * (1 + scale[b][c])) * smooth[c]
-//        B[b][c] = ((bias[c] * (1 + scale[b][c])) + shift[b][c]) * smooth[c]
-//      (absent weight = 1, bias = 0, smooth = 1), so steps 1-3 become one FMA
-//      per element, y = n * A + B. The table is batch x hidden x 8 bytes.
-//   2. the row kernel, a programmatic dependent of the table kernel: the
-//      ring kernel (ada_layernorm_quant_ring.cuh) for rows of 16-byte vectors,
-//      else ada_layernorm_quant_generic_kernel below. The table kernel is
-//      itself a programmatic dependent of the work before it and releases the
-//      row kernel only after that work has completed, so the row kernel may
-//      start copying rows of x before it waits for the table.
+// The per-(batch, column) parameters of steps 1-3 fold into a table
+//     A[b][c] = (w[c] * (1 + scale[b][c])) * smooth[c]
+//     B[b][c] = ((bias[c] * (1 + scale[b][c])) + shift[b][c]) * smooth[c]
+// (absent weight = 1, bias = 0, smooth = 1), so steps 1-3 become one FMA per
+// element, y = n * A + B (ada_fold, the one evaluation of these formulas).
+//   * The ring kernel (ada_layernorm_quant_ring.cuh) with the table staged in
+//     shared memory folds the table rows of its batches itself: one launch
+//     per call.
+//   * Otherwise two launches: ada_affine_table_kernel writes the table
+//     (batch x hidden x 8 bytes) into the caller's workspace, then the row
+//     kernel, a programmatic dependent of it (the ring kernel reading the
+//     table through L1, or ada_layernorm_quant_generic_kernel below). The
+//     table kernel is itself a programmatic dependent of the work before it
+//     and releases the row kernel only after that work has completed, so the
+//     row kernel may start copying rows of x before it waits for the table.
 //
 // Arithmetic of the ring kernel:
 //   * E(x), Var(x) from one row reduction: each thread sums d = x - K and d^2
@@ -34,6 +36,8 @@
 //   * steps 4-5 are the DynamicQuant quantizer (exact IEEE semantics).
 #pragma once
 
+#include <type_traits>
+
 #include "dq_args.cuh"
 #include "dq_device.cuh"
 #include "tma_pipeline.cuh"
@@ -43,6 +47,29 @@ namespace dq {
 // ============================================================ affine table
 
 constexpr int kTableBlock = 256;
+
+// A[b][c], B[b][c] of the folded table (ParamT: the parameters' type).
+template <typename ParamT>
+__device__ __forceinline__ float param_at(const void* p, int64_t i) {
+  if constexpr (sizeof(ParamT) == 4) {
+    return __ldg(static_cast<const float*>(p) + i);
+  } else if constexpr (std::is_same<ParamT, __half>::value) {
+    return __half2float(__ldg(static_cast<const __half*>(p) + i));
+  } else {
+    return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p) + i));
+  }
+}
+template <typename ParamT>
+__device__ __forceinline__ void ada_fold(const AdaArgs& a, int64_t b, int64_t c, float& A, float& B) {
+  const int64_t idx = b * a.hidden + c;
+  const float onep = __fadd_rn(1.0f, param_at<ParamT>(a.ada_scale, idx));
+  const float w = a.weight ? param_at<ParamT>(a.weight, c) : 1.0f;
+  const float bs = a.bias ? param_at<ParamT>(a.bias, c) : 0.0f;
+  const float sm = a.smooth ? param_at<ParamT>(a.smooth, c) : 1.0f;
+  const float sh = param_at<ParamT>(a.ada_shift, idx);
+  A = __fmul_rn(__fmul_rn(w, onep), sm);
+  B = __fmul_rn(__fadd_rn(__fmul_rn(bs, onep), sh), sm);
+}
 
 __global__ void __launch_bounds__(kTableBlock) ada_affine_table_kernel(const AdaArgs a) {
   // launched as a programmatic dependent of the previous work in the stream:
@@ -54,14 +81,17 @@ __global__ void __launch_bounds__(kTableBlock) ada_affine_table_kernel(const Ada
   const int64_t total = a.batch * H;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t c = idx % H;
-    const float onep = __fadd_rn(1.0f, load_param(a.ada_scale, a.param_dtype, idx));
-    const float w = a.weight ? load_param(a.weight, a.param_dtype, c) : 1.0f;
-    const float bs = a.bias ? load_param(a.bias, a.param_dtype, c) : 0.0f;
-    const float sm = a.smooth ? load_param(a.smooth, a.param_dtype, c) : 1.0f;
-    const float sh = load_param(a.ada_shift, a.param_dtype, idx);
-    a.table[idx] = __fmul_rn(__fmul_rn(w, onep), sm);
-    a.table[total + idx] = __fmul_rn(__fadd_rn(__fmul_rn(bs, onep), sh), sm);
+    const int64_t b = idx / H, c = idx - (idx / H) * H;
+    float A, B;
+    if (a.param_dtype == kF32) {
+      ada_fold<float>(a, b, c, A, B);
+    } else if (a.param_dtype == kF16) {
+      ada_fold<__half>(a, b, c, A, B);
+    } else {
+      ada_fold<__nv_bfloat16>(a, b, c, A, B);
+    }
+    a.table[idx] = A;
+    a.table[total + idx] = B;
   }
 }
 

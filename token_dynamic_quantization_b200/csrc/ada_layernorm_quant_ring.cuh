@@ -45,6 +45,27 @@ __host__ __device__ inline size_t ada_ring_smem_bytes(int slots, uint32_t stride
 #define DQ_ADA_RING_MAX_REGS 128
 #endif
 
+// The folded table rows (ada_fold) of batches b_lo .. b_lo + nb - 1 into
+// shared memory, each row as two planes (elements 0-3 and 4-7 of every
+// 8-column vector), so that 32 lanes reading consecutive vectors read
+// consecutive 16-byte words: no bank conflicts.
+template <typename ParamT>
+__device__ __forceinline__ void fold_table_rows(const AdaArgs& a, int64_t b_lo, int nb, float* A_s, float* B_s) {
+  const int H = static_cast<int>(a.hidden);
+  const int nv = H / 8;
+  for (int bi = 0; bi < nb; ++bi) {
+#pragma unroll 4
+    for (int c = threadIdx.x; c < H; c += blockDim.x) {
+      float A, B;
+      ada_fold<ParamT>(a, b_lo + bi, c, A, B);
+      const int w = c >> 2;
+      const int d = bi * H + ((w & 1) * nv + (w >> 1)) * 4 + (c & 3);
+      A_s[d] = A;
+      B_s[d] = B;
+    }
+  }
+}
+
 template <typename InT, int VPT, bool kRagged, bool kStaged>
 __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kernel(const AdaArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -95,37 +116,42 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
     bulk_copy_g2s(smem + static_cast<size_t>(s) * stride, x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes,
                   full + s, policy);
   };
-  // The first ceil(NC / 2) rows go out before the wait for the table kernel
-  // (that kernel waited for the work before it before it let this one start,
-  // so x is already final), the rest of the ring once the table is staged:
-  // copies in flight together land at about the same time, so a few issued
-  // first let the row groups start early (see dynamic_quant_ring.cuh).
+  // The first ceil(NC / 2) rows go out at once, the rest of the ring once the
+  // table is staged: copies in flight together land at about the same time,
+  // so a few issued first let the row groups start early (see
+  // dynamic_quant_ring.cuh).
   const int first_fill = (NC + 1) / 2;
-  if (threadIdx.x == 0) {
-    for (int j = 0; j < first_fill && j < n; ++j) issue(j, j, 0);
-  }
-  pdl_wait_primary();  // the affine table is complete and visible from here on
-  pdl_launch_dependents();
-
-  // The table rows of the batches this CTA's rows belong to. Each row is
-  // staged as two planes (elements 0-3 and 4-7 of every 8-column vector), so
-  // that 32 lanes reading consecutive vectors read consecutive 16-byte words:
-  // no bank conflicts.
   const int64_t b_lo = n > 0 ? r_begin / a.seq : 0;
-  if (kStaged && n > 0) {
-    const int64_t nb = (r_begin + n - 1) / a.seq - b_lo + 1;  // <= table_batches (host)
-    const int64_t per = H / 4;                                // float4 per table row
-    const int64_t nv = H / 8;
-    const float4* A_g = reinterpret_cast<const float4*>(a.table + b_lo * H);
-    const float4* B_g = reinterpret_cast<const float4*>(a.table + a.batch * H + b_lo * H);
-    float4* A_s = reinterpret_cast<float4*>(table_s);
-    float4* B_s = reinterpret_cast<float4*>(table_s + static_cast<int64_t>(a.table_batches) * H);
-    for (int64_t i = threadIdx.x; i < nb * per; i += blockDim.x) {
-      const int64_t row = i / per, w = i - row * per;
-      const int64_t d = row * per + (w & 1) * nv + (w >> 1);
-      A_s[d] = __ldg(A_g + i);
-      B_s[d] = __ldg(B_g + i);
+  if (kStaged) {
+    // one launch per call: launched as a programmatic dependent of the work
+    // before it (x and the parameters may come from it), this kernel folds
+    // the table rows of its batches itself while its first rows are copied
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    if (threadIdx.x == 0) {
+      for (int j = 0; j < first_fill && j < n; ++j) issue(j, j, 0);
     }
+    if (n > 0) {
+      const int nb = static_cast<int>((r_begin + n - 1) / a.seq - b_lo + 1);  // <= table_batches (host)
+      float* A_s = table_s;
+      float* B_s = table_s + static_cast<int64_t>(a.table_batches) * H;
+      if (a.param_dtype == kF32) {
+        fold_table_rows<float>(a, b_lo, nb, A_s, B_s);
+      } else if (a.param_dtype == kF16) {
+        fold_table_rows<__half>(a, b_lo, nb, A_s, B_s);
+      } else {
+        fold_table_rows<__nv_bfloat16>(a, b_lo, nb, A_s, B_s);
+      }
+    }
+  } else {
+    // a programmatic dependent of the table kernel, which waited for the
+    // work before it before it let this one start: x is already final, and
+    // the table is complete and visible after the wait
+    if (threadIdx.x == 0) {
+      for (int j = 0; j < first_fill && j < n; ++j) issue(j, j, 0);
+    }
+    pdl_wait_primary();
+    pdl_launch_dependents();
   }
   __syncthreads();
   if (threadIdx.x == 0) {
