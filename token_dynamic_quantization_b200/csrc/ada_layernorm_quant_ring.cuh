@@ -4,12 +4,14 @@
 // The row kernel of the fused path, on the structure of the DynamicQuant ring
 // kernel (dynamic_quant_ring.cuh): one persistent CTA per SM owns a
 // contiguous range of rows and a CTA-wide ring of NS slots filled with
-// cp.async.bulk; NC row groups of G warps take rows c, c + NC, ..., and the
-// last warp of a group to have its row in registers refills the slot.
-// The folded affine table (A, B per batch and column, written by
-// ada_affine_table_kernel) is staged in shared memory for the batches the
-// CTA's rows belong to, so the per-element reads of steps 1-3 are shared
-// loads instead of L1/L2 loads on every row.
+// cp.async.bulk; NC row groups of G warps take rows c, c + NC, ..., and once
+// every warp of a group has its row in registers, the group's first lane
+// refills the slot. The folded affine table (A, B per batch and column) of
+// the batches the CTA's rows belong to is folded by this kernel straight into
+// shared memory when it fits (one launch per call), so the per-element reads
+// of steps 1-3 are shared loads instead of L1/L2 loads on every row;
+// otherwise ada_affine_table_kernel writes the table first and this kernel
+// reads it through L1.
 //
 // Arithmetic per row: both moments of
 // d = x - K (K the mean of the row's first 4 elements) from one reduction,
@@ -33,8 +35,8 @@
 namespace dq {
 
 // Shared memory of the AdaLN ring kernel: NS row slots of `stride` bytes;
-// full[NS] mbarriers; per slot a release counter and the fill round of its
-// last copy; a 16-byte abort word; then, when staged,
+// full[NS] mbarriers; per slot the fill round of its last issued copy (and a
+// spare word); a 16-byte abort word; then, when staged,
 // A[table_batches][hidden] and B[table_batches][hidden] (fp32).
 __host__ __device__ inline size_t ada_ring_smem_bytes(int slots, uint32_t stride, int table_batches, int64_t hidden) {
   return static_cast<size_t>(slots) * stride + static_cast<size_t>(slots) * 16 + 16 +

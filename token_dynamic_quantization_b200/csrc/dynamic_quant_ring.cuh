@@ -12,11 +12,12 @@
 //     on their way (8192 x 4096 bf16: 18.6 us against 20.4 us per launch).
 //   * The warps form NC row groups of G warps; group c takes the CTA's rows
 //     c, c + NC, c + 2NC, ... A group reads its row once from the slot into
-//     registers (pass 1: widen, multiply by the smooth scales, reduce). The
-//     last of its warps to finish reading (a shared-memory counter) refills
-//     the slot at once with the row NS further on. The group then combines
-//     its warps' partial reductions, derives the row constants and quantizes
-//     from registers (pass 2).
+//     registers (pass 1: widen, multiply by the smooth scales, reduce). Once
+//     all of its warps are past that point (the group's barrier, which also
+//     exchanges their partial reductions), its first lane refills the slot
+//     with the row NS further on. The group then combines the partial
+//     reductions, derives the row constants and quantizes from registers
+//     (pass 2).
 // Because the slots are shared by the whole CTA, copies run ahead of every
 // group by up to NS rows, independently of which group is slowest, and no
 // warp is set aside for issuing copies.
@@ -40,8 +41,8 @@
 namespace dq {
 
 // Shared memory of the ring kernel, in this order: NS row slots of `stride`
-// bytes; full[NS] mbarriers; per slot a release counter and the fill round
-// of its last copy; a 16-byte abort word; the staged smooth table
+// bytes; full[NS] mbarriers; per slot the fill round of its last issued copy
+// (and a spare word); a 16-byte abort word; the staged smooth table
 // (`smooth_bytes`, a multiple of 16); the MoE group index.
 __host__ __device__ inline size_t ring_smem_bytes(int slots, uint32_t stride, size_t smooth_bytes, int num_groups) {
   return static_cast<size_t>(slots) * stride + static_cast<size_t>(slots) * 16 + 16 + smooth_bytes +
