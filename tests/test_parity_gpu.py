@@ -177,6 +177,46 @@ def test_ring_moe_many_rows_per_cta(dq, rows, cols, experts):
     assert got[3] == 0
 
 
+def _mixed_expert_sizes(rows, seed):
+    """Cumulative group index whose experts alternate between runs of large
+    experts and runs of tiny or empty ones, ending before the last row: on
+    148 CTAs some CTAs' rows belong to one expert, some to two (the ring
+    kernel stages those experts' smooth rows) and some to three or more (the
+    rest are read through L1), and the last CTA has rows past the last group."""
+    g = torch.Generator().manual_seed(seed)
+    sizes = []
+    while sum(sizes) < rows - 120:
+        if torch.rand(1, generator=g).item() < 0.5:
+            sizes.append(int(torch.randint(150, 400, (1,), generator=g)))
+        else:
+            sizes += [int(v) for v in torch.randint(0, 3, (int(torch.randint(3, 9, (1,), generator=g)),), generator=g)]
+    end = rows - 60  # rows past the last group
+    gi, acc = [], 0
+    for sz in sizes:
+        acc = min(acc + sz, end)
+        gi.append(acc)
+    return np.asarray(gi, dtype=np.int32)
+
+
+@pytest.mark.parametrize("smooth_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("mode", ["symmetric", "asymmetric"])
+def test_moe_staged_and_unstaged_expert_rows(dq, smooth_dtype, mode):
+    rows, cols = 12000, 2048
+    gi = _mixed_expert_sizes(rows, 17)
+    experts = len(gi)
+    x, smooth, gi_t = _moe_inputs(rows, cols, experts, 18, gi)
+    smooth = smooth.to(smooth_dtype)
+    want = oracle.dynamic_quant(x[: gi[-1]], smooth=smooth, group_index=gi, mode=mode)
+    got = run_gpu(dq, x, smooth=smooth, group_index=gi_t, mode=mode)
+    end = int(gi[-1])
+    np.testing.assert_array_equal(got[0][:end], want[0])
+    np.testing.assert_array_equal(_bits(got[1][:end]), _bits(want[1]))
+    if mode == "asymmetric":
+        np.testing.assert_array_equal(_bits(got[2][:end]), _bits(want[2]))
+    assert np.all(got[1][end:] == 0)
+    assert got[3] == dq.DQ_WS_ROWS_PAST_LAST_GROUP
+
+
 @pytest.mark.parametrize("mode", ["symmetric", "asymmetric"])
 @pytest.mark.parametrize("y_dtype", ["int8", "int4"])
 def test_misaligned_pointers_take_the_scalar_path(dq, mode, y_dtype):

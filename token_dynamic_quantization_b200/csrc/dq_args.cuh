@@ -32,6 +32,7 @@ struct RowQuantArgs {
   int groups;                  // row groups per CTA (bulk-copy kernel)
   int stages;                  // ring depth per group (bulk-copy kernel)
   uint32_t stage_stride;       // bytes between stages (multiple of 128)
+  int moe_stage;               // ring kernel, MoE: stage up to 2 expert smooth rows per CTA
 };
 
 // ---- AdaLayerNormQuant (aclnnAdaLayerNormQuant)

@@ -22,8 +22,12 @@
 // group by up to NS rows, independently of which group is slowest, and no
 // warp is set aside for issuing copies.
 //
-// Dense smooth-scale tables are staged once per CTA in shared memory; MoE
-// tables (one row per expert) are read through L1.
+// Dense smooth-scale tables are staged once per CTA in shared memory. MoE
+// tables (one row per expert): the rows of the experts of the CTA's first
+// and last rows are staged too when they are at most two (a CTA's contiguous
+// rows rarely span more; 32768 x 7168 bf16, 64 experts: 116 us against
+// 130 us reading them through L1), and any row of another expert reads
+// its smooth row through L1.
 //
 // Failure handling: every wait is bounded in time (tma_pipeline.cuh) and also
 // gives up when a shared abort flag is set. A group whose row copy never
@@ -72,7 +76,9 @@ __device__ __forceinline__ void load_smooth8_smem(const uint8_t* s, int vi, int 
 #endif
 
 // kSmemSmooth: the smooth table (dense, no group index) is staged in shared
-// memory; otherwise smooth rows are read with __ldg.
+// memory; otherwise smooth rows are read with __ldg, or, for MoE inputs with
+// a.moe_stage set, from the up to two expert rows staged in shared memory
+// (the staged region holds 2 rows then).
 template <typename InT, int MODE, int OUT, int SMK, int VPT, bool kRagged, bool kSmemSmooth>
 __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const RowQuantArgs a) {
   using C = QuantConsts<MODE, OUT>;
@@ -96,7 +102,9 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   volatile int32_t* issued_round = reinterpret_cast<volatile int32_t*>(full + NS);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(issued_round + 2 * NS);
   uint8_t* smooth_s = reinterpret_cast<uint8_t*>(const_cast<int32_t*>(issued_round) + 2 * NS) + 16;
-  const size_t smooth_bytes = kSmemSmooth ? static_cast<size_t>(a.cols) * kSmoothElem : 0;
+  const size_t smooth_row_bytes = static_cast<size_t>(a.cols) * kSmoothElem;
+  const bool moe_stage = !kSmemSmooth && kSmooth && a.group_index != nullptr && a.moe_stage != 0;
+  const size_t smooth_bytes = kSmemSmooth ? smooth_row_bytes : (moe_stage ? 2 * smooth_row_bytes : 0);
   int32_t* gi_s = reinterpret_cast<int32_t*>(smooth_s + smooth_bytes);
 
   const int warp = threadIdx.x >> 5;
@@ -140,19 +148,34 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   if (threadIdx.x == 0) {
     for (int j = 0; j < first_fill && j < n; ++j) issue(j, j, 0);
   }
-  if (kSmemSmooth) {
-    const uint4* src = static_cast<const uint4*>(a.smooth);
-    uint4* dst = reinterpret_cast<uint4*>(smooth_s);
-    const int words = static_cast<int>(smooth_bytes / 16);
-    const int nv = static_cast<int>(a.cols >> 3);
-    for (int i = threadIdx.x; i < words; i += blockDim.x) {
-      // fp32: word i is half (i & 1) of vector i / 2 -> plane (i & 1)
-      const int d = SMK == kSmF32 ? (i & 1) * nv + (i >> 1) : i;
-      dst[d] = __ldg(src + i);
-    }
-  }
   if (moe) {
     for (int i = threadIdx.x; i < a.num_groups; i += blockDim.x) gi_s[i] = a.group_index[i];
+  }
+  // smooth rows staged: the dense table, or the experts e_lo .. e_lo +
+  // n_staged - 1 of the CTA's first and last rows
+  int e_lo = 0, n_staged = kSmemSmooth ? 1 : 0;
+  if (moe_stage) {
+    __syncthreads();  // the group index is in shared memory
+    if (n > 0) {
+      e_lo = expert_of(gi_s, a.num_groups, r_begin);
+      int e_hi = expert_of(gi_s, a.num_groups, r_begin + n - 1);
+      if (e_hi >= a.num_groups) e_hi = a.num_groups - 1;  // rows past the last group use no smooth row
+      if (e_lo < a.num_groups && e_hi >= e_lo && e_hi - e_lo <= 1) n_staged = e_hi - e_lo + 1;
+    }
+  }
+  if (kSmemSmooth || moe_stage) {
+    const int words = static_cast<int>(smooth_row_bytes / 16);
+    const int nv = static_cast<int>(a.cols >> 3);
+    for (int t = 0; t < n_staged; ++t) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.smooth) +
+                                                        static_cast<size_t>(e_lo + t) * smooth_row_bytes);
+      uint4* dst = reinterpret_cast<uint4*>(smooth_s + static_cast<size_t>(t) * smooth_row_bytes);
+      for (int i = threadIdx.x; i < words; i += blockDim.x) {
+        // fp32: word i is half (i & 1) of vector i / 2 -> plane (i & 1)
+        const int d = SMK == kSmF32 ? (i & 1) * nv + (i >> 1) : i;
+        dst[d] = __ldg(src + i);
+      }
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -170,8 +193,9 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   const int vbase = wg * (32 * VPT) + lane;  // this thread's vector k is vbase + 32 * k
   auto in_row = [&](int k) { return !kRagged || vbase + 32 * k < nvec; };
 
-  const size_t smooth_row_bytes = static_cast<size_t>(a.cols) * kSmoothElem;
   const uint8_t* smooth_row = static_cast<const uint8_t*>(a.smooth);
+  const uint8_t* smooth_row_s = smooth_s;  // the row's staged smooth scales (when row_staged)
+  bool row_staged = kSmemSmooth;
   int cur_expert = moe ? -1 : 0;
   int64_t expert_end = moe ? -1 : INT64_MAX;
   const int64_t y_row_bytes = OUT == kOutInt8 ? a.cols : (a.cols >> 1);
@@ -195,6 +219,8 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
         expert_end = e < a.num_groups ? static_cast<int64_t>(gi_s[e]) : INT64_MAX;
         smooth_row = static_cast<const uint8_t*>(a.smooth) +
                      static_cast<size_t>(e < a.num_groups ? e : 0) * smooth_row_bytes;
+        row_staged = moe_stage && e >= e_lo && e < e_lo + n_staged;
+        smooth_row_s = smooth_s + static_cast<size_t>(row_staged ? e - e_lo : 0) * smooth_row_bytes;
       }
       row_valid = cur_expert < a.num_groups;
     }
@@ -218,8 +244,8 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
         if (in_row(k)) {
           float v[8], sm[8];
           InTraits<InT>::widen8(raw[k], v);
-          if (kSmemSmooth) {
-            load_smooth8_smem<SMK>(smooth_s, vbase + 32 * k, nvec, sm);
+          if (kSmemSmooth || row_staged) {
+            load_smooth8_smem<SMK>(smooth_row_s, vbase + 32 * k, nvec, sm);
           } else {
             load_smooth8<SMK>(smooth_row, vbase + 32 * k, sm);
           }

@@ -80,7 +80,18 @@ dq_status launch_dq_ring(dq::RowQuantArgs a, int device, int sms, cudaStream_t s
   int64_t nc = max_threads / a.tpr;
   if (G > 1 && nc > 15) nc = 15;
   if (nc > per_cta) nc = per_cta;
-  const size_t smooth_bytes = kSS ? static_cast<size_t>(a.cols) * (SMK == dq::kSmF32 ? 4 : 2) : 0;
+  const size_t smooth_row = static_cast<size_t>(a.cols) * (SMK == dq::kSmF32 ? 4 : 2);
+  size_t smooth_bytes = kSS ? smooth_row : 0;
+  a.moe_stage = 0;
+  if (!kSS && SMK != dq::kSmNone && a.group_index != nullptr) {
+    // MoE: two expert smooth rows staged per CTA, when a ring of one slot per
+    // group still fits beside them
+    const size_t with = dq::ring_smem_bytes(static_cast<int>(nc), a.stage_stride, 2 * smooth_row, a.num_groups);
+    if (with <= kRingSmemBudget) {
+      smooth_bytes = 2 * smooth_row;
+      a.moe_stage = 1;
+    }
+  }
   const size_t fixed = dq::ring_smem_bytes(0, a.stage_stride, smooth_bytes, a.group_index ? a.num_groups : 0);
   if (fixed >= kRingSmemBudget) return kNotLaunchable;
   const int64_t ns_fit = static_cast<int64_t>((kRingSmemBudget - fixed) / (a.stage_stride + 16));
