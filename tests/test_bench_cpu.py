@@ -11,6 +11,7 @@ import os
 import sys
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
@@ -59,3 +60,29 @@ def test_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.source_hash("probe") == h0
     src.write_text("int f(int x) {\n  return x + 2;\n}\n")
     assert bench.source_hash("probe") != h0
+
+
+def test_launch_counts_and_timed_kernels():
+    """The bench's claim of kernel launches per call and of the kernel it
+    times follow the library's dispatch: the ring kernel for long rows, the
+    one-warp kernel for few short rows, one AdaLayerNormQuant launch while the
+    CTA's affine table rows fit in 64 KB of shared memory (two otherwise)."""
+    c1 = workloads.make("sym_int8_f16_64x1024")
+    c2 = workloads.make("sym_int8_smooth_bf16_8192x4096")
+    c5 = workloads.make("ada_layernorm_quant_bf16_4x4096x3072")
+    gemm = workloads.make("w8a8_gemm_int8_bf16_4096x4096x4096")
+    assert bench.timed_kernel(c1) == "dynamic_quant_warp_kernel"
+    assert bench.timed_kernel(c2) == "dynamic_quant_ring_kernel"
+    assert bench.timed_kernel(gemm) == "w8a8_gemm_persistent_kernel"
+    assert bench.timed_kernel(c5).startswith("ada_layernorm_quant_ring_kernel")
+    for wl in (c1, c2, gemm, c5):
+        assert bench.launches_per_call(wl) == 1
+    # 2 batches of 3072 columns per CTA: 48 KB of table rows, folded in the kernel
+    assert bench.ada_table_staged(c5)
+
+    class Wide:  # 2 batches of 8192 columns per CTA: 128 KB, the table kernel runs first
+        kind = "ada_layernorm_quant"
+        primary = torch.empty((4, 4096, 8192), dtype=torch.bfloat16, device="meta")
+
+    assert not bench.ada_table_staged(Wide)
+    assert bench.launches_per_call(Wide) == 2
