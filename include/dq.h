@@ -173,8 +173,9 @@ dq_status dq_dynamic_quant(const void* x, dq_dtype x_dtype, int64_t rows, int64_
 
 /* Workspace query for dq_ada_layernorm_quant (the first phase of
  * aclnnAdaLayerNormQuant's two-phase convention). Writes the bytes of device
- * workspace the call needs: batch * hidden * 8 (a folded table of the affine
- * parameters, rebuilt on every call), or 0 when batch * seq == 0. Host only.
+ * workspace the call needs: batch * hidden * 8 (room for a folded table of
+ * the affine parameters, rebuilt by any call that keeps the table in global
+ * memory), or 0 when batch * seq == 0. Host only.
  * Errors: DQ_ERR_NULL_POINTER, DQ_ERR_BAD_SHAPE, DQ_ERR_BAD_DTYPE. */
 dq_status dq_ada_layernorm_quant_get_workspace_size(int64_t batch, int64_t seq, int64_t hidden,
                                                     dq_dtype x_dtype, dq_dtype param_dtype,
@@ -201,11 +202,13 @@ dq_status dq_ada_layernorm_quant_get_workspace_size(int64_t batch, int64_t seq, 
  *                      float [batch, seq].
  *   workspace          device, 16-byte aligned, at least the bytes
  *                      dq_ada_layernorm_quant_get_workspace_size returned.
- *                      Its contents are scratch, overwritten by every call;
+ *                      Its contents are scratch, which a call may overwrite;
  *                      calls that run concurrently need separate workspaces.
- * Two kernels are launched on `stream`: one folds steps 1-3's parameters into
- * y = n * A + B (A, B per batch and column, in the workspace), the second
- * processes the rows and overlaps its start with the first.
+ * Steps 1-3's parameters are folded into y = n * A + B (A, B per batch and
+ * column). When the table rows of the batches one CTA processes fit in 64 KB
+ * of shared memory, one kernel is launched on `stream` and folds them there;
+ * otherwise a first kernel writes the table into the workspace and the row
+ * kernel, launched second, overlaps its start with it.
  * The row statistics are reduced in a different order than a sequential loop
  * and steps 1-3 are folded, so a result may differ from a sequential fp32
  * evaluation in the last bits: quant_scale by a relative 1e-5 at most, and

@@ -20,8 +20,10 @@
 // stream capture.
 //
 // Nothing in the array has to start at zero: every call writes each table
-// entry it reads (the table kernel runs first on the same stream and the row
-// kernel waits for it). The array is shared by all calls on a device, so two
+// entry it reads (when the row kernel reads the table from global memory, the
+// table kernel writes it first on the same stream and the row kernel waits
+// for it; otherwise the row kernel folds the table in shared memory and the
+// array is not touched). The array is shared by all calls on a device, so two
 // calls whose executions overlap (different streams, or different host
 // threads) race on it; such callers use the regular entry point with
 // separate workspaces.
