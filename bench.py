@@ -47,6 +47,7 @@ METRIC = "DynamicQuant GB/s and % of B200 HBM roofline (rows/s at 8192x4096 bf16
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
 PRE_ROLL_CYCLES = 2_000_000  # device sleep queued ahead of the timed launches (~1 ms at 1.9 GHz)
+PRE_ROLL_CYCLES_PER_STEP = 20_000  # and ~10 us more per timed step, so the host stays ahead of the device
 
 
 # ---------------------------------------------------------------- helpers
@@ -170,9 +171,9 @@ def measured_peaks(tensor: bool = False):
 # figure stays valid while these are unchanged).
 KERNEL_SOURCES = {
     "dynamic_quant": ("dynamic_quant_kernels.cuh", "dynamic_quant_ring.cuh", "dq_device.cuh", "tma_pipeline.cuh",
-                      "dq_args.cuh", "quant_launch.cuh", "dq_launch.cuh"),
+                      "ring_prefetch.cuh", "dq_args.cuh", "quant_launch.cuh", "dq_launch.cuh"),
     "ada_layernorm_quant": ("ada_layernorm_quant_kernels.cuh", "ada_layernorm_quant_ring.cuh", "dq_device.cuh",
-                            "tma_pipeline.cuh", "dq_args.cuh", "ada_launch.cu", "dq_launch.cuh"),
+                            "tma_pipeline.cuh", "ring_prefetch.cuh", "dq_args.cuh", "ada_launch.cu", "dq_launch.cuh"),
     "dequant_per_token": ("dequant_kernels.cuh", "dq_device.cuh", "dq_args.cuh", "dequant_launch.cu", "dq_launch.cuh"),
     "dequant_per_group": ("dequant_kernels.cuh", "dq_device.cuh", "dq_args.cuh", "dequant_launch.cu", "dq_launch.cuh"),
     "w8a8_gemm": ("w8a8_gemm.cu", "tma_pipeline.cuh"),
@@ -472,10 +473,11 @@ def run_ours(args, world, rank, local):
     end = torch.cuda.Event(enable_timing=True)
     t0 = time.perf_counter()
     with torch.cuda.stream(L.stream):
-        # the device sleeps ~1 ms before the start event, while the host queues
-        # the K launches: the host's launch latency stays outside the timed
-        # region, which holds exactly the K steps
-        torch.cuda._sleep(PRE_ROLL_CYCLES)
+        # the device sleeps ~1 ms (+ ~10 us per step) before the start event,
+        # while the host queues the K launches: the host's launch latency stays
+        # outside the timed region, which holds exactly the K steps (a 2 us
+        # call would otherwise wait on the host's ~4 us per launch)
+        torch.cuda._sleep(PRE_ROLL_CYCLES + PRE_ROLL_CYCLES_PER_STEP * args.steps)
         start.record(L.stream)
         if graph is not None:
             graph.replay()  # replays on the current stream, i.e. L.stream

@@ -30,6 +30,7 @@
 #include "ada_layernorm_quant_kernels.cuh"
 #include "dq_args.cuh"
 #include "dq_device.cuh"
+#include "ring_prefetch.cuh"
 #include "tma_pipeline.cuh"
 
 namespace dq {
@@ -129,7 +130,13 @@ __global__ void __maxnreg__(DQ_ADA_RING_MAX_REGS) ada_layernorm_quant_ring_kerne
   if (kStaged) {
     // one launch per call: launched as a programmatic dependent of the work
     // before it (x and the parameters may come from it), this kernel folds
-    // the table rows of its batches itself while its first rows are copied
+    // the table rows of its batches itself while its first rows are copied;
+    // those rows are prefetched into L2 before the wait, as in the
+    // DynamicQuant ring kernel
+    if (threadIdx.x == 0) {
+      const int npf = ring_prefetch_rows(row_bytes, NS, n);
+      for (int j = 0; j < npf; ++j) bulk_prefetch_l2(x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes);
+    }
     pdl_launch_dependents();
     pdl_wait_primary();
     if (threadIdx.x == 0) {

