@@ -67,18 +67,18 @@ def test_launch_counts_and_timed_kernels():
     times follow the library's dispatch: the ring kernel for long rows, the
     one-warp kernel for few short rows, one AdaLayerNormQuant launch while the
     CTA's affine table rows fit in 64 KB of shared memory (two otherwise)."""
-    c1 = workloads.make("sym_int8_f16_64x1024")
-    c2 = workloads.make("sym_int8_smooth_bf16_8192x4096")
-    c5 = workloads.make("ada_layernorm_quant_bf16_4x4096x3072")
+    small = workloads.make("sym_int8_f16_64x1024")
+    large = workloads.make("sym_int8_smooth_bf16_8192x4096")
+    ada = workloads.make("ada_layernorm_quant_bf16_4x4096x3072")
     gemm = workloads.make("w8a8_gemm_int8_bf16_4096x4096x4096")
-    assert bench.timed_kernel(c1) == "dynamic_quant_warp_kernel"
-    assert bench.timed_kernel(c2) == "dynamic_quant_ring_kernel"
+    assert bench.timed_kernel(small) == "dynamic_quant_warp_kernel"
+    assert bench.timed_kernel(large) == "dynamic_quant_ring_kernel"
     assert bench.timed_kernel(gemm) == "w8a8_gemm_persistent_kernel"
-    assert bench.timed_kernel(c5).startswith("ada_layernorm_quant_ring_kernel")
-    for wl in (c1, c2, gemm, c5):
+    assert bench.timed_kernel(ada).startswith("ada_layernorm_quant_ring_kernel")
+    for wl in (small, large, gemm, ada):
         assert bench.launches_per_call(wl) == 1
     # 2 batches of 3072 columns per CTA: 48 KB of table rows, folded in the kernel
-    assert bench.ada_table_staged(c5)
+    assert bench.ada_table_staged(ada)
 
     class Wide:  # 2 batches of 8192 columns per CTA: 128 KB, the table kernel runs first
         kind = "ada_layernorm_quant"

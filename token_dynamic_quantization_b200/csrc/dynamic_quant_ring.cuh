@@ -439,7 +439,7 @@ namespace dq {
 
 // ============================================================ small inputs
 
-// Few short rows (c1: 64 rows of 1024 fp16): the ring's per-CTA set-up is not
+// Few short rows (e.g. 64 rows of 1024 fp16): the ring's per-CTA set-up is not
 // amortized, so one warp per row loads its row straight into registers with
 // 16-byte read-only loads (lane l holds vectors l + 32k, k < VPT: coalesced),
 // reduces it with one warp instruction, derives the row constants and stores
@@ -457,6 +457,12 @@ __global__ void __launch_bounds__(kWarpRowThreads) dynamic_quant_warp_kernel(con
   const int lane = threadIdx.x;
   const int nvec = static_cast<int>(a.cols >> 3);
   auto in_row = [&](int k) { return !kRagged || lane + 32 * k < nvec; };
+  // the CTA's first row into L2 while the kernel before finishes (see
+  // ring_prefetch.cuh; 64 x 1024 fp16: 2.15 us against 2.33 us per call)
+  if (lane == 0 && static_cast<int64_t>(blockIdx.x) < a.rows) {
+    bulk_prefetch_l2(static_cast<const uint8_t*>(a.x) + static_cast<int64_t>(blockIdx.x) * a.cols * 2,
+                     static_cast<uint32_t>(a.cols * 2));
+  }
   pdl_launch_dependents();
   pdl_wait_primary();
   write_group_status(a);
