@@ -153,7 +153,8 @@ inline dq_status launch_status() {
 
 // Launch `kernel` as a programmatic dependent of the previous work in
 // `stream`: it may start before that work finishes and waits for it
-// (griddepcontrol.wait) before touching global memory.
+// (griddepcontrol.wait) before it reads or writes global memory (the ring
+// kernels issue only L2 prefetch hints before the wait).
 template <typename Args>
 dq_status launch_programmatic(void (*kernel)(const Args), const Args& a, int grid, int block, size_t smem,
                               cudaStream_t stream) {

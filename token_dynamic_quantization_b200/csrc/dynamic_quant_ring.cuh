@@ -129,7 +129,8 @@ __global__ void __maxnreg__(DQ_RING_MAX_REGS) dynamic_quant_ring_kernel(const Ro
   }
   // launched as a programmatic dependent: the set-up above overlaps the tail
   // of the previous kernel, and so does an L2 prefetch of the CTA's first
-  // rows; every global memory access comes after the wait
+  // rows (a hint: it returns no data); every global load and store comes
+  // after the wait
   const uint8_t* x_cta = static_cast<const uint8_t*>(a.x) + r_begin * static_cast<int64_t>(row_bytes);
   if (threadIdx.x == 0) {
     const int npf = ring_prefetch_rows(row_bytes, NS, n);
