@@ -543,3 +543,24 @@ def test_ada_workload_parity_full_size(dq):
     got = run_ada_gpu(dq, t["x"], t["ada_scale"], t["ada_shift"], t["weight"], t["bias"], t["smooth"], wl.epsilon)
     rel, frac = assert_ada_close(got, want)
     print(f"\nAdaLayerNormQuant full size: max quant_scale rel err {rel:.3g}, code mismatch fraction {frac:.3g}")
+
+
+@pytest.mark.parametrize("pdtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("which", [0, 2])
+def test_ada_misaligned_parameters_fold_the_same_table(dq, pdtype, which):
+    """The ring kernel folds its affine table from 16-byte parameter loads when
+    every parameter is 16-byte aligned, one column at a time otherwise: the
+    same parameters one element past a 16-byte boundary give the same bits."""
+    dev = torch.device("cuda:0")
+    x, sc, sh, w, bias, sm = _ada_inputs(2, 300, 3072, torch.bfloat16, pdtype, seed=77 + which)
+    aligned = run_ada_gpu(dq, x, sc, sh, w, bias, sm, 1e-6)
+    params = [t.to(dev) for t in (sc, sh, w, bias, sm)]
+    buf = torch.empty(params[which].numel() + 1, dtype=pdtype, device=dev)
+    shifted = buf[1:].view(params[which].shape)
+    shifted.copy_(params[which])
+    assert shifted.data_ptr() % 16 != 0
+    params[which] = shifted
+    got = run_ada_gpu(dq, x, *params, 1e-6)
+    np.testing.assert_array_equal(got[0], aligned[0])
+    np.testing.assert_array_equal(got[1].view(np.uint32), aligned[1].view(np.uint32))
+    assert_ada_close(got, oracle.ada_layernorm_quant(x, sc, sh, w, bias, sm, epsilon=1e-6))

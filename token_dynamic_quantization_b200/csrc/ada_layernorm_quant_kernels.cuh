@@ -5,7 +5,7 @@
 //     A[b][c] = (w[c] * (1 + scale[b][c])) * smooth[c]
 //     B[b][c] = ((bias[c] * (1 + scale[b][c])) + shift[b][c]) * smooth[c]
 // (absent weight = 1, bias = 0, smooth = 1), so steps 1-3 become one FMA per
-// element, y = n * A + B (ada_fold, the one evaluation of these formulas).
+// element, y = n * A + B (ada_fold_values, the one evaluation of these formulas).
 //   * The ring kernel (ada_layernorm_quant_ring.cuh) with the table staged in
 //     shared memory folds the table rows of its batches itself: one launch
 //     per call.
@@ -59,16 +59,20 @@ __device__ __forceinline__ float param_at(const void* p, int64_t i) {
     return __bfloat162float(__ldg(static_cast<const __nv_bfloat16*>(p) + i));
   }
 }
+// A, B of one column from its parameter values: the batch's scale and shift,
+// the column's weight, bias and smooth scale (1, 0 and 1 when absent)
+__device__ __forceinline__ void ada_fold_values(float scale, float shift, float w, float bs, float sm, float& A,
+                                                float& B) {
+  const float onep = __fadd_rn(1.0f, scale);
+  A = __fmul_rn(__fmul_rn(w, onep), sm);
+  B = __fmul_rn(__fadd_rn(__fmul_rn(bs, onep), shift), sm);
+}
 template <typename ParamT>
 __device__ __forceinline__ void ada_fold(const AdaArgs& a, int64_t b, int64_t c, float& A, float& B) {
   const int64_t idx = b * a.hidden + c;
-  const float onep = __fadd_rn(1.0f, param_at<ParamT>(a.ada_scale, idx));
-  const float w = a.weight ? param_at<ParamT>(a.weight, c) : 1.0f;
-  const float bs = a.bias ? param_at<ParamT>(a.bias, c) : 0.0f;
-  const float sm = a.smooth ? param_at<ParamT>(a.smooth, c) : 1.0f;
-  const float sh = param_at<ParamT>(a.ada_shift, idx);
-  A = __fmul_rn(__fmul_rn(w, onep), sm);
-  B = __fmul_rn(__fadd_rn(__fmul_rn(bs, onep), sh), sm);
+  ada_fold_values(param_at<ParamT>(a.ada_scale, idx), param_at<ParamT>(a.ada_shift, idx),
+                  a.weight ? param_at<ParamT>(a.weight, c) : 1.0f, a.bias ? param_at<ParamT>(a.bias, c) : 0.0f,
+                  a.smooth ? param_at<ParamT>(a.smooth, c) : 1.0f, A, B);
 }
 
 __global__ void __launch_bounds__(kTableBlock) ada_affine_table_kernel(const AdaArgs a) {

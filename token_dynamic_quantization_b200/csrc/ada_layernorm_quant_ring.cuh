@@ -48,14 +48,59 @@ __host__ __device__ inline size_t ada_ring_smem_bytes(int slots, uint32_t stride
 #define DQ_ADA_RING_MAX_REGS 128
 #endif
 
-// The folded table rows (ada_fold) of batches b_lo .. b_lo + nb - 1 into
-// shared memory, each row as two planes (elements 0-3 and 4-7 of every
+// 8 consecutive parameter values from a 16-byte aligned address, widened to
+// fp32, or `fill` when the parameter is absent.
+template <typename ParamT>
+__device__ __forceinline__ void param8(const void* p, int64_t i, float fill, float (&v)[8]) {
+  if (p == nullptr) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = fill;
+  } else if constexpr (sizeof(ParamT) == 4) {
+    const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+    const float4 lo = __ldg(q), hi = __ldg(q + 1);
+    v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+    v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+  } else {
+    InTraits<ParamT>::widen8(__ldg(reinterpret_cast<const uint4*>(static_cast<const ParamT*>(p) + i)), v);
+  }
+}
+
+// The folded table rows (ada_fold_values) of batches b_lo .. b_lo + nb - 1
+// into shared memory, each row as two planes (elements 0-3 and 4-7 of every
 // 8-column vector), so that 32 lanes reading consecutive vectors read
-// consecutive 16-byte words: no bank conflicts.
+// consecutive 16-byte words: no bank conflicts. This runs at the start of
+// every CTA, before its first row's pass 2: with 16-byte aligned parameters
+// each thread takes 8 columns with one 16-byte load per parameter (4 x 4096
+// x 3072 bf16: 32.8 us per call against 34.0 with one 2-byte load per
+// parameter and column); otherwise one column at a time.
 template <typename ParamT>
 __device__ __forceinline__ void fold_table_rows(const AdaArgs& a, int64_t b_lo, int nb, float* A_s, float* B_s) {
   const int H = static_cast<int>(a.hidden);
-  const int nv = H / 8;
+  const int nv = H / 8;  // the ring kernel's rows are whole 16-byte vectors
+  const uintptr_t any = reinterpret_cast<uintptr_t>(a.ada_scale) | reinterpret_cast<uintptr_t>(a.ada_shift) |
+                        reinterpret_cast<uintptr_t>(a.weight) | reinterpret_cast<uintptr_t>(a.bias) |
+                        reinterpret_cast<uintptr_t>(a.smooth);
+  if ((any & 15u) == 0) {
+    for (int i = threadIdx.x; i < nb * nv; i += blockDim.x) {
+      const int bi = i / nv, vi = i - bi * nv;
+      const int64_t at = (b_lo + bi) * a.hidden + 8 * vi;
+      float sc[8], sh[8], w[8], bs[8], sm[8], A[8], B[8];
+      param8<ParamT>(a.ada_scale, at, 0.0f, sc);
+      param8<ParamT>(a.ada_shift, at, 0.0f, sh);
+      param8<ParamT>(a.weight, 8 * vi, 1.0f, w);
+      param8<ParamT>(a.bias, 8 * vi, 0.0f, bs);
+      param8<ParamT>(a.smooth, 8 * vi, 1.0f, sm);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ada_fold_values(sc[e], sh[e], w[e], bs[e], sm[e], A[e], B[e]);
+      float4* A4 = reinterpret_cast<float4*>(A_s + bi * H);
+      float4* B4 = reinterpret_cast<float4*>(B_s + bi * H);
+      A4[vi] = make_float4(A[0], A[1], A[2], A[3]);
+      A4[nv + vi] = make_float4(A[4], A[5], A[6], A[7]);
+      B4[vi] = make_float4(B[0], B[1], B[2], B[3]);
+      B4[nv + vi] = make_float4(B[4], B[5], B[6], B[7]);
+    }
+    return;
+  }
   for (int bi = 0; bi < nb; ++bi) {
 #pragma unroll 4
     for (int c = threadIdx.x; c < H; c += blockDim.x) {
