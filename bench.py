@@ -10,14 +10,15 @@ headline metric is quoted on). The metric is GB/s of algorithmic HBM traffic
 (x read + codes and scales written + side tables read), with rows/s and the
 fraction of the measured HBM copy bandwidth alongside.
 
-Timing: W untimed warm-up steps, then exactly K steps between a barrier +
-device synchronize on both sides, timed with CUDA events on the launching
-stream; the max over ranks is reported. Consecutive steps rotate over several
-input/output buffer sets whose total is at least 12 x the 126 MB L2, so no step
-reads data an earlier one left in L2 (with 3 x the L2, some lines survived a
-rotation: 8192 x 4096 bf16 ran 0.5 us per call faster and read 6 % less from
-DRAM than it moves); tiny workloads stop at 1024 sets, still above the L2. SM clocks and throttle reasons are sampled through NVML
-during the timed region.
+Timing: one untimed step on each buffer set, W untimed warm-up steps, then
+exactly K steps between a barrier + device synchronize on both sides, timed
+with CUDA events on the launching stream; the max over ranks is reported.
+Consecutive steps rotate over several input/output buffer sets whose total is
+at least 12 x the 126 MB L2, so no step reads data an earlier one left in L2
+(with 3 x the L2, some lines survived a rotation: 8192 x 4096 bf16 ran 0.5 us
+per call faster and read 6 % less from DRAM than it moves); tiny workloads
+stop at 1024 sets, still above the L2. SM clocks and throttle reasons are
+sampled through NVML during the timed region.
 
 Multi-GPU (torchrun, one process per GPU): rows are independent, so each rank
 quantizes its own full batch with no collective on the data path (weak
@@ -462,6 +463,11 @@ def run_ours(args, world, rank, local):
     sampler.start()
     graph = None
     with torch.cuda.stream(L.stream):
+        # every buffer set once, then the W warm-up steps: the first launch on
+        # a set is slower (per-token dequantization over 12 sets: 18.6 us per
+        # call in a 20-step window after 5 warm-up steps, 17.9 after 24)
+        for i in range(sets):
+            L.step(i)
         for i in range(args.warmup):
             L.step(i)
         if args.graph:
@@ -537,6 +543,7 @@ def run_ours(args, world, rank, local):
                 "parallelism": f"dp{world} (independent row batches, no collective)",
                 "l2": f"inputs larger than L2: {sets} rotating buffer sets, {sets * per_set / 1e6:.0f} MB "
                       f"> 126 MB (target {L2_ROTATION} x)",
+                "priming": f"{sets} untimed steps, one per buffer set, before the W warm-up steps",
                 "launch": "cuda graph of K launches" if args.graph else
                           "eager C-ABI launches, queued behind a ~1 ms device sleep (host launch latency untimed)",
             },
