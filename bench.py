@@ -444,6 +444,12 @@ class Launcher:
             raise RuntimeError(f"launch failed: {self.dq.dq_status_string(st)}")
 
 
+def rotation_sets(per_set: int) -> int:
+    """Buffer sets the timed steps rotate over: at least L2_ROTATION L2
+    capacities in all (two sets at least, MAX_SETS at most)."""
+    return min(MAX_SETS, max(2, math.ceil(L2_ROTATION * L2_BYTES / per_set)))
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -455,7 +461,7 @@ def run_ours(args, world, rank, local):
     wl = workloads.make(args.workload, rows=args.rows)
     nbytes = algorithmic_bytes(wl)
     per_set = wl.primary.numel() * wl.primary.element_size() + nbytes
-    sets = min(MAX_SETS, max(2, math.ceil(L2_ROTATION * L2_BYTES / per_set)))
+    sets = rotation_sets(per_set)
     L = Launcher(dq, wl, device, sets)
     torch.cuda.synchronize(device)
 

@@ -86,3 +86,17 @@ def test_launch_counts_and_timed_kernels():
 
     assert not bench.ada_table_staged(Wide)
     assert bench.launches_per_call(Wide) == 2
+
+
+def test_rotation_sets_cover_twelve_l2_capacities():
+    """The timed steps rotate over buffer sets of at least 12 x the L2 (input
+    lines survived a rotation of 3 x), at least two sets, at most 1024."""
+    l2 = bench.L2_BYTES
+    for per_set in (168_000_000, 250_000_000, 83_000_000, 1_180_000_000, 3 * l2):
+        sets = bench.rotation_sets(per_set)
+        assert sets >= 2
+        assert sets * per_set >= 12 * l2 or sets == 2
+    assert bench.rotation_sets(1_180_000_000) == 2
+    assert bench.rotation_sets(168_000_000) == 10
+    assert bench.rotation_sets(330_000) == bench.MAX_SETS == 1024
+    assert bench.MAX_SETS * 330_000 > l2
